@@ -1,0 +1,183 @@
+/*
+ * dca.h -- C ABI of the B200 (sm_100a) Dual Chunk Attention prefill library.
+ *
+ * Dual Chunk Attention (DCA) is causal grouped-query attention whose RoPE
+ * positions are remapped per (query i, key j) pair so that every relative
+ * distance stays below the pretraining window c.  With chunk size s, local
+ * window w, n_x = x / s and r_x = x mod s (chunks start at token 0):
+ *   key position   Pk(j)   = j mod s                     (periodic key index)
+ *   query position Pq(i,j) = r_i        if n_i == n_j    (intra-chunk)
+ *                          = s + r_i    if n_i - n_j == 1 and r_i < w
+ *                                                         (successive chunk, local window)
+ *                          = c - 1      otherwise         (inter-chunk: fixed large index)
+ *   logit = m^2 / sqrt(d) * < R(Pq) q_i, R(Pk) k_j >, R(p) = RoPE rotation of the
+ *   pairs (x_k, x_{k+d/2}) by p * base^(-2k/d); m = 1 for yarn_scale <= 1, else
+ *   0.1 ln(yarn_scale) + 1 (YaRN attention temperature).
+ *   out_i = sum_{j <= i} softmax_j(logit) v_j;  query head h reads KV head h / (Hq/Hkv).
+ * Sources: "Qwen2.5-1M 不重训外推 1M" (mizuki-eaf.pages.dev), sections 核心思想,
+ * Intra-Chunk / Successive-Chunk / Inter-Chunk Attention, "DCA + YaRN",
+ * "Chunked Prefill"; news article on the Qwen2.5-1M release (7a8v.yksolo.com),
+ * section 如何炼成的？ (RoPE base 10,000,000).  The window test r_i < w is one
+ * reading of the Successive-Chunk section (the pages do not fix it).
+ *
+ * Conventions for every entry point
+ *   - Tensors are contiguous row-major: q, out [L][Hq][d]; k, v [L][Hkv][d].
+ *   - Device pointers must be 16-byte aligned; the workspace 256-byte aligned.
+ *   - The caller owns every buffer; the library never allocates or frees
+ *     device memory and never synchronises, except dca_device_status().
+ *   - Work is enqueued on `cuda_stream` (a cudaStream_t; NULL = legacy default
+ *     stream) of the current device and returns immediately.
+ *   - Errors are return codes (dca_status); nothing is thrown across the ABI.
+ *     Argument errors are detected on the host before any launch.
+ *   - d must be 128.  dtype DCA_BF16 runs the tcgen05/TMA tensor-core kernel
+ *     (bf16 in, fp32 accumulate, bf16 out); DCA_F32 runs an fp32 CUDA-core
+ *     kernel (fp32 in/out).
+ *   - Parameter domain: Hq % Hkv == 0, chunk_size >= 1,
+ *     0 <= local_window <= chunk_size, pretrain_window >= 1, and
+ *     chunk_size + local_window <= pretrain_window whenever the key length
+ *     exceeds chunk_size (so every remapped distance stays below
+ *     pretrain_window).  rope_base > 0, yarn_scale > 0.
+ */
+#ifndef DCA_B200_H
+#define DCA_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum { DCA_BF16 = 0, DCA_F32 = 1 } dca_dtype;
+
+typedef enum {
+  DCA_OK = 0,
+  DCA_ERR_ARG = -1,         /* bad size, pointer, alignment or parameter       */
+  DCA_ERR_UNSUPPORTED = -2, /* valid but not implemented (e.g. d != 128)       */
+  DCA_ERR_CUDA = -3,        /* a CUDA runtime/driver call failed               */
+  DCA_ERR_WORKSPACE = -4,   /* workspace missing, misaligned or too small      */
+  DCA_ERR_TIMEOUT = -5      /* a kernel gave up on a bounded wait (device status) */
+} dca_status;
+
+/* Library version (major*10000 + minor*100 + patch). */
+int dca_version(void);
+
+/* Human-readable name of a dca_status value (static string, never NULL). */
+const char* dca_status_string(int status);
+
+/*
+ * Workspace bytes needed for key lengths up to `kv_capacity` with these
+ * parameters.  Returns 0 when the arguments are invalid.  The workspace holds
+ * a status header, a RoPE cos/sin table computed in float64 and stored fp32,
+ * and the keys rotated to their periodic positions (R(j mod s) k_j).  Its
+ * layout depends only on (kv_capacity, Hkv, d, chunk sizes, dtype), so one
+ * workspace can be reused across the calls of a chunked prefill.
+ */
+size_t dca_workspace_size(int64_t kv_capacity, int Hq, int Hkv, int d, int64_t chunk_size,
+                          int64_t local_window, int64_t pretrain_window, int dtype);
+
+/* Zero the workspace status header (call once after allocating it). */
+int dca_workspace_init(void* workspace, size_t ws_bytes, void* cuda_stream);
+
+/*
+ * One-shot DCA prefill: q [L][Hq][d], k, v [L][Hkv][d] -> out [L][Hq][d].
+ * Equivalent to dca_prefill_chunked(q, k, v, out, 0, L, L, ...).
+ */
+int dca_prefill(const void* q, const void* k, const void* v, void* out, int64_t L, int Hq,
+                int Hkv, int d, int64_t chunk_size, int64_t local_window,
+                int64_t pretrain_window, double rope_base, double yarn_scale, int dtype,
+                void* workspace, size_t ws_bytes, void* cuda_stream);
+
+/*
+ * Chunked prefill ("Chunked Prefill" section: the input is processed in query
+ * blocks that attend to the growing KV cache).  Query block row t has absolute
+ * position q_start + t and attends cache rows j <= q_start + t.
+ *   q_block, out_block [Lq][Hq][d];  k_cache, v_cache [Lk][Hkv][d] holding
+ *   UNROTATED keys.  Requires q_start >= 0, Lq >= 0, q_start + Lq <= Lk.
+ * The result equals rows [q_start, q_start + Lq) of the one-shot call.
+ * Stateless: rotates all Lk keys into the workspace, then attends
+ * (= dca_prepare(..., k_rows_valid = 0) followed by dca_attend).
+ */
+int dca_prefill_chunked(const void* q_block, const void* k_cache, const void* v_cache,
+                        void* out_block, int64_t q_start, int64_t Lq, int64_t Lk, int Hq,
+                        int Hkv, int d, int64_t chunk_size, int64_t local_window,
+                        int64_t pretrain_window, double rope_base, double yarn_scale,
+                        int dtype, void* workspace, size_t ws_bytes, void* cuda_stream);
+
+/*
+ * Stage 1 of a prefill call: build the RoPE table and rotate keys
+ * [k_rows_valid, Lk) of k_cache into the workspace.  k_rows_valid = 0 rebuilds
+ * everything; k_rows_valid > 0 promises that the table and rotated rows
+ * [0, k_rows_valid) already in this workspace were produced by earlier calls
+ * with identical parameters and workspace size (an engine appending one block
+ * of keys per call passes the previous Lk).
+ */
+int dca_prepare(const void* k_cache, int64_t Lk, int64_t k_rows_valid, int Hkv, int d,
+                int64_t chunk_size, int64_t local_window, int64_t pretrain_window,
+                double rope_base, int dtype, void* workspace, size_t ws_bytes,
+                void* cuda_stream);
+
+/*
+ * Stage 2: the fused DCA attention kernel over a query block, reading the
+ * rotated keys from the workspace (prepared for at least Lk rows) and v_cache.
+ * Arguments as for dca_prefill_chunked (rope_base is fixed by dca_prepare).
+ */
+int dca_attend(const void* q_block, const void* v_cache, void* out_block, int64_t q_start,
+               int64_t Lq, int64_t Lk, int Hq, int Hkv, int d, int64_t chunk_size,
+               int64_t local_window, int64_t pretrain_window, double yarn_scale, int dtype,
+               void* workspace, size_t ws_bytes, void* cuda_stream);
+
+/*
+ * Device-side status: synchronises `cuda_stream`, reads and clears the status
+ * word that kernels set when a bounded wait gave up.  Returns DCA_OK,
+ * DCA_ERR_TIMEOUT or DCA_ERR_CUDA.
+ */
+int dca_device_status(void* workspace, void* cuda_stream);
+
+/*
+ * Host-buffer entry point: whole prefill of L tokens from HOST memory.
+ * q_h, out_h [L][Hq][d]; k_h, v_h [L][Hkv][d] in host memory (pinned memory
+ * gives full copy bandwidth).  The input is processed in query blocks of
+ * `block` rows (block <= 0: one block): per block the library copies the
+ * block's q, k and v rows host->device, appends the keys to the rotated-key
+ * cache, runs the attention kernel and copies the block's output rows back.
+ * All device memory comes from the caller's `arena` (dca_host_arena_size bytes,
+ * 256-byte aligned).  Returns after enqueuing; call dca_device_status or
+ * synchronise the stream before reading out_h.
+ */
+size_t dca_host_arena_size(int64_t L, int64_t block, int Hq, int Hkv, int d,
+                           int64_t chunk_size, int64_t local_window, int64_t pretrain_window,
+                           int dtype);
+int dca_prefill_host(const void* q_h, const void* k_h, const void* v_h, void* out_h, int64_t L,
+                     int64_t block, int Hq, int Hkv, int d, int64_t chunk_size,
+                     int64_t local_window, int64_t pretrain_window, double rope_base,
+                     double yarn_scale, int dtype, void* arena, size_t arena_bytes,
+                     void* cuda_stream);
+
+/*
+ * Host-side introspection of the tile plan the attention kernels follow
+ * (no GPU needed).  For the query tile whose rows are [i0, i0 + tile_rows)
+ * with real rows up to i_last, and key tiles of `bn` keys, writes up to
+ * `max_items` triples (k_tile, class, full) in work-list order: class 2 =
+ * inter-chunk, 1 = successive chunk, 0 = intra-chunk (the three parts of the
+ * score matrix in section 核心思想 of "Qwen2.5-1M 不重训外推 1M"); full = 1
+ * when every pair of the tile is causal and of that class (no mask).
+ * Returns the number of items (which may exceed max_items) or DCA_ERR_ARG.
+ */
+int dca_plan_items(int64_t i0, int64_t i_last, int64_t tile_rows, int64_t chunk_size, int bn,
+                   int32_t* items, int max_items);
+
+/*
+ * Test hooks.  dca_set_wait_timeout_ns sets the limit of every bounded device
+ * wait (default 10 s).  dca_set_debug_flags(1) makes the next attention launch
+ * withhold its first key-tile load, so that its waits run out and the kernel
+ * returns through the timeout path (status word set, DCA_ERR_TIMEOUT from
+ * dca_device_status); flags reset to 0 after that launch.
+ */
+void dca_set_wait_timeout_ns(int64_t ns);
+void dca_set_debug_flags(int flags);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* DCA_B200_H */

@@ -1,0 +1,162 @@
+"""Python API over the C ABI of the DCA prefill library.
+
+Argument marshalling only: torch provides device memory and the current CUDA
+stream; every step of the computation runs in the library's kernels.
+"""
+from __future__ import annotations
+
+from typing import Optional
+
+import torch
+
+from . import _native as N
+
+_DTYPES = {torch.bfloat16: N.DCA_BF16, torch.float32: N.DCA_F32}
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype not in _DTYPES:
+        raise TypeError(f"unsupported dtype {t.dtype} (bfloat16 or float32)")
+    return _DTYPES[t.dtype]
+
+
+def _check_cuda(*ts):
+    for t in ts:
+        if not t.is_cuda:
+            raise ValueError("tensors must be CUDA tensors (the library has no CPU path)")
+        if not t.is_contiguous():
+            raise ValueError("tensors must be contiguous")
+
+
+def _stream_ptr(device) -> int:
+    return torch.cuda.current_stream(device).cuda_stream
+
+
+def workspace_size(kv_capacity, Hq, Hkv, d, chunk_size, local_window, pretrain_window,
+                   dtype) -> int:
+    code = _DTYPES[dtype] if isinstance(dtype, torch.dtype) else int(dtype)
+    n = N.lib().dca_workspace_size(int(kv_capacity), int(Hq), int(Hkv), int(d), int(chunk_size),
+                                   int(local_window), int(pretrain_window), code)
+    if n == 0:
+        raise N.DCAError(N.DCA_ERR_ARG, "dca_workspace_size")
+    return n
+
+
+class Workspace:
+    """Caller-owned device workspace (RoPE table, rotated keys, status word).
+
+    One workspace serves every call whose key length is <= its capacity and
+    whose (Hkv, d, chunk_size, local_window, dtype) match.
+    """
+
+    def __init__(self, kv_capacity, Hq, Hkv, d, chunk_size, local_window, pretrain_window,
+                 dtype, device="cuda"):
+        self.nbytes = workspace_size(kv_capacity, Hq, Hkv, d, chunk_size, local_window,
+                                     pretrain_window, dtype)
+        self.buf = torch.empty(self.nbytes, dtype=torch.uint8, device=device)
+        self.device = self.buf.device
+        N.check(N.lib().dca_workspace_init(self.buf.data_ptr(), self.nbytes,
+                                           _stream_ptr(self.device)), "dca_workspace_init")
+
+    @property
+    def ptr(self) -> int:
+        return self.buf.data_ptr()
+
+    def status(self) -> int:
+        """Synchronise the current stream and read/clear the device status word."""
+        return N.lib().dca_device_status(self.ptr, _stream_ptr(self.device))
+
+
+def _ws_for(ws: Optional[Workspace], Lk, Hq, Hkv, d, p, dtype, device) -> Workspace:
+    if ws is not None:
+        return ws
+    return Workspace(Lk, Hq, Hkv, d, p["chunk_size"], p["local_window"], p["pretrain_window"],
+                     dtype, device)
+
+
+def prefill(q, k, v, *, chunk_size, local_window, pretrain_window, rope_base=1e7,
+            yarn_scale=1.0, out=None, workspace: Optional[Workspace] = None):
+    """One-shot DCA prefill.  q [L,Hq,d], k, v [L,Hkv,d] (CUDA, bf16 or fp32)."""
+    return prefill_chunked(q, k, v, q_start=0, chunk_size=chunk_size, local_window=local_window,
+                           pretrain_window=pretrain_window, rope_base=rope_base,
+                           yarn_scale=yarn_scale, out=out, workspace=workspace)
+
+
+def prefill_chunked(q_block, k_cache, v_cache, *, q_start, chunk_size, local_window,
+                    pretrain_window, rope_base=1e7, yarn_scale=1.0, kv_len=None, out=None,
+                    workspace: Optional[Workspace] = None):
+    """A query block (absolute rows q_start ..) against the KV cache rows [0, kv_len)."""
+    _check_cuda(q_block, k_cache, v_cache)
+    Lq, Hq, d = q_block.shape
+    Lk = k_cache.shape[0] if kv_len is None else int(kv_len)
+    Hkv = k_cache.shape[1]
+    dt = _dtype_code(q_block)
+    if not (k_cache.dtype == v_cache.dtype == q_block.dtype):
+        raise TypeError("q, k, v must share a dtype")
+    if out is None:
+        out = torch.empty_like(q_block)
+    p = dict(chunk_size=chunk_size, local_window=local_window, pretrain_window=pretrain_window)
+    ws = _ws_for(workspace, Lk, Hq, Hkv, d, p, q_block.dtype, q_block.device)
+    rc = N.lib().dca_prefill_chunked(
+        q_block.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(), out.data_ptr(), int(q_start),
+        Lq, Lk, Hq, Hkv, d, int(chunk_size), int(local_window), int(pretrain_window),
+        float(rope_base), float(yarn_scale), dt, ws.ptr, ws.nbytes, _stream_ptr(q_block.device))
+    N.check(rc, "dca_prefill_chunked")
+    return out
+
+
+def prepare(k_cache, *, kv_len, k_rows_valid, chunk_size, local_window, pretrain_window,
+            rope_base, workspace: Workspace):
+    """Stage 1: RoPE table (when k_rows_valid == 0) and rotated keys [k_rows_valid, kv_len)."""
+    _check_cuda(k_cache)
+    rc = N.lib().dca_prepare(k_cache.data_ptr(), int(kv_len), int(k_rows_valid), k_cache.shape[1],
+                             k_cache.shape[2], int(chunk_size), int(local_window),
+                             int(pretrain_window), float(rope_base), _dtype_code(k_cache),
+                             workspace.ptr, workspace.nbytes, _stream_ptr(k_cache.device))
+    N.check(rc, "dca_prepare")
+
+
+def attend(q_block, v_cache, out, *, q_start, kv_len, chunk_size, local_window, pretrain_window,
+           yarn_scale, workspace: Workspace):
+    """Stage 2: the fused attention kernel over one query block."""
+    _check_cuda(q_block, v_cache, out)
+    Lq, Hq, d = q_block.shape
+    rc = N.lib().dca_attend(q_block.data_ptr(), v_cache.data_ptr(), out.data_ptr(), int(q_start),
+                            Lq, int(kv_len), Hq, v_cache.shape[1], d, int(chunk_size),
+                            int(local_window), int(pretrain_window), float(yarn_scale),
+                            _dtype_code(q_block), workspace.ptr, workspace.nbytes,
+                            _stream_ptr(q_block.device))
+    N.check(rc, "dca_attend")
+
+
+def host_arena_size(L, block, Hq, Hkv, d, chunk_size, local_window, pretrain_window, dtype):
+    code = _DTYPES[dtype] if isinstance(dtype, torch.dtype) else int(dtype)
+    n = N.lib().dca_host_arena_size(int(L), int(block), int(Hq), int(Hkv), int(d),
+                                    int(chunk_size), int(local_window), int(pretrain_window), code)
+    if n == 0:
+        raise N.DCAError(N.DCA_ERR_ARG, "dca_host_arena_size")
+    return n
+
+
+def prefill_host(q_h, k_h, v_h, out_h, *, block, chunk_size, local_window, pretrain_window,
+                 rope_base=1e7, yarn_scale=1.0, arena: torch.Tensor, stream=None):
+    """Whole prefill from host (CPU, ideally pinned) tensors through the C ABI."""
+    for t in (q_h, k_h, v_h, out_h):
+        if t.is_cuda or not t.is_contiguous():
+            raise ValueError("host tensors must be contiguous CPU tensors")
+    L, Hq, d = q_h.shape
+    Hkv = k_h.shape[1]
+    st = (stream or torch.cuda.current_stream(arena.device)).cuda_stream
+    rc = N.lib().dca_prefill_host(q_h.data_ptr(), k_h.data_ptr(), v_h.data_ptr(), out_h.data_ptr(),
+                                  L, int(block), Hq, Hkv, d, int(chunk_size), int(local_window),
+                                  int(pretrain_window), float(rope_base), float(yarn_scale),
+                                  _dtype_code(q_h), arena.data_ptr(), arena.numel(), st)
+    N.check(rc, "dca_prefill_host")
+
+
+def set_wait_timeout_ns(ns: int):
+    N.lib().dca_set_wait_timeout_ns(int(ns))
+
+
+def set_debug_flags(flags: int):
+    N.lib().dca_set_debug_flags(int(flags))

@@ -1,0 +1,328 @@
+// dca_api.cu -- the library's C ABI (declared in include/dca.h): argument
+// validation on the host, workspace layout, and the launches of the
+// preparation and attention kernels on the caller's stream.
+#include <cuda_runtime.h>
+#include <math.h>
+#include <stdint.h>
+
+#include <atomic>
+
+#include "../../include/dca.h"
+#include "dca_internal.h"
+#include "dca_plan.cuh"
+
+namespace {
+
+constexpr size_t HDR_BYTES = 1024;  // status word + padding
+constexpr int VERSION = 100;        // 0.1.0
+
+std::atomic<long long> g_timeout_ns{10LL * 1000 * 1000 * 1000};
+std::atomic<int> g_debug_flags{0};
+
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+struct Layout {
+  int64_t cap = 0;       // key capacity
+  int64_t T = 0;         // RoPE table rows
+  int64_t n_direct = 0;  // table rows indexed by position
+  size_t tab_off = 0, kr_off = 0, total = 0;
+};
+
+bool basic_params_ok(int Hq, int Hkv, int d, int64_t s, int64_t w, int64_t c, int dtype) {
+  if (Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0) return false;
+  if (d <= 0 || d % 2 != 0) return false;
+  if (s < 1 || w < 0 || w > s || c < 1) return false;
+  if (dtype != DCA_BF16 && dtype != DCA_F32) return false;
+  return true;
+}
+
+Layout make_layout(int64_t cap, int Hkv, int d, int64_t s, int64_t w, int dtype) {
+  Layout L;
+  L.cap = cap;
+  L.T = dca::table_rows(cap, s, w);
+  L.n_direct = L.T - 1;
+  const size_t esize = dtype == DCA_BF16 ? 2 : 4;
+  L.tab_off = HDR_BYTES;
+  L.kr_off = align_up(L.tab_off + static_cast<size_t>(L.T) * (d / 2) * sizeof(float2), 1024);
+  L.total = L.kr_off + align_up(static_cast<size_t>(cap) * Hkv * d * esize, 1024);
+  return L;
+}
+
+// Largest key capacity whose layout fits in ws_bytes (layout size grows with cap).
+int64_t capacity_for(size_t ws_bytes, int Hkv, int d, int64_t s, int64_t w, int dtype) {
+  int64_t lo = 0, hi = (1LL << 31) - 1;
+  if (make_layout(0, Hkv, d, s, w, dtype).total > ws_bytes) return -1;
+  while (lo < hi) {
+    const int64_t mid = lo + (hi - lo + 1) / 2;
+    if (make_layout(mid, Hkv, d, s, w, dtype).total <= ws_bytes)
+      lo = mid;
+    else
+      hi = mid - 1;
+  }
+  return lo;
+}
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+// Checks shared by every compute entry point; returns a dca_status.
+int check_common(int64_t q_start, int64_t Lq, int64_t Lk, int Hq, int Hkv, int d, int64_t s,
+                 int64_t w, int64_t c, double yarn_scale, int dtype, const void* ws,
+                 size_t ws_bytes, Layout* layout) {
+  if (!basic_params_ok(Hq, Hkv, d, s, w, c, dtype)) return DCA_ERR_ARG;
+  if (q_start < 0 || Lq < 0 || Lk < 0 || q_start + Lq > Lk) return DCA_ERR_ARG;
+  if (Lk > (1LL << 31) - 1) return DCA_ERR_ARG;
+  if (Lk > s && s + w > c) return DCA_ERR_ARG;
+  if (!(yarn_scale > 0.0) || !isfinite(yarn_scale)) return DCA_ERR_ARG;
+  if (d != 128) return DCA_ERR_UNSUPPORTED;
+  if (ws == nullptr || !aligned(ws, 256)) return DCA_ERR_WORKSPACE;
+  const int64_t cap = capacity_for(ws_bytes, Hkv, d, s, w, dtype);
+  if (cap < Lk) return DCA_ERR_WORKSPACE;
+  *layout = make_layout(cap, Hkv, d, s, w, dtype);
+  return DCA_OK;
+}
+
+float logit_scale_log2(double yarn_scale, int d) {
+  const double m = yarn_scale <= 1.0 ? 1.0 : 0.1 * log(yarn_scale) + 1.0;
+  return static_cast<float>(m * m / sqrt(static_cast<double>(d)) * 1.4426950408889634);
+}
+
+int prepare_impl(const void* k_cache, int64_t Lk, int64_t k_rows_valid, int Hkv, int d,
+                 int64_t s, int64_t w, int64_t c, double rope_base, int dtype, void* ws,
+                 const Layout& L, cudaStream_t st) {
+  uint8_t* base = static_cast<uint8_t*>(ws);
+  float2* tab = reinterpret_cast<float2*>(base + L.tab_off);
+  cudaError_t e = cudaSuccess;
+  if (k_rows_valid == 0) e = dca::launch_rope_table(tab, L.T, L.n_direct, c, rope_base, d, st);
+  if (e == cudaSuccess)
+    e = dca::launch_rotate_keys(k_cache, base + L.kr_off, tab, k_rows_valid, Lk, Hkv, s, dtype,
+                                st);
+  return e == cudaSuccess ? DCA_OK : DCA_ERR_CUDA;
+}
+
+int attend_impl(const void* q, const void* v, void* out, int64_t q_start, int64_t Lq, int64_t Lk,
+                int Hq, int Hkv, int d, int64_t s, int64_t w, double yarn_scale, int dtype,
+                void* ws, const Layout& L, cudaStream_t st) {
+  if (Lq == 0) return DCA_OK;
+  uint8_t* base = static_cast<uint8_t*>(ws);
+  dca::AttnArgs a;
+  a.q = q;
+  a.kr = base + L.kr_off;
+  a.v = v;
+  a.out = out;
+  a.tab = reinterpret_cast<const float2*>(base + L.tab_off);
+  a.q_start = q_start;
+  a.Lq = Lq;
+  a.Lk = Lk;
+  a.s = s;
+  a.w = w;
+  a.tab_c1 = L.T - 1;
+  a.Hq = Hq;
+  a.Hkv = Hkv;
+  a.scale_log2 = logit_scale_log2(yarn_scale, d);
+  a.status = reinterpret_cast<unsigned int*>(base);
+  a.timeout_ns = static_cast<unsigned long long>(g_timeout_ns.load());
+  a.debug = g_debug_flags.exchange(0);
+  cudaError_t e = dtype == DCA_BF16 ? dca::launch_attention_sm100(a, st)
+                                    : dca::launch_attention_f32(a, st);
+  return e == cudaSuccess ? DCA_OK : DCA_ERR_CUDA;
+}
+
+bool ptrs_ok(const void* p) { return p != nullptr && aligned(p, 16); }
+
+}  // namespace
+
+extern "C" {
+
+int dca_version(void) { return VERSION; }
+
+const char* dca_status_string(int status) {
+  switch (status) {
+    case DCA_OK: return "DCA_OK";
+    case DCA_ERR_ARG: return "DCA_ERR_ARG: invalid size, pointer, alignment or parameter";
+    case DCA_ERR_UNSUPPORTED: return "DCA_ERR_UNSUPPORTED: head dim must be 128";
+    case DCA_ERR_CUDA: return "DCA_ERR_CUDA: a CUDA call failed";
+    case DCA_ERR_WORKSPACE: return "DCA_ERR_WORKSPACE: workspace missing, misaligned or too small";
+    case DCA_ERR_TIMEOUT: return "DCA_ERR_TIMEOUT: a kernel gave up on a bounded wait";
+    default: return "unknown dca status";
+  }
+}
+
+size_t dca_workspace_size(int64_t kv_capacity, int Hq, int Hkv, int d, int64_t chunk_size,
+                          int64_t local_window, int64_t pretrain_window, int dtype) {
+  if (!basic_params_ok(Hq, Hkv, d, chunk_size, local_window, pretrain_window, dtype)) return 0;
+  if (kv_capacity < 0 || kv_capacity > (1LL << 31) - 1) return 0;
+  return make_layout(kv_capacity, Hkv, d, chunk_size, local_window, dtype).total;
+}
+
+int dca_workspace_init(void* workspace, size_t ws_bytes, void* cuda_stream) {
+  if (workspace == nullptr || ws_bytes < HDR_BYTES || !aligned(workspace, 256))
+    return DCA_ERR_WORKSPACE;
+  return cudaMemsetAsync(workspace, 0, HDR_BYTES, static_cast<cudaStream_t>(cuda_stream)) ==
+                 cudaSuccess
+             ? DCA_OK
+             : DCA_ERR_CUDA;
+}
+
+int dca_prepare(const void* k_cache, int64_t Lk, int64_t k_rows_valid, int Hkv, int d,
+                int64_t chunk_size, int64_t local_window, int64_t pretrain_window,
+                double rope_base, int dtype, void* workspace, size_t ws_bytes,
+                void* cuda_stream) {
+  Layout L;
+  int rc = check_common(0, 0, Lk, Hkv, Hkv, d, chunk_size, local_window, pretrain_window, 1.0,
+                        dtype, workspace, ws_bytes, &L);
+  if (rc != DCA_OK) return rc;
+  if (!(rope_base > 0.0) || !isfinite(rope_base)) return DCA_ERR_ARG;
+  if (k_rows_valid < 0 || k_rows_valid > Lk) return DCA_ERR_ARG;
+  if (Lk > k_rows_valid && !ptrs_ok(k_cache)) return DCA_ERR_ARG;
+  return prepare_impl(k_cache, Lk, k_rows_valid, Hkv, d, chunk_size, local_window,
+                      pretrain_window, rope_base, dtype, workspace, L,
+                      static_cast<cudaStream_t>(cuda_stream));
+}
+
+int dca_attend(const void* q_block, const void* v_cache, void* out_block, int64_t q_start,
+               int64_t Lq, int64_t Lk, int Hq, int Hkv, int d, int64_t chunk_size,
+               int64_t local_window, int64_t pretrain_window, double yarn_scale, int dtype,
+               void* workspace, size_t ws_bytes, void* cuda_stream) {
+  Layout L;
+  int rc = check_common(q_start, Lq, Lk, Hq, Hkv, d, chunk_size, local_window, pretrain_window,
+                        yarn_scale, dtype, workspace, ws_bytes, &L);
+  if (rc != DCA_OK) return rc;
+  if (Lq > 0 && (!ptrs_ok(q_block) || !ptrs_ok(v_cache) || !ptrs_ok(out_block)))
+    return DCA_ERR_ARG;
+  return attend_impl(q_block, v_cache, out_block, q_start, Lq, Lk, Hq, Hkv, d, chunk_size,
+                     local_window, yarn_scale, dtype, workspace, L,
+                     static_cast<cudaStream_t>(cuda_stream));
+}
+
+int dca_prefill_chunked(const void* q_block, const void* k_cache, const void* v_cache,
+                        void* out_block, int64_t q_start, int64_t Lq, int64_t Lk, int Hq,
+                        int Hkv, int d, int64_t chunk_size, int64_t local_window,
+                        int64_t pretrain_window, double rope_base, double yarn_scale,
+                        int dtype, void* workspace, size_t ws_bytes, void* cuda_stream) {
+  Layout L;
+  int rc = check_common(q_start, Lq, Lk, Hq, Hkv, d, chunk_size, local_window, pretrain_window,
+                        yarn_scale, dtype, workspace, ws_bytes, &L);
+  if (rc != DCA_OK) return rc;
+  if (!(rope_base > 0.0) || !isfinite(rope_base)) return DCA_ERR_ARG;
+  if (Lq == 0) return DCA_OK;
+  if (!ptrs_ok(q_block) || !ptrs_ok(k_cache) || !ptrs_ok(v_cache) || !ptrs_ok(out_block))
+    return DCA_ERR_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
+  rc = prepare_impl(k_cache, Lk, 0, Hkv, d, chunk_size, local_window, pretrain_window, rope_base,
+                    dtype, workspace, L, st);
+  if (rc != DCA_OK) return rc;
+  return attend_impl(q_block, v_cache, out_block, q_start, Lq, Lk, Hq, Hkv, d, chunk_size,
+                     local_window, yarn_scale, dtype, workspace, L, st);
+}
+
+int dca_prefill(const void* q, const void* k, const void* v, void* out, int64_t L, int Hq,
+                int Hkv, int d, int64_t chunk_size, int64_t local_window,
+                int64_t pretrain_window, double rope_base, double yarn_scale, int dtype,
+                void* workspace, size_t ws_bytes, void* cuda_stream) {
+  return dca_prefill_chunked(q, k, v, out, 0, L, L, Hq, Hkv, d, chunk_size, local_window,
+                             pretrain_window, rope_base, yarn_scale, dtype, workspace, ws_bytes,
+                             cuda_stream);
+}
+
+int dca_device_status(void* workspace, void* cuda_stream) {
+  if (workspace == nullptr) return DCA_ERR_WORKSPACE;
+  cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
+  if (cudaStreamSynchronize(st) != cudaSuccess) return DCA_ERR_CUDA;
+  unsigned int word = 0;
+  if (cudaMemcpy(&word, workspace, sizeof word, cudaMemcpyDeviceToHost) != cudaSuccess)
+    return DCA_ERR_CUDA;
+  if (word != 0) {
+    if (cudaMemset(workspace, 0, sizeof word) != cudaSuccess) return DCA_ERR_CUDA;
+    return DCA_ERR_TIMEOUT;
+  }
+  return DCA_OK;
+}
+
+size_t dca_host_arena_size(int64_t L, int64_t block, int Hq, int Hkv, int d, int64_t chunk_size,
+                           int64_t local_window, int64_t pretrain_window, int dtype) {
+  const size_t ws = dca_workspace_size(L, Hq, Hkv, d, chunk_size, local_window, pretrain_window,
+                                       dtype);
+  if (ws == 0 || L < 0) return 0;
+  const int64_t blk = (block <= 0 || block > L) ? L : block;
+  const size_t esize = dtype == DCA_BF16 ? 2 : 4;
+  const size_t kv = align_up(static_cast<size_t>(L) * Hkv * d * esize, 1024);
+  const size_t qo = align_up(static_cast<size_t>(blk) * Hq * d * esize, 1024);
+  return align_up(ws, 1024) + 2 * kv + 2 * qo;
+}
+
+int dca_prefill_host(const void* q_h, const void* k_h, const void* v_h, void* out_h, int64_t L,
+                     int64_t block, int Hq, int Hkv, int d, int64_t chunk_size,
+                     int64_t local_window, int64_t pretrain_window, double rope_base,
+                     double yarn_scale, int dtype, void* arena, size_t arena_bytes,
+                     void* cuda_stream) {
+  if (q_h == nullptr || k_h == nullptr || v_h == nullptr || out_h == nullptr) return DCA_ERR_ARG;
+  const size_t need = dca_host_arena_size(L, block, Hq, Hkv, d, chunk_size, local_window,
+                                          pretrain_window, dtype);
+  if (need == 0) return DCA_ERR_ARG;
+  if (arena == nullptr || !aligned(arena, 256) || arena_bytes < need) return DCA_ERR_WORKSPACE;
+  if (L == 0) return DCA_OK;
+  const int64_t blk = (block <= 0 || block > L) ? L : block;
+  const size_t esize = dtype == DCA_BF16 ? 2 : 4;
+  const size_t ws_bytes =
+      dca_workspace_size(L, Hq, Hkv, d, chunk_size, local_window, pretrain_window, dtype);
+  const size_t kv = align_up(static_cast<size_t>(L) * Hkv * d * esize, 1024);
+  const size_t qo = align_up(static_cast<size_t>(blk) * Hq * d * esize, 1024);
+  uint8_t* base = static_cast<uint8_t*>(arena);
+  uint8_t* ws = base;
+  uint8_t* kc = base + align_up(ws_bytes, 1024);
+  uint8_t* vc = kc + kv;
+  uint8_t* qb = vc + kv;
+  uint8_t* ob = qb + qo;
+  cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
+  if (dca_workspace_init(ws, ws_bytes, cuda_stream) != DCA_OK) return DCA_ERR_CUDA;
+  const size_t krow = static_cast<size_t>(Hkv) * d * esize;
+  const size_t qrow = static_cast<size_t>(Hq) * d * esize;
+  for (int64_t q0 = 0; q0 < L; q0 += blk) {
+    const int64_t lq = (L - q0 < blk) ? L - q0 : blk;
+    const int64_t lk = q0 + lq;
+    if (cudaMemcpyAsync(kc + q0 * krow, static_cast<const uint8_t*>(k_h) + q0 * krow, lq * krow,
+                        cudaMemcpyHostToDevice, st) != cudaSuccess ||
+        cudaMemcpyAsync(vc + q0 * krow, static_cast<const uint8_t*>(v_h) + q0 * krow, lq * krow,
+                        cudaMemcpyHostToDevice, st) != cudaSuccess ||
+        cudaMemcpyAsync(qb, static_cast<const uint8_t*>(q_h) + q0 * qrow, lq * qrow,
+                        cudaMemcpyHostToDevice, st) != cudaSuccess)
+      return DCA_ERR_CUDA;
+    // the rotated-key cache keeps rows [0, q0) from earlier blocks
+    int rc = dca_prepare(kc, lk, q0, Hkv, d, chunk_size, local_window, pretrain_window, rope_base,
+                         dtype, ws, ws_bytes, cuda_stream);
+    if (rc != DCA_OK) return rc;
+    rc = dca_attend(qb, vc, ob, q0, lq, lk, Hq, Hkv, d, chunk_size, local_window,
+                    pretrain_window, yarn_scale, dtype, ws, ws_bytes, cuda_stream);
+    if (rc != DCA_OK) return rc;
+    if (cudaMemcpyAsync(static_cast<uint8_t*>(out_h) + q0 * qrow, ob, lq * qrow,
+                        cudaMemcpyDeviceToHost, st) != cudaSuccess)
+      return DCA_ERR_CUDA;
+  }
+  return DCA_OK;
+}
+
+int dca_plan_items(int64_t i0, int64_t i_last, int64_t tile_rows, int64_t chunk_size, int bn,
+                   int32_t* items, int max_items) {
+  if (i0 < 0 || i_last < i0 || tile_rows < 1 || i_last >= i0 + tile_rows || chunk_size < 1 ||
+      bn < 1 || max_items < 0 || (max_items > 0 && items == nullptr))
+    return DCA_ERR_ARG;
+  const dca::TilePlan P = dca::make_plan(i0, i_last, chunk_size, bn);
+  for (int n = 0; n < P.n_items && n < max_items; ++n) {
+    int kt, cls;
+    dca::plan_item(P, n, kt, cls);
+    const int64_t j0 = static_cast<int64_t>(kt) * bn;
+    items[3 * n + 0] = kt;
+    items[3 * n + 1] = cls;
+    items[3 * n + 2] =
+        dca::item_is_full(i0, i0 + tile_rows - 1, j0, j0 + bn - 1, chunk_size, cls) ? 1 : 0;
+  }
+  return P.n_items;
+}
+
+void dca_set_wait_timeout_ns(int64_t ns) {
+  g_timeout_ns.store(ns > 0 ? ns : 10LL * 1000 * 1000 * 1000);
+}
+
+void dca_set_debug_flags(int flags) { g_debug_flags.store(flags); }
+
+}  // extern "C"

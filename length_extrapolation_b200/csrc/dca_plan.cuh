@@ -1,0 +1,111 @@
+// dca_plan.cuh -- tile classification of Dual Chunk Attention, shared by the
+// host code and the kernels of the CUDA path.
+//
+// "Qwen2.5-1M 不重训外推 1M", section 核心思想, splits the causal L x L score
+// matrix into intra-chunk, successive-chunk and inter-chunk parts.  With
+// n_x = x / s, a (query i, key j) pair has chunk distance n_i - n_j:
+//   0 -> INTRA  (query rotated by r_i)
+//   1 -> SUCC   (query rotated by s + r_i when r_i < w, else by c - 1)
+//  >=2 -> INTER (query rotated by c - 1)
+// and every key is rotated by j mod s.  The query rotation therefore depends
+// only on the row and the class, so a (q-tile, k-tile) pair whose pairs all
+// share one class is one plain MMA with that class's rotated Q.
+//
+// For a q-tile with rows [i0, i_last] the keys of each class form one
+// contiguous range, so the k-tiles carrying a class are one contiguous range
+// too.  A q-tile's work list is: INTER k-tiles, then SUCC k-tiles, then INTRA
+// k-tiles (one Q rotation per phase).  A k-tile that holds keys of several
+// classes appears once per class and is masked per element to that class;
+// tiles crossing the causal diagonal are masked to j <= i.
+#pragma once
+#include <stdint.h>
+
+#ifdef __CUDACC__
+#define DCA_HD __host__ __device__ __forceinline__
+#else
+#define DCA_HD inline
+#endif
+
+namespace dca {
+
+enum : int { CLS_INTRA = 0, CLS_SUCC = 1, CLS_INTER = 2 };
+
+struct TilePlan {
+  int lo[3];  // first k-tile of each class (indexed by CLS_*)
+  int hi[3];  // one past the last k-tile
+  int n_items;
+};
+
+DCA_HD int64_t cdiv64(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+DCA_HD int class_of_distance(int64_t chunk_dist) {
+  return chunk_dist <= 0 ? CLS_INTRA : (chunk_dist == 1 ? CLS_SUCC : CLS_INTER);
+}
+
+// Work list of the q-tile whose real rows are [i0, i_last] (absolute indices),
+// for key tiles of `bn` keys.
+DCA_HD TilePlan make_plan(int64_t i0, int64_t i_last, int64_t s, int bn) {
+  TilePlan P;
+  const int64_t n0 = i0 / s, n1 = i_last / s;
+  // INTER: keys with n_j <= n1 - 2, i.e. j < s*(n1-1)
+  P.lo[CLS_INTER] = 0;
+  P.hi[CLS_INTER] = (n1 >= 2) ? static_cast<int>(cdiv64(s * (n1 - 1), bn)) : 0;
+  // SUCC: keys with n_j in [n0-1, n1-1]
+  if (n1 >= 1) {
+    const int64_t a = s * (n0 >= 1 ? n0 - 1 : 0), b = s * n1;
+    P.lo[CLS_SUCC] = static_cast<int>(a / bn);
+    P.hi[CLS_SUCC] = static_cast<int>(cdiv64(b, bn));
+  } else {
+    P.lo[CLS_SUCC] = P.hi[CLS_SUCC] = 0;
+  }
+  // INTRA: keys with n_j in [n0, n1] and j <= i_last
+  P.lo[CLS_INTRA] = static_cast<int>((s * n0) / bn);
+  P.hi[CLS_INTRA] = static_cast<int>(i_last / bn) + 1;
+  P.n_items = (P.hi[CLS_INTER] - P.lo[CLS_INTER]) + (P.hi[CLS_SUCC] - P.lo[CLS_SUCC]) +
+              (P.hi[CLS_INTRA] - P.lo[CLS_INTRA]);
+  return P;
+}
+
+// Item n of the work list -> (k-tile, class).  Order: INTER, SUCC, INTRA.
+DCA_HD void plan_item(const TilePlan& P, int n, int& kt, int& cls) {
+  const int c2 = P.hi[CLS_INTER] - P.lo[CLS_INTER];
+  const int c1 = P.hi[CLS_SUCC] - P.lo[CLS_SUCC];
+  if (n < c2) {
+    cls = CLS_INTER;
+    kt = P.lo[CLS_INTER] + n;
+  } else if (n < c2 + c1) {
+    cls = CLS_SUCC;
+    kt = P.lo[CLS_SUCC] + (n - c2);
+  } else {
+    cls = CLS_INTRA;
+    kt = P.lo[CLS_INTRA] + (n - c2 - c1);
+  }
+}
+
+// True when every (i, j) with i in [i0, i_hi], j in [j0, j_hi] is causal
+// (j <= i) and of class `cls`: the tile needs no per-element mask.
+DCA_HD bool item_is_full(int64_t i0, int64_t i_hi, int64_t j0, int64_t j_hi, int64_t s,
+                         int cls) {
+  const int64_t ni0 = i0 / s, ni1 = i_hi / s, nj0 = j0 / s, nj1 = j_hi / s;
+  if (cls == CLS_INTER) return ni0 - nj1 >= 2;
+  if (cls == CLS_SUCC) return (ni0 - nj1 >= 1) && (ni1 - nj0 <= 1);
+  return ni0 == ni1 && nj0 == nj1 && ni0 == nj0 && j_hi <= i0;
+}
+
+// Position (row of the RoPE table) by which query row i is rotated in class
+// `cls`.  The table stores positions [0, min(s, cap)) directly, positions
+// [s, s + w) directly when cap > s, and position c - 1 at row `tab_c1`.
+DCA_HD int64_t query_table_row(int64_t i, int cls, int64_t s, int64_t w, int64_t tab_c1) {
+  const int64_t r = i % s;
+  if (cls == CLS_INTRA) return r;
+  if (cls == CLS_SUCC && r < w) return s + r;
+  return tab_c1;
+}
+
+// Number of table rows for key capacity `cap`: direct rows plus one for c - 1.
+DCA_HD int64_t table_rows(int64_t cap, int64_t s, int64_t w) {
+  const int64_t direct = (cap < s ? cap : s) + (cap > s ? w : 0);
+  return direct + 1;
+}
+
+}  // namespace dca

@@ -1,0 +1,217 @@
+"""Parity of the CUDA path (through the C ABI) with the fp64 oracle.
+
+Small cases: every output element, sizes spanning several 128-row tiles with
+ragged tails, chunk sizes that are not tile multiples (mixed-class tiles),
+odd GQA groups, YaRN on and off.  Full-size workloads: sampled rows and heads
+(the oracle computes them one by one), run in the same staged launch sequence
+that the benchmark times.
+"""
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import length_extrapolation_b200 as dca
+from length_extrapolation_b200 import _native as N
+from length_extrapolation_b200 import build as B
+from length_extrapolation_b200 import runner
+from length_extrapolation_b200.workloads import WORKLOADS, Workload, generate, sample_heads, sample_rows
+from tests.gpu_helpers import TOL, assert_close, errors, gather
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda:0"
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _built():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    B.build()
+    N.lib()
+
+
+def small(name, L, Hq, Hkv, s, w, c, yarn=1.0, dtype="bf16", sqrt_d=True):
+    return Workload(name, L=L, Hq=Hq, Hkv=Hkv, d=128, dtype=dtype, chunk_size=s, local_window=w,
+                    pretrain_window=c, yarn_scale=yarn, scale_by_sqrt_d=sqrt_d)
+
+
+SMALL = [
+    small("ragged_mixed", 1000, 4, 1, 300, 50, 400),
+    small("g7_yarn2", 777, 7, 1, 256, 128, 512, yarn=2.0),
+    small("g5_yarn4", 2048, 10, 2, 512, 128, 1024, yarn=4.0),
+    small("g1_w0", 130, 2, 2, 64, 0, 64),
+    small("w_eq_s", 900, 2, 1, 200, 200, 400),
+    small("single_chunk", 384, 4, 2, 384, 16, 512),
+    small("tiny_chunks", 300, 2, 1, 3, 2, 5),
+    small("one_token", 1, 3, 1, 64, 8, 128),
+    small("sensitive_N01", 1500, 4, 1, 384, 128, 640, sqrt_d=False),
+    small("f32_small", 700, 3, 1, 200, 40, 300, dtype="f32", sqrt_d=False),
+]
+
+
+def run_small(w, seed=0):
+    q, k, v = generate(w, device=DEV, seed=seed)
+    out = dca.prefill(q, k, v, **w.params())
+    torch.cuda.synchronize()
+    return q, k, v, out
+
+
+@pytest.mark.parametrize("w", SMALL, ids=lambda w: w.name)
+def test_small_all_rows(w):
+    q, k, v, out = run_small(w)
+    want = oracle.attention(q.cpu(), k.cpu(), v.cpu(), **w.params())
+    assert_close(out.double().cpu().numpy(), want, w.torch_dtype, w.name)
+
+
+def test_tiny_f32_workload_all_rows():
+    w = WORKLOADS["tiny_f32_4k"]
+    q, k, v, out = run_small(w)
+    want = oracle.attention(q.cpu(), k.cpu(), v.cpu(), **w.params())
+    ma, rl = assert_close(out.double().cpu().numpy(), want, torch.float32, w.name)
+    print(f"tiny_f32_4k: max_abs {ma:.2e} rel_l2 {rl:.2e}")
+
+
+def test_negative_controls_see_the_mapping():
+    """On inputs with O(1) logits the GPU output differs from oracles with a
+    deliberately wrong position map by far more than the tolerance, so the
+    parity comparison does see the DCA mapping."""
+    w = small("neg", 1024, 2, 1, 256, 64, 384, sqrt_d=False)
+    q, k, v, out = run_small(w)
+    got = out.double().cpu().numpy()
+    qc, kc, vc = q.cpu(), k.cpu(), v.cpu()
+    _, rl_ok = errors(got, oracle.attention(qc, kc, vc, **w.params()))
+    assert rl_ok <= TOL[torch.bfloat16]["rel_l2"]
+    for name in ("query_c", "key_not_periodic", "succ_as_inter", "window_le"):
+        bad = oracle.attention(qc, kc, vc, mutation=oracle.MUTATIONS[name], **w.params())
+        _, rl = errors(got, bad)
+        assert rl > 10 * rl_ok and rl > 2 * TOL[torch.bfloat16]["rel_l2"], (name, rl, rl_ok)
+    bad = oracle.attention(qc, kc, vc, reading=1, **w.params())
+    assert errors(got, bad)[1] > 2 * TOL[torch.bfloat16]["rel_l2"]
+
+
+@pytest.mark.parametrize("aligned", [True, False])
+def test_chunked_blocks_equal_oneshot(aligned):
+    w = small("chunk", 1280, 4, 2, 320, 64, 512, yarn=2.0)
+    q, k, v, full = run_small(w)
+    blk = 256 if aligned else 200
+    parts = []
+    for q0 in range(0, w.L, blk):
+        lq = min(blk, w.L - q0)
+        parts.append(dca.prefill_chunked(q[q0:q0 + lq], k[:q0 + lq], v[:q0 + lq], q_start=q0,
+                                         **w.params()))
+    got = torch.cat(parts)
+    torch.cuda.synchronize()
+    if aligned:
+        assert torch.equal(got, full)
+    else:
+        assert_close(got.double().cpu().numpy(), full.double().cpu().numpy(), torch.bfloat16)
+
+
+def test_incremental_prepare_equals_full_rebuild():
+    w = Workload("inc", L=1536, Hq=4, Hkv=1, d=128, dtype="bf16", chunk_size=512,
+                 local_window=64, pretrain_window=640, yarn_scale=2.0, block=384)
+    q, k, v = generate(w, device=DEV)
+    ws = runner.make_workspace(w, DEV)
+    out = torch.empty_like(q)
+    runner.run_workload(w, q, k, v, out, ws)
+    ref = dca.prefill(q, k, v, **w.params())
+    torch.cuda.synchronize()
+    assert ws.status() == N.DCA_OK
+    assert torch.equal(out, ref)
+
+
+def test_host_entry_matches_device_path():
+    w = Workload("host", L=1000, Hq=4, Hkv=2, d=128, dtype="bf16", chunk_size=256,
+                 local_window=32, pretrain_window=384, yarn_scale=1.5, block=256)
+    q, k, v = generate(w, device="cpu")
+    qh, kh, vh = q.pin_memory(), k.pin_memory(), v.pin_memory()
+    oh = torch.empty_like(qh).pin_memory()
+    n = dca.host_arena_size(w.L, w.block, w.Hq, w.Hkv, w.d, w.chunk_size, w.local_window,
+                            w.pretrain_window, torch.bfloat16)
+    arena = torch.empty(n, dtype=torch.uint8, device=DEV)
+    dca.prefill_host(qh, kh, vh, oh, block=w.block, arena=arena, **w.params())
+    torch.cuda.synchronize()
+    dev = torch.empty_like(q, device=DEV)
+    ws = runner.make_workspace(w, DEV)
+    runner.run_workload(w, q.to(DEV), k.to(DEV), v.to(DEV), dev, ws)
+    torch.cuda.synchronize()
+    assert torch.equal(oh, dev.cpu())
+
+
+def test_bounded_wait_timeout_reports_and_recovers():
+    """Withhold one TMA load: every wait of the kernel runs out after the short
+    limit, the kernel exits cleanly and the status word reports the timeout;
+    the context stays usable."""
+    w = small("timeout", 512, 2, 1, 128, 32, 256)
+    q, k, v = generate(w, device=DEV)
+    ws = runner.make_workspace(w, DEV)
+    out = torch.zeros_like(q)
+    dca.set_wait_timeout_ns(20_000_000)
+    try:
+        dca.set_debug_flags(1)
+        dca.prefill(q, k, v, workspace=ws, out=out, **w.params())
+        assert ws.status() == N.DCA_ERR_TIMEOUT
+    finally:
+        dca.set_debug_flags(0)
+        dca.set_wait_timeout_ns(0)
+    out2 = dca.prefill(q, k, v, workspace=ws, **w.params())
+    assert ws.status() == N.DCA_OK
+    want = oracle.attention(q.cpu(), k.cpu(), v.cpu(), **w.params())
+    assert_close(out2.double().cpu().numpy(), want, torch.bfloat16)
+
+
+def test_empty_block_is_a_no_op():
+    w = small("empty", 256, 2, 1, 128, 32, 256)
+    q, k, v = generate(w, device=DEV)
+    out = torch.full_like(q, 7.0)
+    dca.prefill_chunked(q[:0], k, v, q_start=100, out=out[:0], **w.params())
+    torch.cuda.synchronize()
+    assert torch.all(out == 7.0)
+
+
+# ------------------------------------------------------------------ full size
+def _full_size_check(name, max_rows=None, n_random=48, blocks_to_check=None):
+    w = WORKLOADS[name]
+    q, k, v = generate(w, device=DEV)
+    ws = runner.make_workspace(w, DEV)
+    out = torch.empty_like(q)
+    runner.run_workload(w, q, k, v, out, ws)
+    assert ws.status() == N.DCA_OK
+    heads = sample_heads(w).numpy()
+    kc, vc = k.cpu(), v.cpu()
+    blocks = w.blocks()
+    if blocks_to_check is not None:
+        blocks = [blocks[b] for b in blocks_to_check]
+    worst = (0.0, 0.0)
+    for q0, lq, lk in blocks:
+        rows = sample_rows(w, q0, lq, n_random=n_random).numpy()
+        if max_rows is not None and len(rows) > max_rows:
+            sel = np.linspace(0, len(rows) - 1, max_rows).round().astype(int)
+            rows = rows[np.unique(sel)]
+        want = oracle.attention(q[q0:q0 + lq].cpu(), kc[:lk], vc[:lk], q_start=q0, rows=rows,
+                                heads=heads, **w.params())
+        got = gather(out[q0:q0 + lq], rows, heads)
+        ma, rl = assert_close(got, want, w.torch_dtype, f"{name} block q0={q0}")
+        worst = (max(worst[0], ma), max(worst[1], rl))
+    print(f"{name}: worst max_abs {worst[0]:.2e} rel_l2 {worst[1]:.2e}")
+
+
+def test_full_size_qwen7b_32k():
+    _full_size_check("qwen7b_32k")
+
+
+def test_full_size_qwen14b_128k():
+    _full_size_check("qwen14b_128k", max_rows=48, n_random=24)
+
+
+def test_full_size_qwen7b_256k():
+    _full_size_check("qwen7b_256k", max_rows=40, n_random=16)
+
+
+def test_full_size_qwen7b_1m_chunked():
+    # first, a middle and the last query block (all 32 blocks run on the GPU)
+    _full_size_check("qwen7b_1m_chunked", max_rows=12, n_random=4, blocks_to_check=[0, 13, 31])

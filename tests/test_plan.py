@@ -1,0 +1,110 @@
+"""The tile plan of the CUDA kernels (host-side introspection through the C ABI)
+against the oracle's per-pair DCA positions, on CPU.
+
+For every query tile of a sweep of small configurations:
+  * coverage: every causal pair (i, j) of a real row is admitted by exactly one
+    work item -- the item of its key tile whose class is the pair's chunk
+    distance class -- and that class's query rotation equals the oracle's query
+    position for the pair;
+  * full items really are uniform: every pair of a 'full' tile is causal and of
+    the item's class (so skipping the mask is safe).
+"""
+import ctypes
+
+import numpy as np
+import pytest
+
+import oracle
+from length_extrapolation_b200 import _native as N
+from length_extrapolation_b200 import build as B
+
+
+@pytest.fixture(scope="module")
+def lib():
+    B.build()
+    return N.lib()
+
+
+def plan(lib, i0, i_last, rows, s, bn):
+    buf = (ctypes.c_int32 * (3 * 16384))()
+    n = lib.dca_plan_items(i0, i_last, rows, s, bn, buf, 16384)
+    assert 0 <= n <= 16384
+    a = np.frombuffer(buf, dtype=np.int32)[: 3 * n].reshape(n, 3)
+    return a
+
+
+def chunk_class(i, j, s):
+    dn = i // s - j // s
+    return 0 if dn == 0 else (1 if dn == 1 else 2)
+
+
+def query_position(i, cls, s, w, c):
+    """Query rotation of a row in a plan class, as stated in include/dca.h."""
+    r = i % s
+    if cls == 0:
+        return r
+    if cls == 1 and r < w:
+        return s + r
+    return c - 1
+
+
+CASES = [  # (L, s, w, c, bm, bn)
+    (300, 64, 16, 100, 64, 64),
+    (300, 100, 30, 140, 64, 64),
+    (520, 37, 5, 50, 128, 128),
+    (700, 128, 128, 256, 128, 128),
+    (700, 200, 0, 200, 128, 128),
+    (260, 1, 1, 2, 128, 128),
+    (260, 3, 2, 5, 64, 64),
+    (400, 1000, 7, 1, 128, 128),    # single chunk (L <= s): everything intra
+    (1100, 256, 128, 512, 128, 128),
+]
+
+
+@pytest.mark.parametrize("L,s,w,c,bm,bn", CASES)
+def test_plan_matches_oracle_positions(lib, L, s, w, c, bm, bn):
+    for q_start, Lq in [(0, L), (L // 3, L - L // 3)]:
+        for t0 in range(0, Lq, bm):
+            i0 = q_start + t0
+            i_last = min(i0 + bm - 1, q_start + Lq - 1)
+            items = plan(lib, i0, i_last, bm, s, bn)
+            # phases in order INTER, SUCC, INTRA
+            assert list(items[:, 1]) == sorted(items[:, 1], reverse=True)
+            seen = {}
+            for kt, cls, full in items:
+                assert (kt, cls) not in seen
+                seen[(kt, cls)] = full
+                if full:
+                    for i in range(i0, i0 + bm):
+                        for j in range(kt * bn, kt * bn + bn):
+                            assert j <= i and chunk_class(i, j, s) == cls
+            for i in range(i0, i_last + 1):
+                for j in range(0, i + 1):
+                    cls = chunk_class(i, j, s)
+                    assert (j // bn, cls) in seen, (i, j)
+                    _, pq, pk = oracle.position(i, j, s, w, c)
+                    assert pk == j % s
+                    assert query_position(i, cls, s, w, c) == pq, (i, j, cls)
+
+
+def test_plan_rejects_bad_args(lib):
+    buf = (ctypes.c_int32 * 3)()
+    assert lib.dca_plan_items(10, 5, 128, 64, 128, buf, 1) == N.DCA_ERR_ARG
+    assert lib.dca_plan_items(0, 200, 128, 64, 128, buf, 1) == N.DCA_ERR_ARG
+    assert lib.dca_plan_items(0, 5, 128, 0, 128, buf, 1) == N.DCA_ERR_ARG
+
+
+def test_big_config_phase_counts(lib):
+    """Last query tile of the 1M chunked workload: INTER keys of chunks 0-3,
+    SUCC tiles of chunk 4, INTRA tiles of chunk 5 up to the diagonal, all full
+    except the diagonal tile."""
+    s, L = 196608, 1048576
+    i0 = L - 128
+    items = plan(lib, i0, L - 1, 128, s, 128)
+    n_inter = (items[:, 1] == 2).sum()
+    n_succ = (items[:, 1] == 1).sum()
+    n_intra = (items[:, 1] == 0).sum()
+    assert n_inter == 4 * s // 128
+    assert n_succ == s // 128
+    assert n_intra == (L - 5 * s) // 128
+    assert items[:, 2].sum() == len(items) - 1
