@@ -1,0 +1,379 @@
+#!/usr/bin/env python3
+"""DCA prefill benchmark on B200.
+
+One step = one whole prefill of the workload through the library's staged C
+ABI (per query block: rotate the block's keys into the rotated-key cache, then
+the fused attention kernel), inputs resident in HBM.  Default workload: the
+1M-token chunked prefill of the 7B shape (32 query blocks of 32,768 tokens,
+Hq 28 / Hkv 4, d 128, chunk 196,608, local window 32,768, pretraining window
+262,144, YaRN 4, bf16), synthetic seeded inputs.
+
+Prints one JSON line (rank 0):
+  value        whole-job tokens/s (all ranks; replicas, weak scaling)
+  tflops       algorithmic attention TFLOP/s of the whole step (4*d*Hq per causal pair)
+  roofline     the attention kernel: algorithmic FLOPs / CUDA-event time of its launches
+  e2e          same metric through the host-buffer C entry point (copies timed)
+  cpu_baseline the fp64 oracle on a bounded sample, on the host cores (rank 0, N=1)
+``--impl reference`` times that oracle alone as the reference arm.
+
+Multi-GPU: ``torchrun --nproc-per-node N bench.py --gpus N``: N independent
+replicas (the method has no exchange step), timed as the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+from length_extrapolation_b200.workloads import WORKLOADS, generate, sample_heads  # noqa: E402
+
+METRIC = "DCA prefill tokens/s and attention TFLOP/s (fraction of B200 bf16 peak)"
+UNIT = "tokens/s"
+
+
+def parse_args(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=3)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="qwen7b_1m_chunked", choices=sorted(WORKLOADS))
+    ap.add_argument("--e2e-steps", type=int, default=2)
+    ap.add_argument("--cpu-seconds", type=float, default=20.0,
+                    help="approximate CPU seconds for the oracle baseline sample")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args(argv)
+
+
+# ----------------------------------------------------------------------------- helpers
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            pk = json.load(f)
+        return dict(bf16_tflops=float(pk["bf16_tflops"]),
+                    bf16_tflops_sustained=float(pk.get("bf16_tflops_sustained", pk["bf16_tflops"])),
+                    hbm_gbs=float(pk["hbm_gbs"]), source="measured")
+    except (OSError, KeyError, ValueError):
+        return dict(bf16_tflops=1590.0, bf16_tflops_sustained=1400.0, hbm_gbs=6650.0,
+                    source="fallback")
+
+
+def causal_pairs(q0, lq):
+    """Number of causal (query, key) pairs of rows q0 .. q0+lq-1 (key j <= i)."""
+    return lq * q0 + lq * (lq + 1) // 2
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples every 200 ms while running."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.samples = []
+        self.proc = None
+        self.thread = None
+        try:
+            uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+            sel = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
+        except Exception:  # pragma: no cover
+            sel = str(device_index)
+        self.cmd = ["nvidia-smi", "-i", sel, f"--query-gpu={self.FIELDS}",
+                    "--format=csv,noheader,nounits", "-lms", "200"]
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(self.cmd, stdout=subprocess.PIPE,
+                                         stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+            return self
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) >= 9:
+                self.samples.append(parts)
+
+    def stop(self):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+        if self.thread is not None:
+            self.thread.join(timeout=5)
+        return self.summary()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"], "samples": 0}
+
+        def num(x):
+            try:
+                return float(x)
+            except ValueError:
+                return None
+
+        sm = [num(s[1]) for s in self.samples if num(s[1]) is not None]
+        smax = [num(s[2]) for s in self.samples if num(s[2]) is not None]
+        load = [x for x in sm if smax and x > 0.3 * max(smax)] or sm
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[k] for s in self.samples for k in range(4)
+                          if s[5 + k].lower().startswith("active")})
+        return {"sm_mhz": statistics.median(load) if load else None,
+                "sm_max_mhz": max(smax) if smax else None, "reasons": reasons,
+                "samples": len(self.samples),
+                "power_w_max": max((num(s[3]) or 0.0) for s in self.samples)}
+
+
+def oracle_sample_rate(w, q_block, k, v, q0, lq, budget_s, rows_from_end=True):
+    """Time the fp64 oracle on (row, head) samples of one block; returns
+    (pairs*heads per second, description, threads used)."""
+    import numpy as np
+
+    import oracle
+    threads = os.cpu_count() or 1
+    heads = sample_heads(w).numpy()
+    qc = q_block.cpu()
+    lk = q0 + lq
+    kc, vc = k[:lk].cpu(), v[:lk].cpu()
+    # calibrate on one row, then size the sample to the time budget
+    rows = np.array([lq - 1], dtype=np.int64)
+    t0 = time.perf_counter()
+    oracle.attention(qc, kc, vc, q_start=q0, rows=rows, heads=heads[:1], n_threads=threads,
+                     **w.params())
+    dt1 = max(time.perf_counter() - t0, 1e-3)
+    n_rows = int(max(1, min(lq, budget_s / dt1 * threads / len(heads))))
+    rows = np.arange(lq - n_rows, lq, dtype=np.int64) if rows_from_end else np.arange(n_rows)
+    t0 = time.perf_counter()
+    oracle.attention(qc, kc, vc, q_start=q0, rows=rows, heads=heads, n_threads=threads,
+                     **w.params())
+    dt = time.perf_counter() - t0
+    pairs = sum(q0 + int(r) + 1 for r in rows) * len(heads)
+    desc = (f"{len(rows)} rows x {len(heads)} heads of block q_start={q0} "
+            f"({pairs:.3e} causal pair-heads in {dt:.1f} s)")
+    return pairs / dt, desc, threads, dt
+
+
+def total_pair_heads(w):
+    return sum(causal_pairs(q0, lq) for q0, lq, _ in w.blocks()) * w.Hq
+
+
+# ----------------------------------------------------------------------------- reference arm
+def run_reference(args, w, rank, world):
+    """The oracle as it stands, on the host cores: each step times a bounded
+    sample of the workload and reports extrapolated tokens/s."""
+    if rank != 0:
+        return 0
+    import numpy as np  # noqa: F401
+    q, k, v = generate(w, device="cpu")
+    q0, lq, _ = w.blocks()[-1]
+    budget = max(2.0, 120.0 / max(1, args.steps + args.warmup))
+    rates = []
+    desc = threads = None
+    for it in range(args.warmup + args.steps):
+        rate, desc, threads, _ = oracle_sample_rate(w, q[q0:q0 + lq], k, v, q0, lq, budget)
+        if it >= args.warmup:
+            rates.append(rate)
+    rate = statistics.median(rates)
+    t_full = total_pair_heads(w) / rate
+    value = w.L / t_full
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": t_full * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic",
+        "config": workload_config(w),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
+                         "sample": desc},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def workload_config(w):
+    return {"workload": w.name, "L": w.L, "Hq": w.Hq, "Hkv": w.Hkv, "d": w.d,
+            "chunk_size": w.chunk_size, "local_window": w.local_window,
+            "pretrain_window": w.pretrain_window, "rope_base": w.rope_base,
+            "yarn_scale": w.yarn_scale, "query_block": w.block or w.L,
+            "global_batch": 1, "seq_len": w.L,
+            "l2": "inputs larger than L2 (no flush)"}
+
+
+# ----------------------------------------------------------------------------- our arm
+def main(argv=None):
+    args = parse_args(argv)
+    w = WORKLOADS[args.workload]
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    dist = None
+    if world > 1:
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=900),
+                                device_id=torch.device("cuda", local))
+    if args.impl == "reference":
+        rc = run_reference(args, w, rank, world)
+        if dist is not None:
+            dist.destroy_process_group()
+        return rc
+
+    import length_extrapolation_b200 as dca
+    from length_extrapolation_b200 import _native as N
+    from length_extrapolation_b200 import runner
+
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    peaks = load_peaks()
+    q, k, v = generate(w, device=dev, seed=0)
+    out = torch.empty_like(q)
+    ws = runner.make_workspace(w, dev)
+    blocks = w.blocks()
+    attn_flops = [4.0 * w.d * w.Hq * causal_pairs(q0, lq) for q0, lq, _ in blocks]
+    step_flops = sum(attn_flops)
+    launches_per_step = 1 + 2 * len(blocks)  # RoPE table + (key rotation, attention) per block
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+
+    for _ in range(args.warmup):
+        runner.run_workload(w, q, k, v, out, ws)
+    torch.cuda.synchronize()
+    st = ws.status()
+    if st != N.DCA_OK:
+        raise RuntimeError(f"device status after warm-up: {N.status_string(st)}")
+
+    clocks = ClockSampler(dev.index).start()
+    ev_all = []
+    barrier()
+    torch.cuda.synchronize()
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    t_start.record()
+    for _ in range(args.steps):
+        runner.run_workload(w, q, k, v, out, ws, attn_events=ev_all)
+    t_end.record()
+    torch.cuda.synchronize()
+    barrier()
+    clk = clocks.stop()
+    ms = t_start.elapsed_time(t_end)
+    st = ws.status()
+    if st != N.DCA_OK:
+        raise RuntimeError(f"device status after timing: {N.status_string(st)}")
+    attn_ms = sum(a.elapsed_time(b) for a, b in ev_all)
+    ms_t = torch.tensor([ms, attn_ms], device=dev, dtype=torch.float64)
+    if dist is not None:
+        dist.all_reduce(ms_t, op=dist.ReduceOp.MAX)
+    ms_max, attn_ms_max = float(ms_t[0]), float(ms_t[1])
+    ms_per_step = ms_max / args.steps
+    value = world * w.L / (ms_per_step / 1e3)
+    tflops = world * step_flops / (ms_per_step / 1e3) / 1e12
+
+    achieved = step_flops * args.steps / (attn_ms_max / 1e3) / 1e12
+    roofline = {
+        "kernel": "dca_fwd_kernel (tcgen05 attention)" if w.dtype == "bf16" else "dca_fwd_f32_kernel",
+        "bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops_sustained"],
+        "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops_sustained"],
+        "peak_kind": f"{peaks['source']} sustained bf16 (cuBLAS, power-capped loop)",
+        "frac_of_burst_peak": achieved / peaks["bf16_tflops"],
+        "frac_of_datasheet_2250": achieved / 2250.0,
+        "traffic": None,
+        "launches_per_step": len(blocks),
+        "avg_launch_ms": attn_ms_max / (args.steps * len(blocks)),
+    }
+
+    # ---------------------------------------------------------------- end to end
+    e2e = None
+    if not args.no_e2e:
+        qh = q.cpu().pin_memory()
+        kh = k.cpu().pin_memory()
+        vh = v.cpu().pin_memory()
+        oh = torch.empty_like(qh).pin_memory()
+        n = dca.host_arena_size(w.L, w.block or w.L, w.Hq, w.Hkv, w.d, w.chunk_size,
+                                w.local_window, w.pretrain_window, w.torch_dtype)
+        del out, ws
+        torch.cuda.empty_cache()
+        arena = torch.empty(n, dtype=torch.uint8, device=dev)
+        dca.prefill_host(qh, kh, vh, oh, block=w.block or w.L, arena=arena, **w.params())
+        torch.cuda.synchronize()
+        barrier()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(args.e2e_steps):
+            dca.prefill_host(qh, kh, vh, oh, block=w.block or w.L, arena=arena, **w.params())
+        e1.record()
+        torch.cuda.synchronize()
+        barrier()
+        ems = torch.tensor([e0.elapsed_time(e1)], device=dev, dtype=torch.float64)
+        if dist is not None:
+            dist.all_reduce(ems, op=dist.ReduceOp.MAX)
+        ems_step = float(ems[0]) / args.e2e_steps
+        esz = q.element_size()
+        e2e = {"value": world * w.L / (ems_step / 1e3), "unit": UNIT,
+               "ms_per_step": ems_step,
+               "h2d_bytes_per_step": (q.numel() + k.numel() + v.numel()) * esz,
+               "d2h_bytes_per_step": q.numel() * esz,
+               "path": "dca_prefill_host (pinned host buffers, copies and kernels on one stream)"}
+        del arena
+
+    # ---------------------------------------------------------------- CPU baseline
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        q0, lq, _ = blocks[-1]
+        rate, desc, threads, _ = oracle_sample_rate(w, q[q0:q0 + lq], k, v, q0, lq,
+                                                    args.cpu_seconds)
+        t_full = total_pair_heads(w) / rate
+        cpu = {"value": w.L / t_full, "unit": UNIT, "cores": threads, "kind": "oracle",
+               "sample": desc + "; extrapolated to all causal pairs of the workload"}
+
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
+        "config": {**workload_config(w), "parallelism": f"replicas x{world}" if world > 1 else "1 GPU"},
+        "tflops": tflops,
+        "tflops_frac_of_peak": {"measured_sustained": tflops / world / peaks["bf16_tflops_sustained"],
+                                "measured_burst": tflops / world / peaks["bf16_tflops"],
+                                "datasheet_2250": tflops / world / 2250.0},
+        "roofline": roofline,
+        "e2e": e2e,
+        "cpu_baseline": cpu,
+        "clocks": clk,
+        "gpu_launches": launches_per_step * args.steps,
+        "peaks_source": peaks["source"],
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -85,10 +85,14 @@ def test_negative_controls_see_the_mapping():
     qc, kc, vc = q.cpu(), k.cpu(), v.cpu()
     _, rl_ok = errors(got, oracle.attention(qc, kc, vc, **w.params()))
     assert rl_ok <= TOL[torch.bfloat16]["rel_l2"]
-    for name in ("query_c", "key_not_periodic", "succ_as_inter", "window_le"):
+    for name in ("query_c", "key_not_periodic", "succ_as_inter", "sin_sign", "pair_adjacent"):
         bad = oracle.attention(qc, kc, vc, mutation=oracle.MUTATIONS[name], **w.params())
         _, rl = errors(got, bad)
         assert rl > 10 * rl_ok and rl > 2 * TOL[torch.bfloat16]["rel_l2"], (name, rl, rl_ok)
+    # r_i <= w instead of r_i < w changes one query row per chunk: smaller, but
+    # still outside the tolerance band
+    bad = oracle.attention(qc, kc, vc, mutation=oracle.MUTATIONS["window_le"], **w.params())
+    assert errors(got, bad)[1] > 2 * TOL[torch.bfloat16]["rel_l2"]
     bad = oracle.attention(qc, kc, vc, reading=1, **w.params())
     assert errors(got, bad)[1] > 2 * TOL[torch.bfloat16]["rel_l2"]
 
