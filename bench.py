@@ -180,6 +180,34 @@ def total_pair_heads(w):
     return sum(causal_pairs(q0, lq) for q0, lq, _ in w.blocks()) * w.Hq
 
 
+def init_dist(world: int, local: int):
+    """Process group for N > 1 (one process per GPU; gloo when there is no GPU)."""
+    if world <= 1:
+        return None
+    import torch.distributed as dist
+    if torch.cuda.is_available():
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=900),
+                                device_id=torch.device("cuda", local))
+    else:
+        dist.init_process_group("gloo", timeout=datetime.timedelta(seconds=120))
+    return dist
+
+
+def max_over_ranks(values, dist, device="cpu"):
+    """Element-wise max of a list of floats over all ranks (identity without dist)."""
+    t = torch.tensor([float(x) for x in values], dtype=torch.float64, device=device)
+    if dist is not None:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(x) for x in t.tolist()]
+
+
+def whole_job_rate(tokens_per_rank: int, world: int, ms_per_step: float) -> float:
+    """Replicas: every rank runs the whole workload; the job's rate divides all
+    ranks' tokens by the slowest rank's step time."""
+    return world * tokens_per_rank / (ms_per_step / 1e3)
+
+
 # ----------------------------------------------------------------------------- reference arm
 def run_reference(args, w, rank, world):
     """The oracle as it stands, on the host cores: each step times a bounded
@@ -189,7 +217,7 @@ def run_reference(args, w, rank, world):
     import numpy as np  # noqa: F401
     q, k, v = generate(w, device="cpu")
     q0, lq, _ = w.blocks()[-1]
-    budget = max(2.0, 120.0 / max(1, args.steps + args.warmup))
+    budget = min(args.cpu_seconds, max(2.0, 120.0 / max(1, args.steps + args.warmup)))
     rates = []
     desc = threads = None
     for it in range(args.warmup + args.steps):
@@ -229,12 +257,7 @@ def main(argv=None):
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
-    dist = None
-    if world > 1:
-        import torch.distributed as dist
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=900),
-                                device_id=torch.device("cuda", local))
+    dist = init_dist(world, local)
     if args.impl == "reference":
         rc = run_reference(args, w, rank, world)
         if dist is not None:
@@ -285,12 +308,9 @@ def main(argv=None):
     if st != N.DCA_OK:
         raise RuntimeError(f"device status after timing: {N.status_string(st)}")
     attn_ms = sum(a.elapsed_time(b) for a, b in ev_all)
-    ms_t = torch.tensor([ms, attn_ms], device=dev, dtype=torch.float64)
-    if dist is not None:
-        dist.all_reduce(ms_t, op=dist.ReduceOp.MAX)
-    ms_max, attn_ms_max = float(ms_t[0]), float(ms_t[1])
+    ms_max, attn_ms_max = max_over_ranks([ms, attn_ms], dist, dev)
     ms_per_step = ms_max / args.steps
-    value = world * w.L / (ms_per_step / 1e3)
+    value = whole_job_rate(w.L, world, ms_per_step)
     tflops = world * step_flops / (ms_per_step / 1e3) / 1e12
 
     achieved = step_flops * args.steps / (attn_ms_max / 1e3) / 1e12
@@ -329,12 +349,9 @@ def main(argv=None):
         e1.record()
         torch.cuda.synchronize()
         barrier()
-        ems = torch.tensor([e0.elapsed_time(e1)], device=dev, dtype=torch.float64)
-        if dist is not None:
-            dist.all_reduce(ems, op=dist.ReduceOp.MAX)
-        ems_step = float(ems[0]) / args.e2e_steps
+        ems_step = max_over_ranks([e0.elapsed_time(e1)], dist, dev)[0] / args.e2e_steps
         esz = q.element_size()
-        e2e = {"value": world * w.L / (ems_step / 1e3), "unit": UNIT,
+        e2e = {"value": whole_job_rate(w.L, world, ems_step), "unit": UNIT,
                "ms_per_step": ems_step,
                "h2d_bytes_per_step": (q.numel() + k.numel() + v.numel()) * esz,
                "d2h_bytes_per_step": q.numel() * esz,
