@@ -168,6 +168,32 @@ int dca_plan_items(int64_t i0, int64_t i_last, int64_t tile_rows, int64_t chunk_
                    int32_t* items, int max_items);
 
 /*
+ * No-allocation one-shot prefill (an addition for integrators; the pages on
+ * DCA have no counterpart).  For callers that cannot call cudaMalloc: e.g. a
+ * serving process that hands all free HBM to its own pool at start-up, where a
+ * later allocation fails or stalls the device, or a plugin whose host
+ * framework owns every device allocation.  Same arguments and result as
+ * dca_prefill, minus the workspace: the library uses a fixed scratch area of
+ * DCA_NOALLOC_SCRATCH_BYTES that is part of its image (present on every GPU
+ * that loads the library until the process exits), and calls no cudaMalloc,
+ * cudaFree or allocating library routine.
+ *   - Returns DCA_ERR_WORKSPACE, before any launch, when
+ *     dca_workspace_size(L, ...) exceeds DCA_NOALLOC_SCRATCH_BYTES (about
+ *     L <= 16384 for 4 KV heads in bf16).
+ *   - The first call on a device looks up the scratch address on that device
+ *     (with it current); make that first call before any stream capture.
+ *   - All calls share the one scratch area: calls that overlap on the GPU
+ *     (other streams, other threads) race and must be serialised by the caller.
+ *   - The status word in the scratch is cleared at the start of each call and
+ *     cannot be read back with dca_device_status.
+ */
+#define DCA_NOALLOC_SCRATCH_BYTES (32u * 1024u * 1024u)
+int dca_prefill_noalloc(const void* q, const void* k, const void* v, void* out, int64_t L,
+                        int Hq, int Hkv, int d, int64_t chunk_size, int64_t local_window,
+                        int64_t pretrain_window, double rope_base, double yarn_scale, int dtype,
+                        void* cuda_stream);
+
+/*
  * Test hooks.  dca_set_wait_timeout_ns sets the limit of every bounded device
  * wait (default 10 s).  dca_set_debug_flags(1) makes the next attention launch
  * withhold its first key-tile load, so that its waits run out and the kernel

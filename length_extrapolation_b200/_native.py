@@ -37,6 +37,8 @@ SIGNATURES = {
     "dca_prefill_host": (_i32, [_vp, _vp, _vp, _vp, _i64, _i64, _i32, _i32, _i32, _i64, _i64,
                                 _i64, _dbl, _dbl, _i32, _vp, _sz, _vp]),
     "dca_plan_items": (_i32, [_i64, _i64, _i64, _i64, _i32, _vp, _i32]),
+    "dca_prefill_noalloc": (_i32, [_vp, _vp, _vp, _vp, _i64, _i32, _i32, _i32, _i64, _i64, _i64,
+                                   _dbl, _dbl, _i32, _vp]),
     "dca_set_wait_timeout_ns": (None, [_i64]),
     "dca_set_debug_flags": (None, [_i32]),
 }
