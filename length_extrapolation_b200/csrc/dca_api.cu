@@ -307,14 +307,17 @@ int dca_plan_items(int64_t i0, int64_t i_last, int64_t tile_rows, int64_t chunk_
       bn < 1 || max_items < 0 || (max_items > 0 && items == nullptr))
     return DCA_ERR_ARG;
   const dca::TilePlan P = dca::make_plan(i0, i_last, chunk_size, bn);
+  const dca::FullRanges F = dca::make_full_ranges(i0, i0 + tile_rows - 1, chunk_size, bn);
   for (int n = 0; n < P.n_items && n < max_items; ++n) {
     int kt, cls;
     dca::plan_item(P, n, kt, cls);
     const int64_t j0 = static_cast<int64_t>(kt) * bn;
+    const bool full = dca::item_is_full(i0, i0 + tile_rows - 1, j0, j0 + bn - 1, chunk_size, cls);
+    // the kernels use the precomputed ranges; they must agree with the predicate
+    if (full != dca::is_full(F, kt, cls)) return DCA_ERR_ARG - 100;
     items[3 * n + 0] = kt;
     items[3 * n + 1] = cls;
-    items[3 * n + 2] =
-        dca::item_is_full(i0, i0 + tile_rows - 1, j0, j0 + bn - 1, chunk_size, cls) ? 1 : 0;
+    items[3 * n + 2] = full ? 1 : 0;
   }
   return P.n_items;
 }

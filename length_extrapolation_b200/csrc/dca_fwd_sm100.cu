@@ -2,16 +2,22 @@
 //
 // One CTA computes one 128-row query tile for two query heads of the same KV
 // group (GQA: the K/V tiles it streams are shared by both heads; when the group
-// size is odd the last head runs alone).  Warp roles:
-//   warps 0-3  softmax of head A (one query row per thread, TMEM lanes 0-127)
-//   warps 4-7  softmax of head B
+// size is odd the last head runs alone).  Warp roles (320 threads):
+//   warps 0-7  softmax.  Warp w and warp w+4 share TMEM lanes 32*(w%4)..+31
+//              (one query row per lane) and split each row's 128 keys in two
+//              halves; every work item they process head A's scores, then
+//              head B's, so two warps per SM sub-partition work on the head
+//              whose scores are ready while the tensor cores run the other
+//              head's MMAs (ping-pong).
 //   warp  8    TMA producer: K'/V tiles (128 keys x 128 dims, bf16, 128-byte
-//              swizzle) into a ring of shared-memory slots
+//              swizzle) into a ring of shared-memory slots (no multicast)
 //   warp  9    MMA issuer (one thread): S = Q K'^T and O += P V with
 //              tcgen05.mma kind::f16 (bf16 in, fp32 accumulate in TMEM)
 // TMEM (512 columns): S_A [0,128), S_B [128,256), O_A [256,384), O_B [384,512);
 // P (bf16) overwrites the first 64 columns of its S and is the TMEM A operand
-// of the P.V MMA.
+// of the P.V MMA.  MMA order per item: P.V(A), S(A, next), P.V(B), S(B, next);
+// MMAs of one thread execute in order, so S(next) never overwrites P before
+// P.V has read it.
 //
 // DCA ("Qwen2.5-1M 不重训外推 1M", sections 核心思想 / Intra / Successive /
 // Inter-Chunk Attention): keys arrive pre-rotated by j mod s; each query row is
@@ -22,9 +28,11 @@
 // below the diagonal run unmasked; others are masked per element.
 // YaRN temperature: logits * m^2/sqrt(d), folded into the exp2 argument.
 //
-// Online softmax: running max kept per row; O and the row sum are rescaled
-// only when the max grows by more than 2^8 (P stays <= 256, exact in fp32 and
-// in bf16's exponent range), the final O / l uses the same reference max.
+// Online softmax: the row's reference max is updated (and O, l rescaled) only
+// when the max grows by more than 2^8; the final O / l uses the same reference.
+// A share of the exponentials runs on the FMA pipe (exp2_poly2) to relieve the
+// MUFU pipe, which at d = 128 needs as many SM cycles per score as the tensor
+// cores.
 //
 // Every wait is bounded (globaltimer); on timeout the CTA raises a shared
 // abort flag, ORs a code into the device status word, drains its own TMA
@@ -44,13 +52,23 @@ namespace sm100 {
 constexpr int BM = 128;            // query rows per tile
 constexpr int BN = 128;            // keys per tile
 constexpr int HD = 128;            // head dim
-constexpr int NSLOT = 4;           // K/V ring slots
+#ifndef DCA_NSLOT
+#define DCA_NSLOT 4
+#endif
+constexpr int NSLOT = DCA_NSLOT;   // K/V ring slots
 constexpr int TILE_BYTES = 32768;  // 128 x 128 bf16
 constexpr int HALF_BYTES = 16384;  // 128 rows x 64 bf16 (one 128-byte swizzle column block)
+// 10 warps: 8 softmax (warps 0-3 head A, 4-7 head B; one query row per
+// thread), TMA producer, MMA issuer.
 constexpr int NUM_THREADS = 320;
 constexpr int WARP_LOAD = 8;
 constexpr int WARP_MMA = 9;
 constexpr float RESCALE_LOG2 = 8.0f;
+// How the MMA issuer waits: polling with a short back-off (wait_spin) or a
+// suspending try_wait (wait_bounded).
+#ifndef DCA_MMA_WAIT
+#define DCA_MMA_WAIT wait_spin
+#endif
 
 // status codes (bits) for timeouts, by role
 constexpr unsigned ST_SOFTMAX = 0x10u, ST_LOAD = 0x100u, ST_MMA = 0x1000u, ST_DRAIN = 0x10000u;
@@ -65,6 +83,9 @@ struct SmemCtl {
   uint64_t drain;
   uint32_t tmem_base;
   int abort;
+  // values exchanged between the two threads of a row: [phase parity][half][row]
+  float xval[2][2][128];
+  uint64_t pair_bar[4];  // one per TMEM lane quarter (its two warps arrive)
 };
 
 constexpr size_t SMEM_BYTES = 1024 + 2 * TILE_BYTES + NSLOT * TILE_BYTES + sizeof(SmemCtl);
@@ -88,14 +109,50 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
+// Software 2^x for a pair of arguments x <= 8, on the FMA and ALU pipes, to
+// take part of the exponentials off the MUFU pipe (at d = 128 one MUFU ex2
+// per score costs as much SM time as the score's tensor-core work).
+// Method: x = n + f with n = round(x) (adding 1.5 * 2^23 rounds to an integer
+// in fp32) and f in [-1/2, 1/2]; 2^f by a degree-3 polynomial fitted for
+// minimum relative error with the Remez exchange (exp2_poly_fit.py next to
+// this file: max relative error 7.5e-5, below the 2^-9 half-ulp of the bf16 P);
+// 2^n added to the exponent field.  Arguments below -126 are clamped (result
+// ~0, as for the hardware path).
+constexpr float EXP2_C0 = 0.9999280571937561f;
+constexpr float EXP2_C1 = 0.6932609677314758f;
+constexpr float EXP2_C2 = 0.2426111251115799f;
+constexpr float EXP2_C3 = 0.0551716685295105f;
+
+__device__ __forceinline__ float2 exp2_poly2(float2 x) {
+  const float RND = 12582912.0f;  // 1.5 * 2^23
+  x.x = fmaxf(x.x, -126.0f);
+  x.y = fmaxf(x.y, -126.0f);
+  const float2 t = add2(x, make_float2(RND, RND));
+  const float2 n = add2(t, make_float2(-RND, -RND));
+  const float2 f = fma2(n, make_float2(-1.0f, -1.0f), x);
+  float2 q = fma2(make_float2(EXP2_C3, EXP2_C3), f, make_float2(EXP2_C2, EXP2_C2));
+  q = fma2(q, f, make_float2(EXP2_C1, EXP2_C1));
+  q = fma2(q, f, make_float2(EXP2_C0, EXP2_C0));
+  // the integer n sits in the low mantissa bits of t; shifting by 23 moves it
+  // into the exponent field (the constant part of t shifts out)
+  return make_float2(__uint_as_float(__float_as_uint(q.x) + (__float_as_uint(t.x) << 23)),
+                     __uint_as_float(__float_as_uint(q.y) + (__float_as_uint(t.y) << 23)));
+}
+
+// Of every 8 score pairs of a row, this many take the software exp2.
+#ifndef DCA_EXP2_POLY_PAIRS
+#define DCA_EXP2_POLY_PAIRS 2
+#endif
+
 // Rotate one query row by the positions of table row `trow` and write it to
 // the 128-byte-swizzled K-major operand tile (two 16 KiB column blocks: dims
 // 0-63 and 64-127; RoPE pairs (k, k+64) sit at the same offset of each block).
 __device__ __forceinline__ void write_q_row(uint8_t* qb, int r, const __nv_bfloat16* qrow,
-                                            const float2* trow) {
+                                            const float2* trow, int c0 = 0, int c1 = 8) {
   const uint32_t row_off = static_cast<uint32_t>(r) * 128u;
 #pragma unroll
   for (int c = 0; c < 8; ++c) {
+    if (c < c0 || c >= c1) continue;
     uint4 oa = make_uint4(0, 0, 0, 0), ob = oa;
     if (qrow != nullptr) {
       const uint4 xa = *reinterpret_cast<const uint4*>(qrow + 8 * c);
@@ -120,13 +177,13 @@ __device__ __forceinline__ void write_q_row(uint8_t* qb, int r, const __nv_bfloa
   }
 }
 
-// Mask row i of a score tile (keys j0 .. j0+127) to the pairs that are causal
-// and belong to class `cls`.
-__device__ __forceinline__ void mask_row(uint32_t* sv, int64_t i, int64_t j0, int cls,
-                                         int64_t s) {
+// Mask NC consecutive scores of row i (keys j0 .. j0+NC-1) to the pairs that
+// are causal and belong to class `cls`.
+template <int NC>
+__device__ __forceinline__ void mask_cols(uint32_t* sv, int64_t i, int64_t j0, int cls, int64_t s) {
   const int64_t ni = i / s;
   const int64_t nj0 = j0 / s;
-  int64_t dn64 = ni - nj0;
+  const int64_t dn64 = ni - nj0;
   int dn = static_cast<int>(dn64 > (1 << 20) ? (1 << 20) : dn64);
   const int64_t b64 = (nj0 + 1) * s - j0;  // first column of the next chunk
   int bnd = static_cast<int>(b64 > (1 << 30) ? (1 << 30) : b64);
@@ -135,7 +192,7 @@ __device__ __forceinline__ void mask_row(uint32_t* sv, int64_t i, int64_t j0, in
   const int lim = static_cast<int>(lim64 > 1024 ? 1024 : (lim64 < -1 ? -1 : lim64));
   const uint32_t NEG_INF = 0xff800000u;
 #pragma unroll
-  for (int e = 0; e < BN; ++e) {
+  for (int e = 0; e < NC; ++e) {
     if (e >= bnd) {
       dn -= 1;
       bnd += s32;
@@ -143,6 +200,123 @@ __device__ __forceinline__ void mask_row(uint32_t* sv, int64_t i, int64_t j0, in
     const int ce = dn <= 0 ? CLS_INTRA : (dn == 1 ? CLS_SUCC : CLS_INTER);
     if (e > lim || ce != cls) sv[e] = NEG_INF;
   }
+}
+
+// Maximum of 64 scores: eight independent chains of three-input maxima.
+__device__ __forceinline__ float max64(const uint32_t* sv) {
+  float m8[8];
+#pragma unroll
+  for (int c = 0; c < 8; ++c) m8[c] = __uint_as_float(sv[c]);
+#pragma unroll
+  for (int e = 8; e < 64; e += 16) {
+#pragma unroll
+    for (int c = 0; c < 8; ++c)
+      m8[c] = max3f(m8[c], __uint_as_float(sv[e + c]),
+                    e + 8 + c < 64 ? __uint_as_float(sv[e + 8 + c]) : m8[c]);
+  }
+  return max3f(max3f(m8[0], m8[1], m8[2]), max3f(m8[3], m8[4], m8[5]), fmaxf(m8[6], m8[7]));
+}
+
+// Exchange one float with the thread that holds the other half of the same
+// row (same lane, warp +/- 4) through shared memory and the pair's mbarrier
+// (one arrival per warp).  Phase `ph` alternates two buffers: a thread can be
+// at most one exchange ahead of its partner, so a buffer is rewritten only
+// after the partner has read it.  Bounded like every wait of the kernel.
+struct PairCtx {
+  float* xval;      // [2][2][128]
+  uint64_t* bar;    // this lane quarter's pair barrier
+  uint32_t ph;      // exchanges done so far
+  int half, r, lane;
+};
+
+__device__ __forceinline__ bool pair_exchange(PairCtx& pc, float mine, float& other,
+                                              volatile int* abort, unsigned int* status,
+                                              uint64_t timeout_ns, unsigned int code) {
+  float* slot = pc.xval + (pc.ph & 1u) * 256u;
+  slot[pc.half * 128 + pc.r] = mine;
+  __syncwarp();
+  if (pc.lane == 0) mbar_arrive(pc.bar);
+  bool ok = wait_bounded(pc.bar, pc.ph & 1u, abort, status, timeout_ns, code);
+  ok = __all_sync(0xffffffffu, ok);
+  if (ok) other = slot[(1 - pc.half) * 128 + pc.r];
+  ++pc.ph;
+  return ok;
+}
+
+// Exponentials of 64 scores against the reference `mb` (= m_ref * sc):
+// P (bf16 pairs) into pk, their sum returned.
+__device__ __forceinline__ float exp_pack64(const uint32_t* sv, float sc, float mb, uint32_t* pk) {
+  const float2 sc2 = make_float2(sc, sc);
+  const float2 nmb2 = make_float2(-mb, -mb);
+  float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                   make_float2(0.f, 0.f)};
+#pragma unroll
+  for (int e = 0; e < 32; ++e) {
+    float2 x = fma2(make_float2(__uint_as_float(sv[2 * e]), __uint_as_float(sv[2 * e + 1])), sc2,
+                    nmb2);
+    if ((e & 7) < DCA_EXP2_POLY_PAIRS) {
+      x = exp2_poly2(x);
+    } else {
+      x.x = ex2_approx(x.x);
+      x.y = ex2_approx(x.y);
+    }
+    acc[e & 3] = add2(acc[e & 3], x);
+    pk[e] = pack_bf16(x.x, x.y);
+  }
+  const float2 a = add2(add2(acc[0], acc[1]), add2(acc[2], acc[3]));
+  return a.x + a.y;
+}
+
+// One online-softmax step for HALF of a query row: this thread owns keys
+// [64*half, 64*half + 64) of the scores in TMEM columns tS..tS+127; the thread
+// holding the other half (same TMEM lane, warp +/- 4) exchanges its partial
+// maximum through pair_exchange.  Writes P (bf16) for its keys into columns
+// tS + 32*half .. +31 (scores both halves have read: the exchange orders both
+// loads before either store), keeps its partial row sum, and rescales its half
+// of O (tO) when the row maximum moved more than 2^RESCALE_LOG2 above the
+// reference (otherwise P may reach 2^8, exact in fp32 and in bf16's exponent
+// range; the final O / l uses the same reference).  O holds items < n: their
+// MMAs completed before S(n) did (one commit tracks all earlier MMAs).
+__device__ __forceinline__ bool softmax_half_step(uint32_t tS, uint32_t tO, int n, bool full,
+                                                  int64_t i, int kt, int cls, int64_t s, float sc,
+                                                  float& m_ref, float& l_sum, PairCtx& pc,
+                                                  volatile int* abort, unsigned int* status,
+                                                  uint64_t timeout_ns, unsigned int code) {
+  const int half = pc.half;
+  uint32_t sv[64];
+  tmem_ld64(tS + 64u * half, sv);
+  if (!full) mask_cols<64>(sv, i, static_cast<int64_t>(kt) * BN + 64 * half, cls, s);
+  float mx = max64(sv);
+  float mx_other = -INFINITY;
+  if (!pair_exchange(pc, mx, mx_other, abort, status, timeout_ns, code)) return false;
+  mx = fmaxf(mx, mx_other);
+
+  const float m_new = fmaxf(m_ref, mx);
+  const bool need =
+      (m_new > m_ref) && (m_ref == -INFINITY || (m_new - m_ref) * sc > RESCALE_LOG2);
+  float alpha = 1.f;
+  if (need) {
+    alpha = (m_ref == -INFINITY) ? 0.f : ex2_approx((m_ref - m_new) * sc);
+    m_ref = m_new;
+    l_sum *= alpha;
+  }
+  uint32_t pk[32];
+  l_sum += exp_pack64(sv, sc, (m_ref == -INFINITY) ? 0.f : m_ref * sc, pk);
+  tmem_st32(tS + 32u * half, pk);
+  // TMEM access is warp-collective: rescale when any row of the warp needs it
+  // (rows whose max did not move use alpha = 1)
+  if (n > 0 && __any_sync(0xffffffffu, need)) {
+#pragma unroll
+    for (int c = 0; c < 2; ++c) {
+      uint32_t o[32];
+      tmem_ld32(tO + 64u * half + 32u * c, o);
+#pragma unroll
+      for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+      tmem_st32(tO + 64u * half + 32u * c, o);
+    }
+  }
+  tmem_st_wait();
+  return true;
 }
 
 __global__ void __launch_bounds__(NUM_THREADS, 1)
@@ -172,6 +346,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const int64_t i_last = (i0 + BM - 1 < q_end - 1) ? i0 + BM - 1 : q_end - 1;
   const int64_t i_hi = i0 + BM - 1;
   const TilePlan plan = make_plan(i0, i_last, p.s, BN);
+  const FullRanges fullr = make_full_ranges(i0, i_hi, p.s, BN);
   const int N = plan.n_items;
 
   if (threadIdx.x == 0) {
@@ -181,11 +356,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
     for (int st = 0; st < 2; ++st) {
       mbar_init(&ctl->s_full[st], 1);
-      mbar_init(&ctl->p_full[st], 128);
-      mbar_init(&ctl->q_ready[st], 128);
+      mbar_init(&ctl->p_full[st], 8);   // one arrival per softmax warp
+      mbar_init(&ctl->q_ready[st], 8);
       mbar_init(&ctl->o_final[st], 1);
     }
     mbar_init(&ctl->drain, 1);
+    for (int k = 0; k < 4; ++k) mbar_init(&ctl->pair_bar[k], 2);
     ctl->abort = 0;
     fence_barrier_init();
   }
@@ -205,123 +381,114 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 
   if (warp < 8) {
     // =========================================================== softmax
-    const int stage = warp >> 2;
+    // All 8 warps work on head A's scores, then on head B's, for every item:
+    // warp w and warp w+4 share TMEM lanes 32*(w%4).. (one query row per lane)
+    // and split each row's 128 keys in two halves.  Two warps per SM
+    // sub-partition keep its MUFU/FMA pipes busy on the current head while the
+    // tensor cores run the other head's MMAs.
+    const int half = warp >> 2;
     const int sub = warp & 3;
     const int r = sub * 32 + lane;
+    PairCtx pc;
+    pc.xval = &ctl->xval[0][0][0];
+    pc.bar = &ctl->pair_bar[sub];
+    pc.ph = 0;
+    pc.half = half;
+    pc.r = r;
+    pc.lane = lane;
     const int64_t i = i0 + r;
     const bool real = i <= i_last;
-    if (stage == 0 || two) {
-      uint8_t* qb = stage ? q_buf1 : q_buf0;
-      const int h = h0 + stage;
-      const uint32_t lane_off = static_cast<uint32_t>(sub * 32) << 16;
-      const uint32_t tS = tbase + lane_off + static_cast<uint32_t>(stage * 128);
-      const uint32_t tO = tbase + lane_off + 256u + static_cast<uint32_t>(stage * 128);
-      const __nv_bfloat16* qrow =
-          real ? p.q + ((i - p.q_start) * p.Hq + h) * static_cast<int64_t>(HD) : nullptr;
-      const float sc = p.scale_log2;
+    const uint32_t lane_off = static_cast<uint32_t>(sub * 32) << 16;
+    const float sc = p.scale_log2;
+    const __nv_bfloat16* qrow0 =
+        real ? p.q + ((i - p.q_start) * p.Hq + h0) * static_cast<int64_t>(HD) : nullptr;
+    const __nv_bfloat16* qrow1 = (real && two) ? qrow0 + HD : nullptr;  // head h0 + 1
+    const int c0 = 4 * half, c1 = 4 * half + 4;  // this thread's share of the Q row
 
-      int kt, cls;
-      plan_item(plan, 0, kt, cls);
-      write_q_row(qb, r, qrow,
-                  real ? p.tab + query_table_row(i, cls, p.s, p.w, p.tab_c1) * 64 : nullptr);
+    int kt, cls;
+    plan_item(plan, 0, kt, cls);
+    {
+      const float2* trow = real ? p.tab + query_table_row(i, cls, p.s, p.w, p.tab_c1) * 64 : nullptr;
+      write_q_row(q_buf0, r, qrow0, trow, c0, c1);
+      if (two) write_q_row(q_buf1, r, qrow1, trow, c0, c1);
       fence_proxy_async_smem();
-      mbar_arrive(&ctl->q_ready[stage]);
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(&ctl->q_ready[0]);
+        if (two) mbar_arrive(&ctl->q_ready[1]);
+      }
+    }
 
-      float m_ref = -INFINITY;
-      float l_sum = 0.f;
-      bool ok = true;
-      for (int n = 0; n < N; ++n) {
-        plan_item(plan, n, kt, cls);
-        ok = wait_bounded(&ctl->s_full[stage], static_cast<uint32_t>(n & 1), abort_flag,
-                          p.status, p.timeout_ns, ST_SOFTMAX << stage);
+    float m_ref[2] = {-INFINITY, -INFINITY};
+    float l_sum[2] = {0.f, 0.f};
+    bool ok = true;
+    for (int n = 0; n < N && ok; ++n) {
+      plan_item(plan, n, kt, cls);
+      const bool full = is_full(fullr, kt, cls);
+      int cls_next = cls;
+      if (n + 1 < N) {
+        int kt_next;
+        plan_item(plan, n + 1, kt_next, cls_next);
+      }
+#pragma unroll
+      for (int st = 0; st < 2; ++st) {
+        if (st == 1 && !two) break;
+        ok = wait_bounded(&ctl->s_full[st], static_cast<uint32_t>(n & 1), abort_flag, p.status,
+                          p.timeout_ns, ST_SOFTMAX << st);
         ok = __all_sync(0xffffffffu, ok);
         if (!ok) break;
         tc_fence_after();
-
-        uint32_t sv[BN];
-#pragma unroll
-        for (int c = 0; c < 4; ++c) tmem_ld32(tS + 32u * c, sv + 32 * c);
-        const int64_t j0 = static_cast<int64_t>(kt) * BN;
-        if (!item_is_full(i0, i_hi, j0, j0 + BN - 1, p.s, cls)) mask_row(sv, i, j0, cls, p.s);
-
-        float mx = -INFINITY;
-#pragma unroll
-        for (int e = 0; e < BN; ++e) mx = fmaxf(mx, __uint_as_float(sv[e]));
-        const float m_new = fmaxf(m_ref, mx);
-        const bool need =
-            (m_new > m_ref) && (m_ref == -INFINITY || (m_new - m_ref) * sc > RESCALE_LOG2);
-        float alpha = 1.f;
-        if (need) {
-          alpha = (m_ref == -INFINITY) ? 0.f : ex2_approx((m_ref - m_new) * sc);
-          m_ref = m_new;
-          l_sum *= alpha;
-        }
-        const float mb = (m_ref == -INFINITY) ? 0.f : m_ref * sc;
-        float rs = 0.f;
-#pragma unroll
-        for (int hlf = 0; hlf < 2; ++hlf) {
-          uint32_t pk[32];
-#pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            const float a = ex2_approx(fmaf(__uint_as_float(sv[64 * hlf + 2 * e]), sc, -mb));
-            const float b = ex2_approx(fmaf(__uint_as_float(sv[64 * hlf + 2 * e + 1]), sc, -mb));
-            rs += a + b;
-            pk[e] = pack_bf16(a, b);
-          }
-          tmem_st32(tS + 32u * hlf, pk);
-        }
-        l_sum += rs;
-        // O still holds items < n (their MMAs completed before S(n) did); rescale
-        // it before P(n) V(n) accumulates onto it.  Warp-uniform (TMEM access is
-        // warp-collective); rows whose max did not move use alpha = 1.
-        if (n > 0 && __any_sync(0xffffffffu, need)) {
-#pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            uint32_t o[32];
-            tmem_ld32(tO + 32u * c, o);
-#pragma unroll
-            for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-            tmem_st32(tO + 32u * c, o);
-          }
-        }
-        tmem_st_wait();
-        if (n + 1 < N) {
-          int kt2, cls2;
-          plan_item(plan, n + 1, kt2, cls2);
-          if (cls2 != cls) {  // phase switch: next items need another query rotation
-            write_q_row(qb, r, qrow,
-                        real ? p.tab + query_table_row(i, cls2, p.s, p.w, p.tab_c1) * 64
-                             : nullptr);
-            fence_proxy_async_smem();
-          }
+        const uint32_t tS = tbase + lane_off + static_cast<uint32_t>(st * 128);
+        const uint32_t tO = tbase + lane_off + 256u + static_cast<uint32_t>(st * 128);
+        ok = softmax_half_step(tS, tO, n, full, i, kt, cls, p.s, sc, m_ref[st], l_sum[st], pc,
+                               abort_flag, p.status, p.timeout_ns, ST_SOFTMAX << st);
+        if (!ok) break;
+        if (cls_next != cls) {  // phase switch: the next items need another query rotation
+          write_q_row(st ? q_buf1 : q_buf0, r, st ? qrow1 : qrow0,
+                      real ? p.tab + query_table_row(i, cls_next, p.s, p.w, p.tab_c1) * 64
+                           : nullptr,
+                      c0, c1);
+          fence_proxy_async_smem();
         }
         tc_fence_before();
-        mbar_arrive(&ctl->p_full[stage]);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&ctl->p_full[st]);
       }
+    }
+    // epilogue: O / (l_half0 + l_half1) -> bf16 -> out (each thread writes its 64 columns)
+#pragma unroll
+    for (int st = 0; st < 2; ++st) {
+      if (st == 1 && !two) break;
       if (ok) {
-        ok = wait_bounded(&ctl->o_final[stage], 0u, abort_flag, p.status, p.timeout_ns,
-                          ST_SOFTMAX << stage);
+        ok = wait_bounded(&ctl->o_final[st], 0u, abort_flag, p.status, p.timeout_ns,
+                          ST_SOFTMAX << st);
         ok = __all_sync(0xffffffffu, ok);
       }
-      if (ok) {
-        tc_fence_after();
-        const float inv = 1.f / l_sum;
-        __nv_bfloat16* orow =
-            real ? p.out + ((i - p.q_start) * p.Hq + h) * static_cast<int64_t>(HD) : nullptr;
+      if (!ok) break;
+      float l_other = 0.f;
+      ok = pair_exchange(pc, l_sum[st], l_other, abort_flag, p.status, p.timeout_ns,
+                         ST_SOFTMAX << st);
+      if (!ok) break;
+      const float l_tot = l_sum[st] + l_other;
+      tc_fence_after();
+      const uint32_t tO = tbase + lane_off + 256u + static_cast<uint32_t>(st * 128) + 64u * half;
+      const float inv = 1.f / l_tot;
+      __nv_bfloat16* orow =
+          real ? p.out + ((i - p.q_start) * p.Hq + h0 + st) * static_cast<int64_t>(HD) + 64 * half
+               : nullptr;
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          uint32_t o[32];
-          tmem_ld32(tO + 32u * c, o);
-          if (real) {
+      for (int c = 0; c < 2; ++c) {
+        uint32_t o[32];
+        tmem_ld32(tO + 32u * c, o);
+        if (real) {
 #pragma unroll
-            for (int v4 = 0; v4 < 4; ++v4) {
-              uint4 w4;
-              w4.x = pack_bf16(__uint_as_float(o[8 * v4 + 0]) * inv, __uint_as_float(o[8 * v4 + 1]) * inv);
-              w4.y = pack_bf16(__uint_as_float(o[8 * v4 + 2]) * inv, __uint_as_float(o[8 * v4 + 3]) * inv);
-              w4.z = pack_bf16(__uint_as_float(o[8 * v4 + 4]) * inv, __uint_as_float(o[8 * v4 + 5]) * inv);
-              w4.w = pack_bf16(__uint_as_float(o[8 * v4 + 6]) * inv, __uint_as_float(o[8 * v4 + 7]) * inv);
-              *reinterpret_cast<uint4*>(orow + 32 * c + 8 * v4) = w4;
-            }
+          for (int v4 = 0; v4 < 4; ++v4) {
+            uint4 w4;
+            w4.x = pack_bf16(__uint_as_float(o[8 * v4 + 0]) * inv, __uint_as_float(o[8 * v4 + 1]) * inv);
+            w4.y = pack_bf16(__uint_as_float(o[8 * v4 + 2]) * inv, __uint_as_float(o[8 * v4 + 3]) * inv);
+            w4.z = pack_bf16(__uint_as_float(o[8 * v4 + 4]) * inv, __uint_as_float(o[8 * v4 + 5]) * inv);
+            w4.w = pack_bf16(__uint_as_float(o[8 * v4 + 6]) * inv, __uint_as_float(o[8 * v4 + 7]) * inv);
+            *reinterpret_cast<uint4*>(orow + 32 * c + 8 * v4) = w4;
           }
         }
       }
@@ -361,35 +528,40 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                      p.status, p.timeout_ns, ST_DRAIN);
     }
     __syncwarp();
-  } else {
+  } else if (warp == WARP_MMA) {
     // =========================================================== MMA issuer
     if (lane == 0) {
       const uint32_t id_s = idesc_bf16_f32(BM, BN, false);
       const uint32_t id_o = idesc_bf16_f32(BM, HD, true);
       const uint32_t q_addr[2] = {smem_u32(q_buf0), smem_u32(q_buf1)};
       const uint32_t slot_addr0 = smem_u32(slots);
+      // Descriptors are built once; a k-step only adds its byte offset / 16 to
+      // the start-address field (no carry out of the 14-bit field: shared
+      // memory addresses stay below 256 KiB).
+      const uint64_t dq[2] = {sdesc_sw128(q_addr[0], 16, 1024), sdesc_sw128(q_addr[1], 16, 1024)};
+      const uint64_t dk0 = sdesc_sw128(slot_addr0, 16, 1024);
+      const uint64_t dv0 = sdesc_sw128(slot_addr0, HALF_BYTES, 1024);
       auto issue_s = [&](int st, int li) {
-        const uint32_t kb = slot_addr0 + static_cast<uint32_t>((li % NSLOT) * TILE_BYTES);
+        const uint64_t dk = dk0 + static_cast<uint64_t>(((li % NSLOT) * TILE_BYTES) >> 4);
 #pragma unroll
         for (int kk = 0; kk < HD / 16; ++kk) {
-          const uint32_t off = static_cast<uint32_t>((kk >> 2) * HALF_BYTES + (kk & 3) * 32);
-          mma_ss(tbase + static_cast<uint32_t>(st * 128), sdesc_sw128(q_addr[st] + off, 16, 1024),
-                 sdesc_sw128(kb + off, 16, 1024), id_s, kk > 0 ? 1u : 0u);
+          const uint64_t off = static_cast<uint64_t>(((kk >> 2) * HALF_BYTES + (kk & 3) * 32) >> 4);
+          mma_ss(tbase + static_cast<uint32_t>(st * 128), dq[st] + off, dk + off, id_s,
+                 kk > 0 ? 1u : 0u);
         }
       };
       auto issue_pv = [&](int st, int li, bool acc) {
-        const uint32_t vb = slot_addr0 + static_cast<uint32_t>((li % NSLOT) * TILE_BYTES);
+        const uint64_t dv = dv0 + static_cast<uint64_t>(((li % NSLOT) * TILE_BYTES) >> 4);
 #pragma unroll
         for (int kk = 0; kk < BN / 16; ++kk) {
           mma_ts(tbase + 256u + static_cast<uint32_t>(st * 128),
                  tbase + static_cast<uint32_t>(st * 128 + kk * 8),
-                 sdesc_sw128(vb + static_cast<uint32_t>(kk * 2048), HALF_BYTES, 1024), id_o,
-                 (acc || kk > 0) ? 1u : 0u);
+                 dv + static_cast<uint64_t>((kk * 2048) >> 4), id_o, (acc || kk > 0) ? 1u : 0u);
         }
       };
       auto full_wait = [&](int li) {
-        return wait_bounded(&ctl->slot_full[li % NSLOT], static_cast<uint32_t>((li / NSLOT) & 1),
-                            abort_flag, p.status, p.timeout_ns, ST_MMA);
+        return DCA_MMA_WAIT(&ctl->slot_full[li % NSLOT], static_cast<uint32_t>((li / NSLOT) & 1),
+                         abort_flag, p.status, p.timeout_ns, ST_MMA);
       };
 
       bool ok = wait_bounded(&ctl->q_ready[0], 0u, abort_flag, p.status, p.timeout_ns, ST_MMA);
@@ -411,7 +583,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const bool more = n + 1 < N;
         ok = full_wait(lv);
         if (!ok) break;
-        ok = wait_bounded(&ctl->p_full[0], static_cast<uint32_t>(n & 1), abort_flag, p.status,
+        ok = DCA_MMA_WAIT(&ctl->p_full[0], static_cast<uint32_t>(n & 1), abort_flag, p.status,
                           p.timeout_ns, ST_MMA);
         if (!ok) break;
         tc_fence_after();
@@ -424,7 +596,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           mma_commit(&ctl->s_full[0]);
         }
         if (two) {
-          ok = wait_bounded(&ctl->p_full[1], static_cast<uint32_t>(n & 1), abort_flag, p.status,
+          ok = DCA_MMA_WAIT(&ctl->p_full[1], static_cast<uint32_t>(n & 1), abort_flag, p.status,
                             p.timeout_ns, ST_MMA);
           if (!ok) break;
           tc_fence_after();

@@ -92,6 +92,46 @@ DCA_HD bool item_is_full(int64_t i0, int64_t i_hi, int64_t j0, int64_t j_hi, int
   return ni0 == ni1 && nj0 == nj1 && ni0 == nj0 && j_hi <= i0;
 }
 
+// Per class, the k-tiles [lo, hi) that need no mask for the query tile whose
+// rows are [i0, i_hi] (same predicate as item_is_full, solved for kt once per
+// tile so the kernels avoid per-item 64-bit divisions).
+struct FullRanges {
+  int lo[3];
+  int hi[3];
+};
+
+DCA_HD int64_t floor_div64(int64_t a, int64_t b) { return a >= 0 ? a / b : -((-a + b - 1) / b); }
+
+DCA_HD FullRanges make_full_ranges(int64_t i0, int64_t i_hi, int64_t s, int bn) {
+  FullRanges F;
+  const int64_t ni0 = i0 / s, ni1 = i_hi / s;
+  // INTER: j_hi < s*(ni0-1)  <=>  (kt+1)*bn <= s*(ni0-1)
+  F.lo[CLS_INTER] = 0;
+  F.hi[CLS_INTER] = ni0 >= 1 ? static_cast<int>(floor_div64(s * (ni0 - 1), bn)) : 0;
+  // SUCC: j_hi < s*ni0 and j0 >= s*(ni1-1)
+  {
+    const int64_t lo = ni1 >= 1 ? cdiv64(s * (ni1 - 1), bn) : 0;
+    const int64_t hi = floor_div64(s * ni0, bn);
+    F.lo[CLS_SUCC] = static_cast<int>(lo);
+    F.hi[CLS_SUCC] = static_cast<int>(hi > lo ? hi : lo);
+  }
+  // INTRA: one chunk for all rows, j0 >= s*ni0, j_hi < s*(ni0+1), j_hi <= i0
+  if (ni0 == ni1) {
+    const int64_t lo = cdiv64(s * ni0, bn);
+    const int64_t end = (s * (ni0 + 1) < i0 + 1) ? s * (ni0 + 1) : i0 + 1;
+    const int64_t hi = floor_div64(end, bn);
+    F.lo[CLS_INTRA] = static_cast<int>(lo);
+    F.hi[CLS_INTRA] = static_cast<int>(hi > lo ? hi : lo);
+  } else {
+    F.lo[CLS_INTRA] = F.hi[CLS_INTRA] = 0;
+  }
+  return F;
+}
+
+DCA_HD bool is_full(const FullRanges& F, int kt, int cls) {
+  return kt >= F.lo[cls] && kt < F.hi[cls];
+}
+
 // Position (row of the RoPE table) by which query row i is rotated in class
 // `cls`.  The table stores positions [0, min(s, cap)) directly, positions
 // [s, s + w) directly when cap > s, and position c - 1 at row `tab_c1`.
