@@ -56,6 +56,9 @@ def parse_args(argv=None):
                     help="approximate CPU seconds for the oracle baseline sample")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--record-traffic", metavar="NCU_CSV",
+                    help="store the attention kernel's DRAM bytes per launch from an ncu CSV "
+                         "capture of --workload, then exit")
     return ap.parse_args(argv)
 
 
@@ -71,6 +74,65 @@ def load_peaks():
     except (OSError, KeyError, ValueError):
         return dict(bf16_tflops=1590.0, bf16_tflops_sustained=1400.0, hbm_gbs=6650.0,
                     source="fallback")
+
+
+KERNEL_SOURCES = ["length_extrapolation_b200/csrc/dca_fwd_sm100.cu",
+                  "length_extrapolation_b200/csrc/sm100_ptx.cuh",
+                  "length_extrapolation_b200/csrc/dca_plan.cuh"]
+TRAFFIC_RECORD = os.path.join(ROOT, "profiles", "dca_fwd_kernel_traffic.json")
+
+
+def kernel_source_hash():
+    import hashlib
+    h = hashlib.sha256()
+    for rel in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
+def recorded_traffic(workload: str):
+    """Average DRAM bytes (read + write) per attention launch from an ncu capture
+    of this workload, or None when there is none for the current kernel source."""
+    try:
+        with open(TRAFFIC_RECORD) as f:
+            rec = json.load(f)
+    except (OSError, ValueError):
+        return None
+    ent = rec.get(workload)
+    if not ent or ent.get("source_sha256") != kernel_source_hash():
+        return None
+    return ent.get("bytes_per_launch")
+
+
+def write_traffic_record(workload: str, ncu_csv: str):
+    """Store the average DRAM bytes per attention launch of an ncu CSV capture
+    (metrics dram__bytes_read.sum, dram__bytes_write.sum) under the current
+    kernel source hash."""
+    import csv
+    rows = list(csv.reader(open(ncu_csv)))
+    hdr, per = None, {}
+    for r in rows:
+        if r and r[0] == "ID":
+            hdr = r
+            continue
+        if hdr and len(r) == len(hdr):
+            d = dict(zip(hdr, r))
+            if "dca_fwd_kernel" not in d["Kernel Name"] or not d["Metric Name"].startswith("dram__bytes"):
+                continue
+            scale = {"byte": 1, "Kbyte": 1e3, "Mbyte": 1e6, "Gbyte": 1e9}[d["Metric Unit"]]
+            per[d["ID"]] = per.get(d["ID"], 0.0) + float(d["Metric Value"].replace(",", "")) * scale
+    if not per:
+        raise SystemExit("no dca_fwd_kernel dram__bytes rows in " + ncu_csv)
+    rec = {}
+    if os.path.exists(TRAFFIC_RECORD):
+        with open(TRAFFIC_RECORD) as f:
+            rec = json.load(f)
+    rec[workload] = {"bytes_per_launch": sum(per.values()) / len(per), "launches": len(per),
+                     "source_sha256": kernel_source_hash()}
+    with open(TRAFFIC_RECORD, "w") as f:
+        json.dump(rec, f, indent=1)
+    print(json.dumps({workload: rec[workload]}))
 
 
 def causal_pairs(q0, lq):
@@ -254,6 +316,9 @@ def workload_config(w):
 def main(argv=None):
     args = parse_args(argv)
     w = WORKLOADS[args.workload]
+    if args.record_traffic:
+        write_traffic_record(w.name, args.record_traffic)
+        return 0
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
@@ -321,7 +386,11 @@ def main(argv=None):
         "peak_kind": f"{peaks['source']} sustained bf16 (cuBLAS, power-capped loop)",
         "frac_of_burst_peak": achieved / peaks["bf16_tflops"],
         "frac_of_datasheet_2250": achieved / 2250.0,
-        "traffic": None,
+        "traffic": recorded_traffic(w.name),
+        "traffic_unit": "bytes per launch (dram read + write, ncu)",
+        "algorithmic_bytes_per_launch": sum(
+            (2 * lq * w.Hq + 2 * lk * w.Hkv) * w.d * q.element_size() for q0, lq, lk in blocks)
+            / len(blocks),
         "launches_per_step": len(blocks),
         "avg_launch_ms": attn_ms_max / (args.steps * len(blocks)),
     }

@@ -64,6 +64,15 @@ constexpr int NUM_THREADS = 320;
 constexpr int WARP_LOAD = 8;
 constexpr int WARP_MMA = 9;
 constexpr float RESCALE_LOG2 = 8.0f;
+// How the softmax threads wait for the partner's half-row maximum and for S:
+// polling (no suspension) -- both are on the critical path of every item, and
+// a suspended thread wakes up hundreds of cycles after the phase completes.
+#ifndef DCA_PAIR_WAIT
+#define DCA_PAIR_WAIT wait_poll
+#endif
+#ifndef DCA_S_WAIT
+#define DCA_S_WAIT wait_poll
+#endif
 // How the MMA issuer waits: polling with a short back-off (wait_spin) or a
 // suspending try_wait (wait_bounded).
 #ifndef DCA_MMA_WAIT
@@ -236,7 +245,7 @@ __device__ __forceinline__ bool pair_exchange(PairCtx& pc, float mine, float& ot
   slot[pc.half * 128 + pc.r] = mine;
   __syncwarp();
   if (pc.lane == 0) mbar_arrive(pc.bar);
-  bool ok = wait_bounded(pc.bar, pc.ph & 1u, abort, status, timeout_ns, code);
+  bool ok = DCA_PAIR_WAIT(pc.bar, pc.ph & 1u, abort, status, timeout_ns, code);
   ok = __all_sync(0xffffffffu, ok);
   if (ok) other = slot[(1 - pc.half) * 128 + pc.r];
   ++pc.ph;
@@ -333,10 +342,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
-  // ---- work unit (longest causal rows first)
-  const int units_per_qt = p.Hkv * p.n_pairs;
-  const int qt = p.n_qtiles - 1 - static_cast<int>(blockIdx.x / units_per_qt);
-  const int u = static_cast<int>(blockIdx.x % units_per_qt);
+  // ---- work unit
+  // KV-group-major order: the CTAs running together stream the same group's
+  // K'/V tiles (shared in L2); within a group, longest query tiles first.
+  const int per_group = p.n_qtiles * p.n_pairs;
+  const int u = (static_cast<int>(blockIdx.x) / per_group) * p.n_pairs +
+                static_cast<int>(blockIdx.x % per_group) % p.n_pairs;
+  const int qt = p.n_qtiles - 1 - static_cast<int>((blockIdx.x % per_group) / p.n_pairs);
   const int g = u / p.n_pairs;
   const int pr = u % p.n_pairs;
   const int h0 = g * p.G + 2 * pr;
@@ -433,8 +445,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 #pragma unroll
       for (int st = 0; st < 2; ++st) {
         if (st == 1 && !two) break;
-        ok = wait_bounded(&ctl->s_full[st], static_cast<uint32_t>(n & 1), abort_flag, p.status,
-                          p.timeout_ns, ST_SOFTMAX << st);
+        ok = DCA_S_WAIT(&ctl->s_full[st], static_cast<uint32_t>(n & 1), abort_flag, p.status,
+                        p.timeout_ns, ST_SOFTMAX << st);
         ok = __all_sync(0xffffffffu, ok);
         if (!ok) break;
         tc_fence_after();

@@ -105,6 +105,25 @@ __device__ __forceinline__ bool wait_spin(uint64_t* bar, uint32_t parity, volati
   }
 }
 
+// Polling wait without back-off (bounded like wait_bounded).
+__device__ __forceinline__ bool wait_poll(uint64_t* bar, uint32_t parity, volatile int* abort,
+                                          unsigned int* status, uint64_t timeout_ns,
+                                          unsigned int code) {
+  if (mbar_test_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  for (uint32_t it = 1;; ++it) {
+    if (mbar_test_wait(bar, parity)) return true;
+    if ((it & 15u) == 0) {
+      if (*abort) return false;
+      if (globaltimer_ns() - t0 > timeout_ns) {
+        *abort = 1;
+        atomicOr(status, code);
+        return false;
+      }
+    }
+  }
+}
+
 // Warp-wide wait: lane 0 polls without suspending (prompt wake-up, one lane's
 // worth of issue slots), then every lane observes the completed phase itself
 // (acquire) before touching the data it guards.  Returns the same value in
