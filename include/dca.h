@@ -50,6 +50,26 @@ extern "C" {
 
 typedef enum { DCA_BF16 = 0, DCA_F32 = 1 } dca_dtype;
 
+/*
+ * Reading of the local window of successive-chunk attention ("Qwen2.5-1M
+ * 不重训外推 1M", section Successive-Chunk Attention: pairs inside the window
+ * keep their true relative position, the others fall back to the inter-chunk
+ * rule; the page does not say what the window is measured on).
+ *   DCA_WINDOW_QUERY_OFFSET  (default) the pair (i, j) of adjacent chunks keeps
+ *                            its true distance when the query's offset in its
+ *                            chunk r_i < w;
+ *   DCA_WINDOW_TRUE_DISTANCE it keeps its true distance when i - j < w.
+ * Either way a kept distance is the true i - j and every other adjacent-chunk
+ * pair uses query position c - 1 against key position j mod s.
+ */
+typedef enum { DCA_WINDOW_QUERY_OFFSET = 0, DCA_WINDOW_TRUE_DISTANCE = 1 } dca_window_reading;
+
+/* Options of the _ex entry points (NULL means all defaults; reserved must be 0). */
+typedef struct {
+  int32_t window_reading; /* dca_window_reading */
+  int32_t reserved[7];
+} dca_options;
+
 typedef enum {
   DCA_OK = 0,
   DCA_ERR_ARG = -1,         /* bad size, pointer, alignment or parameter       */
@@ -104,6 +124,14 @@ int dca_prefill_chunked(const void* q_block, const void* k_cache, const void* v_
                         int64_t pretrain_window, double rope_base, double yarn_scale,
                         int dtype, void* workspace, size_t ws_bytes, void* cuda_stream);
 
+/* dca_prefill_chunked with options (window reading).  DCA_ERR_ARG for invalid options. */
+int dca_prefill_chunked_ex(const void* q_block, const void* k_cache, const void* v_cache,
+                           void* out_block, int64_t q_start, int64_t Lq, int64_t Lk, int Hq,
+                           int Hkv, int d, int64_t chunk_size, int64_t local_window,
+                           int64_t pretrain_window, double rope_base, double yarn_scale,
+                           int dtype, const dca_options* opts, void* workspace, size_t ws_bytes,
+                           void* cuda_stream);
+
 /*
  * Stage 1 of a prefill call: build the RoPE table and rotate keys
  * [k_rows_valid, Lk) of k_cache into the workspace.  k_rows_valid = 0 rebuilds
@@ -126,6 +154,12 @@ int dca_attend(const void* q_block, const void* v_cache, void* out_block, int64_
                int64_t Lq, int64_t Lk, int Hq, int Hkv, int d, int64_t chunk_size,
                int64_t local_window, int64_t pretrain_window, double yarn_scale, int dtype,
                void* workspace, size_t ws_bytes, void* cuda_stream);
+
+/* dca_attend with options (window reading).  DCA_ERR_ARG for invalid options. */
+int dca_attend_ex(const void* q_block, const void* v_cache, void* out_block, int64_t q_start,
+                  int64_t Lq, int64_t Lk, int Hq, int Hkv, int d, int64_t chunk_size,
+                  int64_t local_window, int64_t pretrain_window, double yarn_scale, int dtype,
+                  const dca_options* opts, void* workspace, size_t ws_bytes, void* cuda_stream);
 
 /*
  * Device-side status: synchronises `cuda_stream`, reads and clears the status
@@ -157,15 +191,19 @@ int dca_prefill_host(const void* q_h, const void* k_h, const void* v_h, void* ou
 /*
  * Host-side introspection of the tile plan the attention kernels follow
  * (no GPU needed).  For the query tile whose rows are [i0, i0 + tile_rows)
- * with real rows up to i_last, and key tiles of `bn` keys, writes up to
+ * with real rows up to i_last, key tiles of `bn` keys, local window
+ * `local_window` and window reading `window_reading`, writes up to
  * `max_items` triples (k_tile, class, full) in work-list order: class 2 =
- * inter-chunk, 1 = successive chunk, 0 = intra-chunk (the three parts of the
+ * inter-chunk rule (query position c - 1), 1 = successive chunk with its true
+ * distance kept (under the query-offset reading: every adjacent-chunk pair,
+ * the row choosing s + r_i or c - 1), 0 = intra-chunk (the three parts of the
  * score matrix in section 核心思想 of "Qwen2.5-1M 不重训外推 1M"); full = 1
  * when every pair of the tile is causal and of that class (no mask).
  * Returns the number of items (which may exceed max_items) or DCA_ERR_ARG.
  */
-int dca_plan_items(int64_t i0, int64_t i_last, int64_t tile_rows, int64_t chunk_size, int bn,
-                   int32_t* items, int max_items);
+int dca_plan_items(int64_t i0, int64_t i_last, int64_t tile_rows, int64_t chunk_size,
+                   int64_t local_window, int window_reading, int bn, int32_t* items,
+                   int max_items);
 
 /*
  * No-allocation one-shot prefill (an addition for integrators; the pages on

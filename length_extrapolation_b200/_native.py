@@ -14,6 +14,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(HERE, "libdca_b200.so")
 
 DCA_BF16, DCA_F32 = 0, 1
+DCA_WINDOW_QUERY_OFFSET, DCA_WINDOW_TRUE_DISTANCE = 0, 1
 DCA_OK, DCA_ERR_ARG, DCA_ERR_UNSUPPORTED, DCA_ERR_CUDA, DCA_ERR_WORKSPACE, DCA_ERR_TIMEOUT = (
     0, -1, -2, -3, -4, -5)
 
@@ -36,7 +37,11 @@ SIGNATURES = {
     "dca_host_arena_size": (_sz, [_i64, _i64, _i32, _i32, _i32, _i64, _i64, _i64, _i32]),
     "dca_prefill_host": (_i32, [_vp, _vp, _vp, _vp, _i64, _i64, _i32, _i32, _i32, _i64, _i64,
                                 _i64, _dbl, _dbl, _i32, _vp, _sz, _vp]),
-    "dca_plan_items": (_i32, [_i64, _i64, _i64, _i64, _i32, _vp, _i32]),
+    "dca_plan_items": (_i32, [_i64, _i64, _i64, _i64, _i64, _i32, _i32, _vp, _i32]),
+    "dca_prefill_chunked_ex": (_i32, [_vp, _vp, _vp, _vp, _i64, _i64, _i64, _i32, _i32, _i32, _i64,
+                                      _i64, _i64, _dbl, _dbl, _i32, _vp, _vp, _sz, _vp]),
+    "dca_attend_ex": (_i32, [_vp, _vp, _vp, _i64, _i64, _i64, _i32, _i32, _i32, _i64, _i64, _i64,
+                             _dbl, _i32, _vp, _vp, _sz, _vp]),
     "dca_prefill_noalloc": (_i32, [_vp, _vp, _vp, _vp, _i64, _i32, _i32, _i32, _i64, _i64, _i64,
                                    _dbl, _dbl, _i32, _vp]),
     "dca_set_wait_timeout_ns": (None, [_i64]),
@@ -45,6 +50,11 @@ SIGNATURES = {
 
 _lock = threading.Lock()
 _lib = None
+
+
+class DCAOptions(ctypes.Structure):
+    """Mirror of dca_options (include/dca.h)."""
+    _fields_ = [("window_reading", ctypes.c_int32), ("reserved", ctypes.c_int32 * 7)]
 
 
 class DCAError(RuntimeError):

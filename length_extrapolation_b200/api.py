@@ -5,6 +5,7 @@ stream; every step of the computation runs in the library's kernels.
 """
 from __future__ import annotations
 
+import ctypes
 from typing import Optional
 
 import torch
@@ -30,6 +31,19 @@ def _check_cuda(*ts):
 
 def _stream_ptr(device) -> int:
     return torch.cuda.current_stream(device).cuda_stream
+
+
+WINDOW_READINGS = {"query_offset": N.DCA_WINDOW_QUERY_OFFSET,
+                   "true_distance": N.DCA_WINDOW_TRUE_DISTANCE}
+
+
+def _options(window_reading):
+    """dca_options for a window reading ('query_offset' (default) or 'true_distance')."""
+    if window_reading not in WINDOW_READINGS:
+        raise ValueError(f"window_reading must be one of {sorted(WINDOW_READINGS)}")
+    o = N.DCAOptions()
+    o.window_reading = WINDOW_READINGS[window_reading]
+    return o
 
 
 def workspace_size(kv_capacity, Hq, Hkv, d, chunk_size, local_window, pretrain_window,
@@ -75,16 +89,18 @@ def _ws_for(ws: Optional[Workspace], Lk, Hq, Hkv, d, p, dtype, device) -> Worksp
 
 
 def prefill(q, k, v, *, chunk_size, local_window, pretrain_window, rope_base=1e7,
-            yarn_scale=1.0, out=None, workspace: Optional[Workspace] = None):
+            yarn_scale=1.0, out=None, workspace: Optional[Workspace] = None,
+            window_reading="query_offset"):
     """One-shot DCA prefill.  q [L,Hq,d], k, v [L,Hkv,d] (CUDA, bf16 or fp32)."""
     return prefill_chunked(q, k, v, q_start=0, chunk_size=chunk_size, local_window=local_window,
                            pretrain_window=pretrain_window, rope_base=rope_base,
-                           yarn_scale=yarn_scale, out=out, workspace=workspace)
+                           yarn_scale=yarn_scale, out=out, workspace=workspace,
+                           window_reading=window_reading)
 
 
 def prefill_chunked(q_block, k_cache, v_cache, *, q_start, chunk_size, local_window,
                     pretrain_window, rope_base=1e7, yarn_scale=1.0, kv_len=None, out=None,
-                    workspace: Optional[Workspace] = None):
+                    workspace: Optional[Workspace] = None, window_reading="query_offset"):
     """A query block (absolute rows q_start ..) against the KV cache rows [0, kv_len)."""
     _check_cuda(q_block, k_cache, v_cache)
     Lq, Hq, d = q_block.shape
@@ -97,11 +113,13 @@ def prefill_chunked(q_block, k_cache, v_cache, *, q_start, chunk_size, local_win
         out = torch.empty_like(q_block)
     p = dict(chunk_size=chunk_size, local_window=local_window, pretrain_window=pretrain_window)
     ws = _ws_for(workspace, Lk, Hq, Hkv, d, p, q_block.dtype, q_block.device)
-    rc = N.lib().dca_prefill_chunked(
+    opts = _options(window_reading)
+    rc = N.lib().dca_prefill_chunked_ex(
         q_block.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(), out.data_ptr(), int(q_start),
         Lq, Lk, Hq, Hkv, d, int(chunk_size), int(local_window), int(pretrain_window),
-        float(rope_base), float(yarn_scale), dt, ws.ptr, ws.nbytes, _stream_ptr(q_block.device))
-    N.check(rc, "dca_prefill_chunked")
+        float(rope_base), float(yarn_scale), dt, ctypes.byref(opts), ws.ptr, ws.nbytes,
+        _stream_ptr(q_block.device))
+    N.check(rc, "dca_prefill_chunked_ex")
     return out
 
 
@@ -117,16 +135,17 @@ def prepare(k_cache, *, kv_len, k_rows_valid, chunk_size, local_window, pretrain
 
 
 def attend(q_block, v_cache, out, *, q_start, kv_len, chunk_size, local_window, pretrain_window,
-           yarn_scale, workspace: Workspace):
+           yarn_scale, workspace: Workspace, window_reading="query_offset"):
     """Stage 2: the fused attention kernel over one query block."""
     _check_cuda(q_block, v_cache, out)
     Lq, Hq, d = q_block.shape
-    rc = N.lib().dca_attend(q_block.data_ptr(), v_cache.data_ptr(), out.data_ptr(), int(q_start),
-                            Lq, int(kv_len), Hq, v_cache.shape[1], d, int(chunk_size),
-                            int(local_window), int(pretrain_window), float(yarn_scale),
-                            _dtype_code(q_block), workspace.ptr, workspace.nbytes,
-                            _stream_ptr(q_block.device))
-    N.check(rc, "dca_attend")
+    opts = _options(window_reading)
+    rc = N.lib().dca_attend_ex(q_block.data_ptr(), v_cache.data_ptr(), out.data_ptr(),
+                               int(q_start), Lq, int(kv_len), Hq, v_cache.shape[1], d,
+                               int(chunk_size), int(local_window), int(pretrain_window),
+                               float(yarn_scale), _dtype_code(q_block), ctypes.byref(opts),
+                               workspace.ptr, workspace.nbytes, _stream_ptr(q_block.device))
+    N.check(rc, "dca_attend_ex")
 
 
 def host_arena_size(L, block, Hq, Hkv, d, chunk_size, local_window, pretrain_window, dtype):

@@ -101,7 +101,7 @@ int prepare_impl(const void* k_cache, int64_t Lk, int64_t k_rows_valid, int Hkv,
 
 int attend_impl(const void* q, const void* v, void* out, int64_t q_start, int64_t Lq, int64_t Lk,
                 int Hq, int Hkv, int d, int64_t s, int64_t w, double yarn_scale, int dtype,
-                void* ws, const Layout& L, cudaStream_t st) {
+                void* ws, const Layout& L, cudaStream_t st, int reading = 0) {
   if (Lq == 0) return DCA_OK;
   uint8_t* base = static_cast<uint8_t*>(ws);
   dca::AttnArgs a;
@@ -118,6 +118,7 @@ int attend_impl(const void* q, const void* v, void* out, int64_t q_start, int64_
   a.tab_c1 = L.T - 1;
   a.Hq = Hq;
   a.Hkv = Hkv;
+  a.reading = reading;
   a.scale_log2 = logit_scale_log2(yarn_scale, d);
   a.status = reinterpret_cast<unsigned int*>(base);
   a.timeout_ns = static_cast<unsigned long long>(g_timeout_ns.load());
@@ -128,6 +129,17 @@ int attend_impl(const void* q, const void* v, void* out, int64_t q_start, int64_
 }
 
 bool ptrs_ok(const void* p) { return p != nullptr && aligned(p, 16); }
+
+// Window reading from the options (NULL = defaults); -1 when invalid.
+int reading_of(const dca_options* opts) {
+  if (opts == nullptr) return DCA_WINDOW_QUERY_OFFSET;
+  if (opts->window_reading != DCA_WINDOW_QUERY_OFFSET &&
+      opts->window_reading != DCA_WINDOW_TRUE_DISTANCE)
+    return -1;
+  for (int k = 0; k < 7; ++k)
+    if (opts->reserved[k] != 0) return -1;
+  return opts->window_reading;
+}
 
 }  // namespace
 
@@ -183,6 +195,17 @@ int dca_attend(const void* q_block, const void* v_cache, void* out_block, int64_
                int64_t Lq, int64_t Lk, int Hq, int Hkv, int d, int64_t chunk_size,
                int64_t local_window, int64_t pretrain_window, double yarn_scale, int dtype,
                void* workspace, size_t ws_bytes, void* cuda_stream) {
+  return dca_attend_ex(q_block, v_cache, out_block, q_start, Lq, Lk, Hq, Hkv, d, chunk_size,
+                       local_window, pretrain_window, yarn_scale, dtype, nullptr, workspace,
+                       ws_bytes, cuda_stream);
+}
+
+int dca_attend_ex(const void* q_block, const void* v_cache, void* out_block, int64_t q_start,
+                  int64_t Lq, int64_t Lk, int Hq, int Hkv, int d, int64_t chunk_size,
+                  int64_t local_window, int64_t pretrain_window, double yarn_scale, int dtype,
+                  const dca_options* opts, void* workspace, size_t ws_bytes, void* cuda_stream) {
+  const int reading = reading_of(opts);
+  if (reading < 0) return DCA_ERR_ARG;
   Layout L;
   int rc = check_common(q_start, Lq, Lk, Hq, Hkv, d, chunk_size, local_window, pretrain_window,
                         yarn_scale, dtype, workspace, ws_bytes, &L);
@@ -191,7 +214,7 @@ int dca_attend(const void* q_block, const void* v_cache, void* out_block, int64_
     return DCA_ERR_ARG;
   return attend_impl(q_block, v_cache, out_block, q_start, Lq, Lk, Hq, Hkv, d, chunk_size,
                      local_window, yarn_scale, dtype, workspace, L,
-                     static_cast<cudaStream_t>(cuda_stream));
+                     static_cast<cudaStream_t>(cuda_stream), reading);
 }
 
 int dca_prefill_chunked(const void* q_block, const void* k_cache, const void* v_cache,
@@ -199,6 +222,19 @@ int dca_prefill_chunked(const void* q_block, const void* k_cache, const void* v_
                         int Hkv, int d, int64_t chunk_size, int64_t local_window,
                         int64_t pretrain_window, double rope_base, double yarn_scale,
                         int dtype, void* workspace, size_t ws_bytes, void* cuda_stream) {
+  return dca_prefill_chunked_ex(q_block, k_cache, v_cache, out_block, q_start, Lq, Lk, Hq, Hkv,
+                                d, chunk_size, local_window, pretrain_window, rope_base,
+                                yarn_scale, dtype, nullptr, workspace, ws_bytes, cuda_stream);
+}
+
+int dca_prefill_chunked_ex(const void* q_block, const void* k_cache, const void* v_cache,
+                           void* out_block, int64_t q_start, int64_t Lq, int64_t Lk, int Hq,
+                           int Hkv, int d, int64_t chunk_size, int64_t local_window,
+                           int64_t pretrain_window, double rope_base, double yarn_scale,
+                           int dtype, const dca_options* opts, void* workspace, size_t ws_bytes,
+                           void* cuda_stream) {
+  const int reading = reading_of(opts);
+  if (reading < 0) return DCA_ERR_ARG;
   Layout L;
   int rc = check_common(q_start, Lq, Lk, Hq, Hkv, d, chunk_size, local_window, pretrain_window,
                         yarn_scale, dtype, workspace, ws_bytes, &L);
@@ -212,7 +248,7 @@ int dca_prefill_chunked(const void* q_block, const void* k_cache, const void* v_
                     dtype, workspace, L, st);
   if (rc != DCA_OK) return rc;
   return attend_impl(q_block, v_cache, out_block, q_start, Lq, Lk, Hq, Hkv, d, chunk_size,
-                     local_window, yarn_scale, dtype, workspace, L, st);
+                     local_window, yarn_scale, dtype, workspace, L, st, reading);
 }
 
 int dca_prefill(const void* q, const void* k, const void* v, void* out, int64_t L, int Hq,
@@ -301,18 +337,24 @@ int dca_prefill_host(const void* q_h, const void* k_h, const void* v_h, void* ou
   return DCA_OK;
 }
 
-int dca_plan_items(int64_t i0, int64_t i_last, int64_t tile_rows, int64_t chunk_size, int bn,
-                   int32_t* items, int max_items) {
+int dca_plan_items(int64_t i0, int64_t i_last, int64_t tile_rows, int64_t chunk_size,
+                   int64_t local_window, int window_reading, int bn, int32_t* items,
+                   int max_items) {
   if (i0 < 0 || i_last < i0 || tile_rows < 1 || i_last >= i0 + tile_rows || chunk_size < 1 ||
-      bn < 1 || max_items < 0 || (max_items > 0 && items == nullptr))
+      local_window < 0 || local_window > chunk_size || bn < 1 || max_items < 0 ||
+      (max_items > 0 && items == nullptr) ||
+      (window_reading != DCA_WINDOW_QUERY_OFFSET && window_reading != DCA_WINDOW_TRUE_DISTANCE))
     return DCA_ERR_ARG;
-  const dca::TilePlan P = dca::make_plan(i0, i_last, chunk_size, bn);
-  const dca::FullRanges F = dca::make_full_ranges(i0, i0 + tile_rows - 1, chunk_size, bn);
+  const int64_t w = local_window;
+  const int rd = window_reading;
+  const dca::TilePlan P = dca::make_plan(i0, i_last, chunk_size, w, bn, rd);
+  const dca::FullRanges F = dca::make_full_ranges(i0, i0 + tile_rows - 1, chunk_size, w, bn, rd);
   for (int n = 0; n < P.n_items && n < max_items; ++n) {
     int kt, cls;
     dca::plan_item(P, n, kt, cls);
     const int64_t j0 = static_cast<int64_t>(kt) * bn;
-    const bool full = dca::item_is_full(i0, i0 + tile_rows - 1, j0, j0 + bn - 1, chunk_size, cls);
+    const bool full =
+        dca::item_is_full(i0, i0 + tile_rows - 1, j0, j0 + bn - 1, chunk_size, w, cls, rd);
     // the kernels use the precomputed ranges; they must agree with the predicate
     if (full != dca::is_full(F, kt, cls)) return DCA_ERR_ARG - 100;
     items[3 * n + 0] = kt;

@@ -32,6 +32,7 @@ struct Params {
   const float2* tab;
   int64_t q_start, Lq, Lk, s, w, tab_c1;
   int Hq, Hkv, G, n_qtiles;
+  int reading;
   float scale_log2;
 };
 
@@ -49,7 +50,7 @@ __global__ void __launch_bounds__(THREADS) dca_fwd_f32_kernel(const Params p) {
   const int64_t q_end = p.q_start + p.Lq;
   const int64_t i_last = (i0 + BM - 1 < q_end - 1) ? i0 + BM - 1 : q_end - 1;
   const int64_t i_hi = i0 + BM - 1;
-  const TilePlan plan = make_plan(i0, i_last, p.s, BN);
+  const TilePlan plan = make_plan(i0, i_last, p.s, p.w, BN, p.reading);
 
   const int t = threadIdx.x;
   const int rg = t >> 4, cg = t & 15;
@@ -122,7 +123,7 @@ __global__ void __launch_bounds__(THREADS) dca_fwd_f32_kernel(const Params p) {
         for (int b = 0; b < 4; ++b) S[a][b] = fmaf(qa[a], kb[b], S[a][b]);
     }
 
-    const bool full = item_is_full(i0, i_hi, j0, j0 + BN - 1, p.s, cls);
+    const bool full = item_is_full(i0, i_hi, j0, j0 + BN - 1, p.s, p.w, cls, p.reading);
 #pragma unroll
     for (int a = 0; a < 4; ++a) {
       const int64_t i = i0 + 4 * rg + a;
@@ -131,7 +132,7 @@ __global__ void __launch_bounds__(THREADS) dca_fwd_f32_kernel(const Params p) {
 #pragma unroll
         for (int b = 0; b < 4; ++b) {
           const int64_t j = j0 + cg + 16 * b;
-          const bool valid = (j <= i) && (class_of_distance(ni - j / p.s) == cls);
+          const bool valid = (j <= i) && (pair_class(ni - j / p.s, i - j, p.w, p.reading) == cls);
           if (!valid) S[a][b] = -INFINITY;
         }
       }
@@ -202,6 +203,7 @@ cudaError_t launch_attention_f32(const AttnArgs& a, cudaStream_t st) {
   p.Hkv = a.Hkv;
   p.G = a.Hq / a.Hkv;
   p.n_qtiles = static_cast<int>((a.Lq + BM - 1) / BM);
+  p.reading = a.reading;
   p.scale_log2 = a.scale_log2;
   const int64_t blocks = static_cast<int64_t>(p.n_qtiles) * p.Hq;
   if (blocks > 0x7fffffffLL) return cudaErrorInvalidValue;

@@ -107,6 +107,7 @@ struct Params {
   int64_t q_start, Lq, Lk;
   int64_t s, w, tab_c1;
   int Hq, Hkv, G, n_pairs, n_qtiles;
+  int reading;  // READING_A or READING_B
   float scale_log2;
   unsigned int* status;
   unsigned long long timeout_ns;
@@ -187,9 +188,10 @@ __device__ __forceinline__ void write_q_row(uint8_t* qb, int r, const __nv_bfloa
 }
 
 // Mask NC consecutive scores of row i (keys j0 .. j0+NC-1) to the pairs that
-// are causal and belong to class `cls`.
+// are causal and belong to work-list class `cls` under window reading `reading`.
 template <int NC>
-__device__ __forceinline__ void mask_cols(uint32_t* sv, int64_t i, int64_t j0, int cls, int64_t s) {
+__device__ __forceinline__ void mask_cols(uint32_t* sv, int64_t i, int64_t j0, int cls, int64_t s,
+                                          int64_t w, int reading) {
   const int64_t ni = i / s;
   const int64_t nj0 = j0 / s;
   const int64_t dn64 = ni - nj0;
@@ -197,8 +199,11 @@ __device__ __forceinline__ void mask_cols(uint32_t* sv, int64_t i, int64_t j0, i
   const int64_t b64 = (nj0 + 1) * s - j0;  // first column of the next chunk
   int bnd = static_cast<int>(b64 > (1 << 30) ? (1 << 30) : b64);
   const int s32 = static_cast<int>(s > (1 << 30) ? (1 << 30) : s);
-  const int64_t lim64 = i - j0;  // last causal column
+  const int64_t lim64 = i - j0;  // last causal column; also i - j of column 0
   const int lim = static_cast<int>(lim64 > 1024 ? 1024 : (lim64 < -1 ? -1 : lim64));
+  // i - j = (i - j0) - e, compared with w only under reading B
+  const int64_t far64 = lim64 - w;  // columns e <= far64 have i - j >= w
+  const int far = static_cast<int>(far64 > 1024 ? 1024 : (far64 < -1 ? -1 : far64));
   const uint32_t NEG_INF = 0xff800000u;
 #pragma unroll
   for (int e = 0; e < NC; ++e) {
@@ -206,7 +211,9 @@ __device__ __forceinline__ void mask_cols(uint32_t* sv, int64_t i, int64_t j0, i
       dn -= 1;
       bnd += s32;
     }
-    const int ce = dn <= 0 ? CLS_INTRA : (dn == 1 ? CLS_SUCC : CLS_INTER);
+    const int ce = dn <= 0 ? CLS_INTRA
+                           : ((dn == 1 && (reading == READING_A || e > far)) ? CLS_SUCC
+                                                                              : CLS_INTER);
     if (e > lim || ce != cls) sv[e] = NEG_INF;
   }
 }
@@ -287,14 +294,15 @@ __device__ __forceinline__ float exp_pack64(const uint32_t* sv, float sc, float 
 // range; the final O / l uses the same reference).  O holds items < n: their
 // MMAs completed before S(n) did (one commit tracks all earlier MMAs).
 __device__ __forceinline__ bool softmax_half_step(uint32_t tS, uint32_t tO, int n, bool full,
-                                                  int64_t i, int kt, int cls, int64_t s, float sc,
+                                                  int64_t i, int kt, int cls, int64_t s, int64_t w,
+                                                  int reading, float sc,
                                                   float& m_ref, float& l_sum, PairCtx& pc,
                                                   volatile int* abort, unsigned int* status,
                                                   uint64_t timeout_ns, unsigned int code) {
   const int half = pc.half;
   uint32_t sv[64];
   tmem_ld64(tS + 64u * half, sv);
-  if (!full) mask_cols<64>(sv, i, static_cast<int64_t>(kt) * BN + 64 * half, cls, s);
+  if (!full) mask_cols<64>(sv, i, static_cast<int64_t>(kt) * BN + 64 * half, cls, s, w, reading);
   float mx = max64(sv);
   float mx_other = -INFINITY;
   if (!pair_exchange(pc, mx, mx_other, abort, status, timeout_ns, code)) return false;
@@ -357,8 +365,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const int64_t q_end = p.q_start + p.Lq;
   const int64_t i_last = (i0 + BM - 1 < q_end - 1) ? i0 + BM - 1 : q_end - 1;
   const int64_t i_hi = i0 + BM - 1;
-  const TilePlan plan = make_plan(i0, i_last, p.s, BN);
-  const FullRanges fullr = make_full_ranges(i0, i_hi, p.s, BN);
+  const TilePlan plan = make_plan(i0, i_last, p.s, p.w, BN, p.reading);
+  const FullRanges fullr = make_full_ranges(i0, i_hi, p.s, p.w, BN, p.reading);
   const int N = plan.n_items;
 
   if (threadIdx.x == 0) {
@@ -452,7 +460,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         tc_fence_after();
         const uint32_t tS = tbase + lane_off + static_cast<uint32_t>(st * 128);
         const uint32_t tO = tbase + lane_off + 256u + static_cast<uint32_t>(st * 128);
-        ok = softmax_half_step(tS, tO, n, full, i, kt, cls, p.s, sc, m_ref[st], l_sum[st], pc,
+        ok = softmax_half_step(tS, tO, n, full, i, kt, cls, p.s, p.w, p.reading, sc, m_ref[st],
+                               l_sum[st], pc,
                                abort_flag, p.status, p.timeout_ns, ST_SOFTMAX << st);
         if (!ok) break;
         if (cls_next != cls) {  // phase switch: the next items need another query rotation
@@ -698,6 +707,7 @@ cudaError_t launch_attention_sm100(const AttnArgs& a, cudaStream_t st) {
   p.G = a.Hq / a.Hkv;
   p.n_pairs = (p.G + 1) / 2;
   p.n_qtiles = static_cast<int>((a.Lq + BM - 1) / BM);
+  p.reading = a.reading;
   p.scale_log2 = a.scale_log2;
   p.status = a.status;
   p.timeout_ns = a.timeout_ns;

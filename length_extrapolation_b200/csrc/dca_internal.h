@@ -16,6 +16,7 @@ struct AttnArgs {
   int64_t q_start, Lq, Lk;
   int64_t s, w, tab_c1; // chunk size, local window, table row of position c-1
   int Hq, Hkv;
+  int reading;          // window reading: 0 (r_i < w) or 1 (i - j < w)
   float scale_log2;     // m^2 / sqrt(d) * log2(e)
   unsigned int* status; // device status word (workspace header)
   unsigned long long timeout_ns;

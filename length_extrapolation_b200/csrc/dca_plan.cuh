@@ -12,8 +12,8 @@
 // share one class is one plain MMA with that class's rotated Q.
 //
 // For a q-tile with rows [i0, i_last] the keys of each class form one
-// contiguous range, so the k-tiles carrying a class are one contiguous range
-// too.  A q-tile's work list is: INTER k-tiles, then SUCC k-tiles, then INTRA
+// contiguous range (a superset under reading B's diagonal window), so the
+// k-tiles carrying a class are one contiguous range too.  A q-tile's work list is: INTER k-tiles, then SUCC k-tiles, then INTRA
 // k-tiles (one Q rotation per phase).  A k-tile that holds keys of several
 // classes appears once per class and is masked per element to that class;
 // tiles crossing the causal diagonal are masked to j <= i.
@@ -42,19 +42,45 @@ DCA_HD int class_of_distance(int64_t chunk_dist) {
   return chunk_dist <= 0 ? CLS_INTRA : (chunk_dist == 1 ? CLS_SUCC : CLS_INTER);
 }
 
+// Window readings of section "Successive-Chunk Attention":
+//   READING_A: an adjacent-chunk pair keeps its true distance when the query's
+//              offset in its chunk r_i < w (the query rotation depends on the
+//              row only: s + r_i, or c - 1 when r_i >= w);
+//   READING_B: an adjacent-chunk pair keeps its true distance when i - j < w;
+//              the other adjacent-chunk pairs take the inter-chunk rule and are
+//              processed with the INTER rotation (c - 1).
+enum : int { READING_A = 0, READING_B = 1 };
+
+// Work-list class of pair (i, j), j <= i, with chunk distance dn.
+DCA_HD int pair_class(int64_t dn, int64_t i_minus_j, int64_t w, int reading) {
+  if (dn <= 0) return CLS_INTRA;
+  if (dn == 1 && (reading == READING_A || i_minus_j < w)) return CLS_SUCC;
+  return CLS_INTER;
+}
+
 // Work list of the q-tile whose real rows are [i0, i_last] (absolute indices),
 // for key tiles of `bn` keys.
-DCA_HD TilePlan make_plan(int64_t i0, int64_t i_last, int64_t s, int bn) {
+DCA_HD TilePlan make_plan(int64_t i0, int64_t i_last, int64_t s, int64_t w, int bn,
+                          int reading) {
   TilePlan P;
   const int64_t n0 = i0 / s, n1 = i_last / s;
-  // INTER: keys with n_j <= n1 - 2, i.e. j < s*(n1-1)
+  // INTER: keys with n_j <= n1 - 2, i.e. j < s*(n1-1); under reading B also the
+  // adjacent-chunk keys j <= i - w of some row (j < min(s*n1, i_last - w + 1))
+  int64_t inter_end = (n1 >= 2) ? s * (n1 - 1) : 0;
+  if (reading == READING_B && n1 >= 1) {
+    const int64_t far_end = (s * n1 < i_last - w + 1) ? s * n1 : i_last - w + 1;
+    if (far_end > inter_end) inter_end = far_end;
+  }
   P.lo[CLS_INTER] = 0;
-  P.hi[CLS_INTER] = (n1 >= 2) ? static_cast<int>(cdiv64(s * (n1 - 1), bn)) : 0;
-  // SUCC: keys with n_j in [n0-1, n1-1]
-  if (n1 >= 1) {
-    const int64_t a = s * (n0 >= 1 ? n0 - 1 : 0), b = s * n1;
+  P.hi[CLS_INTER] = static_cast<int>(cdiv64(inter_end, bn));
+  // SUCC: keys with n_j in [n0-1, n1-1]; under reading B only those with
+  // i - j < w for some row (j > i0 - w)
+  if (n1 >= 1 && (reading == READING_A || w > 0)) {
+    int64_t a = s * (n0 >= 1 ? n0 - 1 : 0);
+    const int64_t b = s * n1;
+    if (reading == READING_B && i0 - w + 1 > a) a = i0 - w + 1;
     P.lo[CLS_SUCC] = static_cast<int>(a / bn);
-    P.hi[CLS_SUCC] = static_cast<int>(cdiv64(b, bn));
+    P.hi[CLS_SUCC] = a < b ? static_cast<int>(cdiv64(b, bn)) : P.lo[CLS_SUCC];
   } else {
     P.lo[CLS_SUCC] = P.hi[CLS_SUCC] = 0;
   }
@@ -85,10 +111,12 @@ DCA_HD void plan_item(const TilePlan& P, int n, int& kt, int& cls) {
 // True when every (i, j) with i in [i0, i_hi], j in [j0, j_hi] is causal
 // (j <= i) and of class `cls`: the tile needs no per-element mask.
 DCA_HD bool item_is_full(int64_t i0, int64_t i_hi, int64_t j0, int64_t j_hi, int64_t s,
-                         int cls) {
+                         int64_t w, int cls, int reading) {
   const int64_t ni0 = i0 / s, ni1 = i_hi / s, nj0 = j0 / s, nj1 = j_hi / s;
-  if (cls == CLS_INTER) return ni0 - nj1 >= 2;
-  if (cls == CLS_SUCC) return (ni0 - nj1 >= 1) && (ni1 - nj0 <= 1);
+  if (cls == CLS_INTER)
+    return ni0 - nj1 >= 2 || (reading == READING_B && ni0 - nj1 >= 1 && i0 - j_hi >= w);
+  if (cls == CLS_SUCC)
+    return (ni0 - nj1 >= 1) && (ni1 - nj0 <= 1) && (reading == READING_A || i_hi - j0 < w);
   return ni0 == ni1 && nj0 == nj1 && ni0 == nj0 && j_hi <= i0;
 }
 
@@ -102,15 +130,29 @@ struct FullRanges {
 
 DCA_HD int64_t floor_div64(int64_t a, int64_t b) { return a >= 0 ? a / b : -((-a + b - 1) / b); }
 
-DCA_HD FullRanges make_full_ranges(int64_t i0, int64_t i_hi, int64_t s, int bn) {
+DCA_HD FullRanges make_full_ranges(int64_t i0, int64_t i_hi, int64_t s, int64_t w, int bn,
+                                   int reading) {
   FullRanges F;
   const int64_t ni0 = i0 / s, ni1 = i_hi / s;
-  // INTER: j_hi < s*(ni0-1)  <=>  (kt+1)*bn <= s*(ni0-1)
+  // INTER: j_hi < s*(ni0-1)  <=>  (kt+1)*bn <= s*(ni0-1); under reading B also
+  // j_hi < s*ni0 with j_hi <= i0 - w
   F.lo[CLS_INTER] = 0;
-  F.hi[CLS_INTER] = ni0 >= 1 ? static_cast<int>(floor_div64(s * (ni0 - 1), bn)) : 0;
-  // SUCC: j_hi < s*ni0 and j0 >= s*(ni1-1)
   {
-    const int64_t lo = ni1 >= 1 ? cdiv64(s * (ni1 - 1), bn) : 0;
+    int64_t hi = ni0 >= 1 ? floor_div64(s * (ni0 - 1), bn) : 0;
+    if (reading == READING_B && ni0 >= 1) {
+      const int64_t end = (s * ni0 < i0 - w + 1) ? s * ni0 : i0 - w + 1;
+      const int64_t hb = floor_div64(end, bn);
+      if (hb > hi) hi = hb;
+    }
+    F.hi[CLS_INTER] = static_cast<int>(hi > 0 ? hi : 0);
+  }
+  // SUCC: j_hi < s*ni0 and j0 >= s*(ni1-1); under reading B also j0 > i_hi - w
+  {
+    int64_t lo = ni1 >= 1 ? cdiv64(s * (ni1 - 1), bn) : 0;
+    if (reading == READING_B) {
+      const int64_t lb = (i_hi - w + 1) > 0 ? cdiv64(i_hi - w + 1, bn) : 0;
+      if (lb > lo) lo = lb;
+    }
     const int64_t hi = floor_div64(s * ni0, bn);
     F.lo[CLS_SUCC] = static_cast<int>(lo);
     F.hi[CLS_SUCC] = static_cast<int>(hi > lo ? hi : lo);

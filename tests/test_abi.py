@@ -120,6 +120,43 @@ def test_prepare_attend_reject(lib):
     assert lib.dca_attend(p, p, p, 0, 0, 5, 4, 2, 128, 64, 16, 128, 1.0, 0, p, ws, None) == N.DCA_OK
 
 
+def test_window_reading_options(lib):
+    """dca_options: an unknown reading or a non-zero reserved field is an
+    argument error, found before any launch; NULL selects the default."""
+    import ctypes
+    p = 1 << 20
+    ws = lib.dca_workspace_size(512, 4, 2, 128, 64, 16, 128, 0)
+
+    def chunked(opts, lq=10):
+        return lib.dca_prefill_chunked_ex(p, p, p, p, 0, lq, 100, 4, 2, 128, 64, 16, 128, 1e7,
+                                          1.0, 0, opts, p, ws, None)
+
+    def attend(opts, lq=10):
+        return lib.dca_attend_ex(p, p, p, 0, lq, 100, 4, 2, 128, 64, 16, 128, 1.0, 0, opts, p,
+                                 ws, None)
+
+    for bad_reading, bad_reserved in [(2, 0), (-1, 0), (0, 1), (1, 7)]:
+        o = N.DCAOptions()
+        o.window_reading = bad_reading
+        o.reserved[3] = bad_reserved
+        assert chunked(ctypes.byref(o)) == N.DCA_ERR_ARG
+        assert attend(ctypes.byref(o)) == N.DCA_ERR_ARG
+    for reading in (N.DCA_WINDOW_QUERY_OFFSET, N.DCA_WINDOW_TRUE_DISTANCE):
+        o = N.DCAOptions()
+        o.window_reading = reading
+        assert chunked(ctypes.byref(o), lq=0) == N.DCA_OK   # empty block: valid, no launch
+        assert attend(ctypes.byref(o), lq=0) == N.DCA_OK
+    assert chunked(None, lq=0) == N.DCA_OK
+    assert ctypes.sizeof(N.DCAOptions) == 32
+
+
+def test_python_api_rejects_unknown_window_reading():
+    from length_extrapolation_b200 import api
+    with pytest.raises(ValueError):
+        api._options("window")
+    assert api._options("true_distance").window_reading == N.DCA_WINDOW_TRUE_DISTANCE
+
+
 def test_host_entry_rejects(lib):
     need = lib.dca_host_arena_size(1000, 256, 4, 2, 128, 64, 16, 128, 0)
     assert need > lib.dca_workspace_size(1000, 4, 2, 128, 64, 16, 128, 0)

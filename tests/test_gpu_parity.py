@@ -97,6 +97,63 @@ def test_negative_controls_see_the_mapping():
     assert errors(got, bad)[1] > 2 * TOL[torch.bfloat16]["rel_l2"]
 
 
+# Window reading B (true distance kept iff i - j < w): the same small shapes,
+# plus the reading's own degenerate cases.  Reading B differs from reading A
+# only in which successive-chunk pairs keep the true distance.
+READING_B = [
+    small("B_ragged_mixed", 1000, 4, 1, 300, 50, 400),
+    small("B_g7_yarn2", 777, 7, 1, 256, 128, 512, yarn=2.0),
+    small("B_w_eq_s", 900, 2, 1, 200, 200, 400),
+    small("B_w0", 400, 2, 2, 64, 0, 64),          # no pair keeps its true distance across chunks
+    small("B_w1", 520, 2, 1, 128, 1, 160),        # only j = i - 1 at a chunk start
+    small("B_odd_window", 1100, 4, 2, 256, 77, 400, sqrt_d=False),
+    small("B_tiny_chunks", 300, 2, 1, 3, 2, 5),
+    small("B_single_chunk", 384, 4, 2, 384, 16, 512),
+    small("B_f32", 700, 3, 1, 200, 40, 300, dtype="f32", sqrt_d=False),
+]
+
+
+@pytest.mark.parametrize("w", READING_B, ids=lambda w: w.name)
+def test_reading_b_all_rows(w):
+    q, k, v = generate(w, device=DEV, seed=3)
+    out = dca.prefill(q, k, v, window_reading="true_distance", **w.params())
+    torch.cuda.synchronize()
+    want = oracle.attention(q.cpu(), k.cpu(), v.cpu(), reading=1, **w.params())
+    assert_close(out.double().cpu().numpy(), want, w.torch_dtype, w.name)
+
+
+def test_reading_b_differs_from_a():
+    """The two readings give measurably different outputs on O(1) logits, and
+    each kernel option matches its own oracle reading, not the other."""
+    w = small("AB", 1024, 2, 1, 256, 64, 384, sqrt_d=False)
+    q, k, v = generate(w, device=DEV, seed=5)
+    outs = {r: dca.prefill(q, k, v, window_reading=r, **w.params()).double().cpu().numpy()
+            for r in ("query_offset", "true_distance")}
+    qc, kc, vc = q.cpu(), k.cpu(), v.cpu()
+    want = {r: oracle.attention(qc, kc, vc, reading=i, **w.params())
+            for i, r in enumerate(("query_offset", "true_distance"))}
+    tol = TOL[torch.bfloat16]["rel_l2"]
+    for r in outs:
+        assert errors(outs[r], want[r])[1] <= tol
+        other = "true_distance" if r == "query_offset" else "query_offset"
+        assert errors(outs[r], want[other])[1] > 2 * tol
+
+
+def test_reading_b_chunked_blocks_equal_oneshot():
+    w = small("B_chunked", 1300, 4, 2, 256, 100, 512)
+    q, k, v = generate(w, device=DEV, seed=7)
+    one = dca.prefill(q, k, v, window_reading="true_distance", **w.params())
+    ws = dca.Workspace(w.L, w.Hq, w.Hkv, 128, w.chunk_size, w.local_window, w.pretrain_window,
+                       q.dtype, DEV)
+    blk = torch.empty_like(q)
+    for q0 in range(0, w.L, 256):       # tile-aligned blocks: the same tiles as one-shot
+        lq = min(256, w.L - q0)
+        dca.prefill_chunked(q[q0:q0 + lq], k, v, q_start=q0, kv_len=q0 + lq, workspace=ws,
+                            out=blk[q0:q0 + lq], window_reading="true_distance", **w.params())
+    torch.cuda.synchronize()
+    assert torch.equal(one, blk)
+
+
 @pytest.mark.parametrize("aligned", [True, False])
 def test_chunked_blocks_equal_oneshot(aligned):
     w = small("chunk", 1280, 4, 2, 320, 64, 512, yarn=2.0)

@@ -25,17 +25,23 @@ def lib():
     return N.lib()
 
 
-def plan(lib, i0, i_last, rows, s, bn):
+def plan(lib, i0, i_last, rows, s, bn, w=0, reading=0):
     buf = (ctypes.c_int32 * (3 * 16384))()
-    n = lib.dca_plan_items(i0, i_last, rows, s, bn, buf, 16384)
+    n = lib.dca_plan_items(i0, i_last, rows, s, w, reading, bn, buf, 16384)
     assert 0 <= n <= 16384
     a = np.frombuffer(buf, dtype=np.int32)[: 3 * n].reshape(n, 3)
     return a
 
 
-def chunk_class(i, j, s):
+def chunk_class(i, j, s, w=0, reading=0):
+    """Work-list class of a pair: 0 intra, 1 successive with its true distance
+    kept (reading A: every adjacent-chunk pair), 2 inter-chunk rule."""
     dn = i // s - j // s
-    return 0 if dn == 0 else (1 if dn == 1 else 2)
+    if dn == 0:
+        return 0
+    if dn == 1 and (reading == 0 or i - j < w):
+        return 1
+    return 2
 
 
 def query_position(i, cls, s, w, c):
@@ -61,13 +67,14 @@ CASES = [  # (L, s, w, c, bm, bn)
 ]
 
 
+@pytest.mark.parametrize("reading", [0, 1], ids=["query_offset", "true_distance"])
 @pytest.mark.parametrize("L,s,w,c,bm,bn", CASES)
-def test_plan_matches_oracle_positions(lib, L, s, w, c, bm, bn):
+def test_plan_matches_oracle_positions(lib, L, s, w, c, bm, bn, reading):
     for q_start, Lq in [(0, L), (L // 3, L - L // 3)]:
         for t0 in range(0, Lq, bm):
             i0 = q_start + t0
             i_last = min(i0 + bm - 1, q_start + Lq - 1)
-            items = plan(lib, i0, i_last, bm, s, bn)
+            items = plan(lib, i0, i_last, bm, s, bn, w, reading)
             # phases in order INTER, SUCC, INTRA
             assert list(items[:, 1]) == sorted(items[:, 1], reverse=True)
             seen = {}
@@ -77,21 +84,23 @@ def test_plan_matches_oracle_positions(lib, L, s, w, c, bm, bn):
                 if full:
                     for i in range(i0, i0 + bm):
                         for j in range(kt * bn, kt * bn + bn):
-                            assert j <= i and chunk_class(i, j, s) == cls
+                            assert j <= i and chunk_class(i, j, s, w, reading) == cls
             for i in range(i0, i_last + 1):
                 for j in range(0, i + 1):
-                    cls = chunk_class(i, j, s)
+                    cls = chunk_class(i, j, s, w, reading)
                     assert (j // bn, cls) in seen, (i, j)
-                    _, pq, pk = oracle.position(i, j, s, w, c)
+                    _, pq, pk = oracle.position(i, j, s, w, c, reading=reading)
                     assert pk == j % s
                     assert query_position(i, cls, s, w, c) == pq, (i, j, cls)
 
 
 def test_plan_rejects_bad_args(lib):
     buf = (ctypes.c_int32 * 3)()
-    assert lib.dca_plan_items(10, 5, 128, 64, 128, buf, 1) == N.DCA_ERR_ARG
-    assert lib.dca_plan_items(0, 200, 128, 64, 128, buf, 1) == N.DCA_ERR_ARG
-    assert lib.dca_plan_items(0, 5, 128, 0, 128, buf, 1) == N.DCA_ERR_ARG
+    assert lib.dca_plan_items(10, 5, 128, 64, 8, 0, 128, buf, 1) == N.DCA_ERR_ARG
+    assert lib.dca_plan_items(0, 200, 128, 64, 8, 0, 128, buf, 1) == N.DCA_ERR_ARG
+    assert lib.dca_plan_items(0, 5, 128, 0, 0, 0, 128, buf, 1) == N.DCA_ERR_ARG
+    assert lib.dca_plan_items(0, 5, 128, 64, 65, 0, 128, buf, 1) == N.DCA_ERR_ARG
+    assert lib.dca_plan_items(0, 5, 128, 64, 8, 2, 128, buf, 1) == N.DCA_ERR_ARG
 
 
 def test_big_config_phase_counts(lib):
