@@ -38,9 +38,11 @@ if ROOT not in sys.path:
 
 import torch  # noqa: E402
 
-from length_extrapolation_b200.workloads import WORKLOADS, generate, sample_heads  # noqa: E402
+from length_extrapolation_b200.workloads import (DECODE_WORKLOADS, WORKLOADS,  # noqa: E402
+                                                 generate, generate_decode, sample_heads)
 
 METRIC = "DCA prefill tokens/s and attention TFLOP/s (fraction of B200 bf16 peak)"
+DECODE_METRIC = "DCA decode tokens/s (KV-cache stream, fraction of B200 HBM bandwidth)"
 UNIT = "tokens/s"
 
 
@@ -50,7 +52,10 @@ def parse_args(argv=None):
     ap.add_argument("--steps", type=int, default=3)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", default="qwen7b_1m_chunked", choices=sorted(WORKLOADS))
+    ap.add_argument("--workload", default="qwen7b_1m_chunked",
+                    choices=sorted(WORKLOADS) + sorted(DECODE_WORKLOADS),
+                    help="a prefill workload, or a decode step (*_decode*: the new tokens "
+                         "against a full cache)")
     ap.add_argument("--e2e-steps", type=int, default=2)
     ap.add_argument("--cpu-seconds", type=float, default=20.0,
                     help="approximate CPU seconds for the oracle baseline sample")
@@ -312,9 +317,203 @@ def workload_config(w):
             "l2": "inputs larger than L2 (no flush)"}
 
 
+# ----------------------------------------------------------------------------- decode
+def decode_config(dw):
+    w = dw.base
+    return {"workload": dw.name, "kv_len": dw.Lk, "new_tokens": dw.Lq, "Hq": w.Hq,
+            "Hkv": w.Hkv, "d": w.d, "chunk_size": w.chunk_size, "local_window": w.local_window,
+            "pretrain_window": w.pretrain_window, "rope_base": w.rope_base,
+            "yarn_scale": w.yarn_scale, "global_batch": 1, "seq_len": dw.Lk,
+            "l2": "L2 flushed between steps (256 MiB write, untimed)"}
+
+
+def oracle_decode_rate(dw, q, k, v, budget_s):
+    """Time the fp64 oracle on the decode rows for a subset of heads; returns
+    (seconds per whole step extrapolated to all heads, description, threads)."""
+    import oracle
+    w = dw.base
+    threads = os.cpu_count() or 1
+    heads = sample_heads(w).numpy()
+    qc, kc, vc = q.cpu(), k.cpu(), v.cpu()
+    t0 = time.perf_counter()
+    n = 0
+    while True:
+        oracle.attention(qc, kc, vc, q_start=dw.Lk - dw.Lq, heads=heads, n_threads=threads,
+                         **w.params())
+        n += 1
+        if time.perf_counter() - t0 > budget_s or n >= 50:
+            break
+    dt = (time.perf_counter() - t0) / n
+    t_step = dt * w.Hq / len(heads)
+    desc = (f"{dw.Lq} rows x {len(heads)} of {w.Hq} heads against {dw.Lk} keys, "
+            f"{n} repetitions of {dt:.2f} s; extrapolated to all heads")
+    return t_step, desc, threads
+
+
+def run_decode_bench(args, dw, world, rank, local, dist):
+    """One step = one generation step of the library: rotate the Lq new keys
+    into the rotated-key cache (whose earlier rows are already there), then
+    the split-KV decode kernel and its merge, inputs resident in HBM."""
+    w = dw.base
+    if args.impl == "reference":
+        if rank != 0:
+            return 0
+        q, k, v = generate_decode(dw, device="cpu")
+        budget = min(args.cpu_seconds, max(2.0, 120.0 / max(1, args.steps + args.warmup)))
+        times, desc, threads = [], None, None
+        for it in range(min(args.warmup, 1) + min(args.steps, 3)):
+            t_step, desc, threads = oracle_decode_rate(dw, q, k, v, budget / 4)
+            if it >= min(args.warmup, 1):
+                times.append(t_step)
+        t_step = statistics.median(times)
+        value = dw.Lq / t_step
+        print(json.dumps({
+            "impl": "reference", "metric": DECODE_METRIC, "value": value, "unit": UNIT,
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": t_step * 1e3, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic", "config": decode_config(dw),
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
+                             "sample": desc},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}), flush=True)
+        return 0
+
+    import length_extrapolation_b200 as dca
+    from length_extrapolation_b200 import _native as N
+
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    peaks = load_peaks()
+    q, k, v = generate_decode(dw, device=dev, seed=0)
+    kw = dict(chunk_size=w.chunk_size, local_window=w.local_window,
+              pretrain_window=w.pretrain_window)
+    ws = dca.Workspace(dw.Lk, w.Hq, w.Hkv, w.d, w.chunk_size, w.local_window, w.pretrain_window,
+                       q.dtype, dev)
+    scratch = torch.empty(dca.decode_scratch_size(dw.Lq, w.Hq, w.Hkv), dtype=torch.uint8,
+                          device=dev)
+    out = torch.empty_like(q)
+    # the earlier keys are in the rotated-key cache (the prefill before this step)
+    dca.prepare(k, kv_len=dw.Lk - dw.Lq, k_rows_valid=0, rope_base=w.rope_base, workspace=ws,
+                **kw)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+
+    def step(evs=None):
+        if evs is not None:
+            evs[0].record()
+        dca.prepare(k, kv_len=dw.Lk, k_rows_valid=dw.Lk - dw.Lq, rope_base=w.rope_base,
+                    workspace=ws, **kw)
+        if evs is not None:
+            evs[1].record()
+        dca.decode(q, v, out, q_start=dw.Lk - dw.Lq, kv_len=dw.Lk, yarn_scale=w.yarn_scale,
+                   workspace=ws, scratch=scratch, **kw)
+        if evs is not None:
+            evs[2].record()
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    if ws.status() != N.DCA_OK:
+        raise RuntimeError("device status after warm-up")
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    clocks = ClockSampler(dev.index).start()
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    for e in evs:
+        flush.zero_()
+        step(e)
+    torch.cuda.synchronize()
+    if dist is not None:
+        dist.barrier()
+    clk = clocks.stop()
+    if ws.status() != N.DCA_OK:
+        raise RuntimeError("device status after timing")
+    ms = sum(e[0].elapsed_time(e[2]) for e in evs)
+    kern_ms = sum(e[1].elapsed_time(e[2]) for e in evs)
+    ms, kern_ms = max_over_ranks([ms, kern_ms], dist, dev)
+    ms_per_step = ms / args.steps
+    esz = q.element_size()
+    alg_bytes = dw.kv_bytes() + 2 * dw.Lq * w.Hq * w.d * esz   # K', V streamed once; q in, out
+    achieved = alg_bytes / (kern_ms / args.steps / 1e3) / 1e9
+    roofline = {"kernel": "dca_decode_kernel (split-KV, tcgen05) + merge",
+                "bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": achieved / peaks["hbm_gbs"],
+                "peak_kind": f"{peaks['source']} HBM copy bandwidth",
+                "traffic": None, "traffic_unit": "bytes per launch (dram read + write, ncu)",
+                "algorithmic_bytes_per_launch": alg_bytes,
+                "avg_launch_ms": kern_ms / args.steps}
+
+    e2e = None
+    if not args.no_e2e:
+        # host-side inputs of a step: the new tokens' q, k and v rows; result read back
+        qh = q.cpu().pin_memory()
+        knew = k[dw.Lk - dw.Lq:].cpu().pin_memory()
+        vnew = v[dw.Lk - dw.Lq:].cpu().pin_memory()
+        oh = torch.empty_like(qh).pin_memory()
+        qd = torch.empty_like(q)
+
+        def e2e_step():
+            qd.copy_(qh, non_blocking=True)
+            k[dw.Lk - dw.Lq:].copy_(knew, non_blocking=True)
+            v[dw.Lk - dw.Lq:].copy_(vnew, non_blocking=True)
+            dca.decode_step(qd, k, v, kv_len=dw.Lk, rope_base=w.rope_base,
+                            yarn_scale=w.yarn_scale, workspace=ws, scratch=scratch, out=out, **kw)
+            oh.copy_(out, non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize()
+        tot = 0.0
+        for _ in range(args.steps):
+            flush.zero_()
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record()
+            e2e_step()
+            e1.record()
+            torch.cuda.synchronize()
+            tot += e0.elapsed_time(e1)
+        ems = max_over_ranks([tot], dist, dev)[0] / args.steps
+        e2e = {"value": world * dw.Lq / (ems / 1e3), "unit": UNIT, "ms_per_step": ems,
+               "h2d_bytes_per_step": (qh.numel() + knew.numel() + vnew.numel()) * esz,
+               "d2h_bytes_per_step": oh.numel() * esz,
+               "path": "decode_step after pinned host->device copies of the new q/k/v rows; "
+                       "out copied back"}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        t_step, desc, threads = oracle_decode_rate(dw, q, k, v, args.cpu_seconds)
+        cpu = {"value": dw.Lq / t_step, "unit": UNIT, "cores": threads, "kind": "oracle",
+               "sample": desc}
+
+    line = {
+        "metric": DECODE_METRIC, "value": world * dw.Lq / (ms_per_step / 1e3), "unit": UNIT,
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": w.dtype,
+        "data": "synthetic",
+        "config": {**decode_config(dw),
+                   "parallelism": f"replicas x{world}" if world > 1 else "1 GPU"},
+        "roofline": roofline, "e2e": e2e, "cpu_baseline": cpu, "clocks": clk,
+        "gpu_launches": 3 * args.steps,   # key rotation, decode, merge
+        "peaks_source": peaks["source"],
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
 # ----------------------------------------------------------------------------- our arm
 def main(argv=None):
     args = parse_args(argv)
+    if args.workload in DECODE_WORKLOADS:
+        world = int(os.environ.get("WORLD_SIZE", "1"))
+        rank = int(os.environ.get("RANK", "0"))
+        local = int(os.environ.get("LOCAL_RANK", "0"))
+        dist = init_dist(world, local)
+        return run_decode_bench(args, DECODE_WORKLOADS[args.workload], world, rank, local, dist)
     w = WORKLOADS[args.workload]
     if args.record_traffic:
         write_traffic_record(w.name, args.record_traffic)

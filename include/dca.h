@@ -162,6 +162,34 @@ int dca_attend_ex(const void* q_block, const void* v_cache, void* out_block, int
                   const dca_options* opts, void* workspace, size_t ws_bytes, void* cuda_stream);
 
 /*
+ * Decode: a few new query tokens against the whole cache.  The "Chunked
+ * Prefill" section of "Qwen2.5-1M 不重训外推 1M" splits a long prompt into
+ * blocks so that generation (one new token per request per step) is not
+ * held up behind it; a decode step is the same attention with Lq tokens at
+ * the end of the cache.  Rows t of q_block have absolute positions
+ * q_start + t and attend cache rows j <= q_start + t, exactly as in
+ * dca_attend_ex, and the result equals those rows of the one-shot prefill.
+ * The rotated keys [0, Lk) must be in the workspace (dca_prepare; a decode
+ * step that appended Lq keys passes k_rows_valid = Lk - Lq).
+ *   q_block, out_block [Lq][Hq][d]; v_cache [Lk][Hkv][d];
+ *   lse: NULL or [Lq][Hq] fp32, receives ln sum_j exp(logit_ij) per row;
+ *   scratch: device memory of dca_decode_scratch_size(Lq, Hq, Hkv) bytes,
+ *   16-byte aligned, for the partial results of the split-KV kernel (bf16;
+ *   the fp32 path does not use it but the argument is checked the same way).
+ * 1 <= Lq <= DCA_DECODE_MAX_TOKENS (Lq = 0: nothing to do).  bf16 runs a
+ * split-KV tcgen05 kernel (the cache is cut into slices, one CTA per KV head,
+ * group of 16 (token, head) rows and slice) followed by a merge kernel; fp32
+ * runs the fp32 attention kernel.  Overlapping calls must not share scratch.
+ */
+#define DCA_DECODE_MAX_TOKENS 256
+size_t dca_decode_scratch_size(int64_t Lq, int Hq, int Hkv);
+int dca_decode(const void* q_block, const void* v_cache, void* out_block, float* lse,
+               int64_t q_start, int64_t Lq, int64_t Lk, int Hq, int Hkv, int d,
+               int64_t chunk_size, int64_t local_window, int64_t pretrain_window,
+               double yarn_scale, int dtype, const dca_options* opts, void* workspace,
+               size_t ws_bytes, void* scratch, size_t scratch_bytes, void* cuda_stream);
+
+/*
  * Device-side status: synchronises `cuda_stream`, reads and clears the status
  * word that kernels set when a bounded wait gave up.  Returns DCA_OK,
  * DCA_ERR_TIMEOUT or DCA_ERR_CUDA.
@@ -236,7 +264,8 @@ int dca_prefill_noalloc(const void* q, const void* k, const void* v, void* out, 
  * wait (default 10 s).  dca_set_debug_flags(1) makes the next attention launch
  * withhold its first key-tile load, so that its waits run out and the kernel
  * returns through the timeout path (status word set, DCA_ERR_TIMEOUT from
- * dca_device_status); flags reset to 0 after that launch.
+ * dca_device_status); flags reset to 0 after that launch.  The decode kernel
+ * honours the same flag.
  */
 void dca_set_wait_timeout_ns(int64_t ns);
 void dca_set_debug_flags(int flags);

@@ -8,6 +8,9 @@ built.
 from .api import (  # noqa: F401
     Workspace,
     attend,
+    decode,
+    decode_scratch_size,
+    decode_step,
     host_arena_size,
     prefill,
     prefill_chunked,
@@ -19,6 +22,6 @@ from .api import (  # noqa: F401
 )
 
 __all__ = [
-    "Workspace", "attend", "host_arena_size", "prefill", "prefill_chunked", "prefill_host",
+    "Workspace", "attend", "decode", "decode_scratch_size", "decode_step", "host_arena_size", "prefill", "prefill_chunked", "prefill_host",
     "prepare", "set_debug_flags", "set_wait_timeout_ns", "workspace_size",
 ]

@@ -44,12 +44,18 @@ SIGNATURES = {
                              _dbl, _i32, _vp, _vp, _sz, _vp]),
     "dca_prefill_noalloc": (_i32, [_vp, _vp, _vp, _vp, _i64, _i32, _i32, _i32, _i64, _i64, _i64,
                                    _dbl, _dbl, _i32, _vp]),
+    "dca_decode_scratch_size": (_sz, [_i64, _i32, _i32]),
+    "dca_decode": (_i32, [_vp, _vp, _vp, _vp, _i64, _i64, _i64, _i32, _i32, _i32, _i64, _i64,
+                          _i64, _dbl, _i32, _vp, _vp, _sz, _vp, _sz, _vp]),
     "dca_set_wait_timeout_ns": (None, [_i64]),
     "dca_set_debug_flags": (None, [_i32]),
 }
 
 _lock = threading.Lock()
 _lib = None
+
+
+DCA_DECODE_MAX_TOKENS = 256
 
 
 class DCAOptions(ctypes.Structure):

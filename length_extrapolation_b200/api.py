@@ -148,6 +148,59 @@ def attend(q_block, v_cache, out, *, q_start, kv_len, chunk_size, local_window, 
     N.check(rc, "dca_attend_ex")
 
 
+def decode_scratch_size(Lq, Hq, Hkv) -> int:
+    n = N.lib().dca_decode_scratch_size(int(Lq), int(Hq), int(Hkv))
+    if n == 0:
+        raise N.DCAError(N.DCA_ERR_ARG, "dca_decode_scratch_size")
+    return n
+
+
+def decode(q_block, v_cache, out=None, *, q_start, kv_len, chunk_size, local_window,
+           pretrain_window, yarn_scale=1.0, workspace: Workspace, scratch=None, lse=None,
+           window_reading="query_offset"):
+    """Decode-stage attention of a few query tokens (absolute rows q_start ..)
+    against the rotated keys [0, kv_len) in `workspace` and v_cache.  `lse`
+    (optional fp32 [Lq, Hq]) receives the natural-log LSE of each row."""
+    _check_cuda(q_block, v_cache)
+    Lq, Hq, d = q_block.shape
+    if out is None:
+        out = torch.empty_like(q_block)
+    _check_cuda(out)
+    if scratch is None:
+        scratch = torch.empty(decode_scratch_size(Lq, Hq, v_cache.shape[1]), dtype=torch.uint8,
+                              device=q_block.device)
+    if lse is not None:
+        _check_cuda(lse)
+        if lse.dtype != torch.float32 or tuple(lse.shape) != (Lq, Hq):
+            raise ValueError("lse must be fp32 [Lq, Hq]")
+    opts = _options(window_reading)
+    rc = N.lib().dca_decode(q_block.data_ptr(), v_cache.data_ptr(), out.data_ptr(),
+                            lse.data_ptr() if lse is not None else None, int(q_start), Lq,
+                            int(kv_len), Hq, v_cache.shape[1], d, int(chunk_size),
+                            int(local_window), int(pretrain_window), float(yarn_scale),
+                            _dtype_code(q_block), ctypes.byref(opts), workspace.ptr,
+                            workspace.nbytes, scratch.data_ptr(), scratch.numel(),
+                            _stream_ptr(q_block.device))
+    N.check(rc, "dca_decode")
+    return out
+
+
+def decode_step(q_new, k_cache, v_cache, *, kv_len, chunk_size, local_window, pretrain_window,
+                rope_base=1e7, yarn_scale=1.0, workspace: Workspace, scratch=None, out=None,
+                lse=None, window_reading="query_offset"):
+    """One generation step: the Lq new keys (cache rows [kv_len - Lq, kv_len))
+    are rotated into the workspace, whose rows [0, kv_len - Lq) already hold
+    the earlier keys, then the Lq new query tokens attend the whole cache."""
+    Lq = q_new.shape[0]
+    prepare(k_cache, kv_len=kv_len, k_rows_valid=kv_len - Lq, chunk_size=chunk_size,
+            local_window=local_window, pretrain_window=pretrain_window, rope_base=rope_base,
+            workspace=workspace)
+    return decode(q_new, v_cache, out, q_start=kv_len - Lq, kv_len=kv_len, chunk_size=chunk_size,
+                  local_window=local_window, pretrain_window=pretrain_window,
+                  yarn_scale=yarn_scale, workspace=workspace, scratch=scratch, lse=lse,
+                  window_reading=window_reading)
+
+
 def host_arena_size(L, block, Hq, Hkv, d, chunk_size, local_window, pretrain_window, dtype):
     code = _DTYPES[dtype] if isinstance(dtype, torch.dtype) else int(dtype)
     n = N.lib().dca_host_arena_size(int(L), int(block), int(Hq), int(Hkv), int(d),

@@ -130,6 +130,14 @@ int attend_impl(const void* q, const void* v, void* out, int64_t q_start, int64_
 
 bool ptrs_ok(const void* p) { return p != nullptr && aligned(p, 16); }
 
+// Scratch bytes of a decode call (0 for invalid sizes).
+size_t decode_scratch_bytes(int64_t Lq, int Hq, int Hkv) {
+  if (Lq < 1 || Lq > DCA_DECODE_MAX_TOKENS || Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0) return 0;
+  const int n_rg = dca::decode_row_groups(Lq, Hq / Hkv);
+  const int n_cta = Hkv * n_rg * dca::decode_max_splits(Hkv, n_rg);
+  return align_up(dca::decode_part_floats(n_cta) * sizeof(float), 256);
+}
+
 // Window reading from the options (NULL = defaults); -1 when invalid.
 int reading_of(const dca_options* opts) {
   if (opts == nullptr) return DCA_WINDOW_QUERY_OFFSET;
@@ -215,6 +223,53 @@ int dca_attend_ex(const void* q_block, const void* v_cache, void* out_block, int
   return attend_impl(q_block, v_cache, out_block, q_start, Lq, Lk, Hq, Hkv, d, chunk_size,
                      local_window, yarn_scale, dtype, workspace, L,
                      static_cast<cudaStream_t>(cuda_stream), reading);
+}
+
+size_t dca_decode_scratch_size(int64_t Lq, int Hq, int Hkv) {
+  return decode_scratch_bytes(Lq, Hq, Hkv);
+}
+
+int dca_decode(const void* q_block, const void* v_cache, void* out_block, float* lse,
+               int64_t q_start, int64_t Lq, int64_t Lk, int Hq, int Hkv, int d,
+               int64_t chunk_size, int64_t local_window, int64_t pretrain_window,
+               double yarn_scale, int dtype, const dca_options* opts, void* workspace,
+               size_t ws_bytes, void* scratch, size_t scratch_bytes, void* cuda_stream) {
+  const int reading = reading_of(opts);
+  if (reading < 0) return DCA_ERR_ARG;
+  Layout L;
+  int rc = check_common(q_start, Lq, Lk, Hq, Hkv, d, chunk_size, local_window, pretrain_window,
+                        yarn_scale, dtype, workspace, ws_bytes, &L);
+  if (rc != DCA_OK) return rc;
+  if (Lq == 0) return DCA_OK;
+  if (Lq > DCA_DECODE_MAX_TOKENS) return DCA_ERR_ARG;
+  if (!ptrs_ok(q_block) || !ptrs_ok(v_cache) || !ptrs_ok(out_block)) return DCA_ERR_ARG;
+  if (lse != nullptr && !aligned(lse, 4)) return DCA_ERR_ARG;
+  if (!ptrs_ok(scratch) || scratch_bytes < decode_scratch_bytes(Lq, Hq, Hkv)) return DCA_ERR_ARG;
+  uint8_t* base = static_cast<uint8_t*>(workspace);
+  dca::AttnArgs a;
+  a.q = q_block;
+  a.kr = base + L.kr_off;
+  a.v = v_cache;
+  a.out = out_block;
+  a.tab = reinterpret_cast<const float2*>(base + L.tab_off);
+  a.q_start = q_start;
+  a.Lq = Lq;
+  a.Lk = Lk;
+  a.s = chunk_size;
+  a.w = local_window;
+  a.tab_c1 = L.T - 1;
+  a.Hq = Hq;
+  a.Hkv = Hkv;
+  a.reading = reading;
+  a.scale_log2 = logit_scale_log2(yarn_scale, d);
+  a.status = reinterpret_cast<unsigned int*>(base);
+  a.timeout_ns = static_cast<unsigned long long>(g_timeout_ns.load());
+  a.debug = g_debug_flags.exchange(0);
+  a.lse = lse;
+  cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
+  cudaError_t e = dtype == DCA_BF16 ? dca::launch_decode_sm100(a, static_cast<float*>(scratch), st)
+                                    : dca::launch_attention_f32(a, st);
+  return e == cudaSuccess ? DCA_OK : DCA_ERR_CUDA;
 }
 
 int dca_prefill_chunked(const void* q_block, const void* k_cache, const void* v_cache,

@@ -1,0 +1,582 @@
+// dca_decode_sm100.cu -- Dual Chunk Attention for a few query rows against a
+// long KV cache (the decode step that follows a chunked prefill), sm_100a.
+//
+// Same position map as the prefill kernel ("Qwen2.5-1M 不重训外推 1M",
+// sections Intra / Successive / Inter-Chunk Attention): keys pre-rotated by
+// j mod s in the workspace, each query row rotated by r_i, s + r_i (or c - 1
+// outside the local window) or c - 1 according to the class of the key tile.
+// With one or a few query rows per KV head the work is a stream over the
+// whole cache (2 x 256 bytes per key and KV head) and HBM-bound, so the
+// kernel is split-KV: the work list of the query block (dca_plan.cuh) is cut
+// into contiguous slices, one CTA per (KV head, row group, slice), and a
+// combine kernel merges the slices' partial softmax states.
+//
+// One CTA (192 threads):
+//   warps 0-3  softmax: thread t owns key t of the current 128-key tile (TMEM
+//              lane t of S^T) and dim t of O^T
+//   warp 4     TMA producer: K'/V tiles (128 keys x 128 dims, bf16, 128-byte
+//              swizzle) into a ring of six 32 KiB slots (no multicast)
+//   warp 5     MMA issuer: S^T = K' Q_cls^T (M = 128 keys, N = 16 query rows)
+//              and O^T += V^T P^T (M = 128 dims, A = V tile read MN-major,
+//              B = P^T in shared memory), tcgen05.mma kind::f16, fp32 in TMEM
+// The G query heads of a KV head share its K'/V stream: up to 16 (token,
+// head) rows per row group; a row group is one MMA N.  Query rows are
+// rotated once per class at the start (three 4 KiB operand tiles).
+// Online softmax per row: the four softmax warps exchange their per-row tile
+// maxima through shared memory; the reference max moves (and O^T, l rescale)
+// only when it grows by more than 2^8, as in the prefill kernel.
+// Every wait is bounded (globaltimer); on timeout the CTA raises its abort
+// flag, ORs a code into the device status word, drains its copies and MMAs,
+// frees TMEM and exits.
+#include <cuda_bf16.h>
+#include <math.h>
+
+#include "dca_internal.h"
+#include "dca_plan.cuh"
+#include "sm100_ptx.cuh"
+
+namespace dca {
+namespace dec {
+
+constexpr int BN = 128;                  // keys per tile (MMA M of S^T)
+constexpr int NR = DECODE_ROWS;          // query rows per CTA (MMA N)
+constexpr int HD = 128;
+constexpr int NTILE = 6;                 // K'/V tile ring
+constexpr int TILE_BYTES = 32768;        // 128 x 128 bf16
+constexpr int HALF_BYTES = 16384;        // 128 rows x 64 bf16 (one swizzle column block)
+constexpr int OPB = NR * HD * 2;         // 4 KiB: a 16-row operand (Q variant or P^T)
+constexpr int OPB_HALF = NR * 128;       // 2 KiB: its 64-column block
+constexpr int NUM_THREADS = 192;
+constexpr int WARP_LOAD = 4;
+constexpr int WARP_MMA = 5;
+constexpr uint32_t TMEM_COLS = 64;       // S^T x2 (16 cols each), O^T (16 cols)
+constexpr uint32_t COL_O = 32;
+constexpr float RESCALE_LOG2 = 8.0f;
+
+constexpr unsigned ST_SOFTMAX = 0x10u, ST_LOAD = 0x100u, ST_MMA = 0x1000u, ST_DRAIN = 0x10000u;
+
+struct SmemCtl {
+  uint64_t tile_full[NTILE];
+  uint64_t tile_empty[NTILE];
+  uint64_t s_full[2];
+  uint64_t s_free[2];   // four softmax warps have read S^T
+  uint64_t p_full[2];   // four softmax warps have written P^T
+  uint64_t pv_done[2];  // O^T += V^T P^T of the item with this parity completed
+  uint64_t max_bar[2];  // four warps' row maxima are in wmax
+  uint64_t q_ready;
+  uint64_t o_final;
+  uint64_t epi_bar;
+  uint64_t drain;
+  uint32_t tmem_base;
+  int abort;
+  alignas(16) float wmax[2][4][NR];  // read as float4
+  float lsum[4][NR];
+};
+
+constexpr size_t SMEM_BYTES = 1024 + NTILE * TILE_BYTES + 3 * OPB + 2 * OPB + sizeof(SmemCtl);
+static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+
+struct Params {
+  const __nv_bfloat16* q;   // [Lq][Hq][128]
+  const float2* tab;
+  float* part;              // partial O [cta][NR][HD], m [cta][NR], l [cta][NR]
+  int64_t q_start, Lq, Lk, s, w, tab_c1;
+  int Hq, Hkv, G, n_rg, n_splits, n_cta;
+  int reading;
+  float scale_log2;
+  TilePlan plan;            // work list of the query block [q_start, q_start + Lq)
+  FullRanges fullr;         // its unmasked k-tiles per class
+  unsigned int* status;
+  unsigned long long timeout_ns;
+  int debug;
+};
+
+// float -> int with the same order (for the integer warp max reduction); an involution.
+__device__ __forceinline__ int ordered(int x) { return x >= 0 ? x : x ^ 0x7fffffff; }
+
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+
+// Absolute position of row rho of row group rg (padding rows repeat the last row).
+__device__ __forceinline__ int64_t row_pos(const Params& p, int rg, int rho) {
+  int64_t t = (static_cast<int64_t>(rg) * NR + rho) / p.G;
+  if (t > p.Lq - 1) t = p.Lq - 1;
+  return p.q_start + t;
+}
+
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+    dca_decode_kernel(const __grid_constant__ CUtensorMap tm_k,
+                      const __grid_constant__ CUtensorMap tm_v, const Params p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint8_t* tiles = smem;
+  uint8_t* qv = tiles + NTILE * TILE_BYTES;  // Q variants, indexed by class
+  uint8_t* pt = qv + 3 * OPB;                // P^T, two buffers
+  SmemCtl* ctl = reinterpret_cast<SmemCtl*>(pt + 2 * OPB);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  // ---- work unit: row group fastest (CTAs reading the same K'/V slice run
+  // together and share it in L2), then slice, then KV head
+  const int b = static_cast<int>(blockIdx.x);
+  const int rg = b % p.n_rg;
+  const int sp = (b / p.n_rg) % p.n_splits;
+  const int g = b / (p.n_rg * p.n_splits);
+  const int cta = (g * p.n_rg + rg) * p.n_splits + sp;
+  const int it0 = static_cast<int>(static_cast<int64_t>(p.plan.n_items) * sp / p.n_splits);
+  const int it1 = static_cast<int>(static_cast<int64_t>(p.plan.n_items) * (sp + 1) / p.n_splits);
+  const int N = it1 - it0;
+  const int64_t rows_total = p.Lq * p.G;
+  const int n_rows = static_cast<int>(
+      rows_total - static_cast<int64_t>(rg) * NR < NR ? rows_total - static_cast<int64_t>(rg) * NR
+                                                      : NR);
+
+  if (threadIdx.x == 0) {
+    for (int k = 0; k < NTILE; ++k) {
+      mbar_init(&ctl->tile_full[k], 1);
+      mbar_init(&ctl->tile_empty[k], 1);
+    }
+    for (int k = 0; k < 2; ++k) {
+      mbar_init(&ctl->s_full[k], 1);
+      mbar_init(&ctl->s_free[k], 4);
+      mbar_init(&ctl->p_full[k], 4);
+      mbar_init(&ctl->pv_done[k], 1);
+      mbar_init(&ctl->max_bar[k], 4);
+    }
+    mbar_init(&ctl->q_ready, 4);
+    mbar_init(&ctl->o_final, 1);
+    mbar_init(&ctl->epi_bar, 4);
+    mbar_init(&ctl->drain, 1);
+    ctl->abort = 0;
+    fence_barrier_init();
+  }
+  if (warp == WARP_MMA) {
+    tmem_alloc(&ctl->tmem_base, TMEM_COLS);
+    tmem_relinquish();
+  }
+  if (warp == WARP_LOAD && lane == 0) {
+    tma_prefetch_desc(&tm_k);
+    tma_prefetch_desc(&tm_v);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tbase = ctl->tmem_base;
+  volatile int* abort_flag = &ctl->abort;
+
+  if (warp < 4) {
+    // =========================================================== softmax
+    const int tau = warp * 32 + lane;
+    const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+    const float sc = p.scale_log2;
+
+    // The rotated query operands (16 rows x 128 dims, K-major, 128-byte
+    // swizzle) of the classes in the work list (the RoPE table holds the
+    // positions s + r only when the cache extends past the first chunk, which
+    // is when the list has successive-chunk items); task = (class, row,
+    // 8-dim chunk of each half).
+    for (int task = tau; task < 3 * NR * 8; task += 128) {
+      const int cls = task >> 7;
+      const int rho = (task >> 3) & (NR - 1);
+      const int c = task & 7;
+      uint4 oa = make_uint4(0, 0, 0, 0), ob = oa;
+      if (rho < n_rows && p.plan.hi[cls] > p.plan.lo[cls]) {
+        const int64_t rho_g = static_cast<int64_t>(rg) * NR + rho;
+        const int64_t t = rho_g / p.G;
+        const int h = g * p.G + static_cast<int>(rho_g % p.G);
+        const __nv_bfloat16* qrow = p.q + (t * p.Hq + h) * static_cast<int64_t>(HD);
+        const float2* trow =
+            p.tab + query_table_row(p.q_start + t, cls, p.s, p.w, p.tab_c1) * (HD / 2);
+        const uint4 xa = *reinterpret_cast<const uint4*>(qrow + 8 * c);
+        const uint4 xb = *reinterpret_cast<const uint4*>(qrow + 64 + 8 * c);
+        const float4* t4 = reinterpret_cast<const float4*>(trow + 8 * c);
+        const __nv_bfloat162* a2 = reinterpret_cast<const __nv_bfloat162*>(&xa);
+        const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&xb);
+        uint32_t* pa = reinterpret_cast<uint32_t*>(&oa);
+        uint32_t* pb = reinterpret_cast<uint32_t*>(&ob);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float4 cs = t4[e];
+          const float2 x = __bfloat1622float2(a2[e]);
+          const float2 y = __bfloat1622float2(b2[e]);
+          pa[e] = pack_bf16(x.x * cs.x - y.x * cs.y, x.y * cs.z - y.y * cs.w);
+          pb[e] = pack_bf16(x.x * cs.y + y.x * cs.x, x.y * cs.w + y.y * cs.z);
+        }
+      }
+      uint8_t* dst = qv + cls * OPB + rho * 128 + ((c ^ (rho & 7)) << 4);
+      *reinterpret_cast<uint4*>(dst) = oa;
+      *reinterpret_cast<uint4*>(dst + OPB_HALF) = ob;
+    }
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&ctl->q_ready);
+
+    // P^T store address of this thread's key for row 0 (rows add 128 bytes
+    // and change the swizzle phase)
+    const int kh = tau >> 6, kin = tau & 63;
+
+    float m_ref[NR], l_part[NR];
+#pragma unroll
+    for (int r = 0; r < NR; ++r) {
+      m_ref[r] = -INFINITY;
+      l_part[r] = 0.f;
+    }
+    bool ok = true;
+    for (int n = 0; n < N && ok; ++n) {
+      int kt, cls;
+      plan_item(p.plan, it0 + n, kt, cls);
+      const bool full = is_full(p.fullr, kt, cls);
+      const int buf = n & 1;
+      const uint32_t ph = static_cast<uint32_t>((n >> 1) & 1);
+
+      ok = wait_poll(&ctl->s_full[buf], ph, abort_flag, p.status, p.timeout_ns, ST_SOFTMAX);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      tc_fence_after();
+      uint32_t sv[NR];
+      tmem_ld16(tbase + lane_off + static_cast<uint32_t>(buf * 16), sv);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&ctl->s_free[buf]);
+
+      if (!full) {
+        const int64_t j = static_cast<int64_t>(kt) * BN + tau;
+        const int64_t nj = j / p.s;
+#pragma unroll
+        for (int r = 0; r < NR; ++r) {
+          const int64_t i = row_pos(p, rg, r);
+          const bool valid =
+              j <= i && pair_class(i / p.s - nj, i - j, p.w, p.reading) == cls;
+          if (!valid) sv[r] = 0xff800000u;  // -inf
+        }
+      }
+
+      // row maxima over the warp's 32 keys, then over the four warps
+      float mine = -INFINITY;
+#pragma unroll
+      for (int r = 0; r < NR; ++r) {
+        const int v = __reduce_max_sync(0xffffffffu, ordered(static_cast<int>(sv[r])));
+        if (lane == r) mine = __int_as_float(ordered(v));
+      }
+      if (lane < NR) ctl->wmax[buf][warp][lane] = mine;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&ctl->max_bar[buf]);
+      ok = wait_poll(&ctl->max_bar[buf], ph, abort_flag, p.status, p.timeout_ns, ST_SOFTMAX);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      float tmax[NR];
+#pragma unroll
+      for (int r4 = 0; r4 < NR / 4; ++r4) {
+        float4 a = reinterpret_cast<const float4*>(ctl->wmax[buf][0])[r4];
+#pragma unroll
+        for (int wq = 1; wq < 4; ++wq) {
+          const float4 o = reinterpret_cast<const float4*>(ctl->wmax[buf][wq])[r4];
+          a.x = fmaxf(a.x, o.x);
+          a.y = fmaxf(a.y, o.y);
+          a.z = fmaxf(a.z, o.z);
+          a.w = fmaxf(a.w, o.w);
+        }
+        tmax[4 * r4 + 0] = a.x;
+        tmax[4 * r4 + 1] = a.y;
+        tmax[4 * r4 + 2] = a.z;
+        tmax[4 * r4 + 3] = a.w;
+      }
+
+      // reference update (identical in every thread: same maxima, same history)
+      float alpha[NR];
+      bool any = false;
+#pragma unroll
+      for (int r = 0; r < NR; ++r) {
+        const float m_new = fmaxf(m_ref[r], tmax[r]);
+        const bool need =
+            (m_new > m_ref[r]) && (m_ref[r] == -INFINITY || (m_new - m_ref[r]) * sc > RESCALE_LOG2);
+        alpha[r] = 1.f;
+        if (need) {
+          alpha[r] = (m_ref[r] == -INFINITY) ? 0.f : ex2_approx((m_ref[r] - m_new) * sc);
+          m_ref[r] = m_new;
+          l_part[r] *= alpha[r];
+          any = true;
+        }
+      }
+      float pv[NR];
+#pragma unroll
+      for (int r = 0; r < NR; ++r) {
+        const float mb = (m_ref[r] == -INFINITY) ? 0.f : m_ref[r] * sc;
+        pv[r] = ex2_approx(fmaf(__uint_as_float(sv[r]), sc, -mb));
+        l_part[r] += pv[r];
+      }
+
+      // O^T holds items < n: rescale its columns once the last P.V landed
+      if (any && n > 0) {
+        const int m = n - 1;
+        ok = wait_bounded(&ctl->pv_done[m & 1], static_cast<uint32_t>((m >> 1) & 1), abort_flag,
+                          p.status, p.timeout_ns, ST_SOFTMAX);
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok) break;
+        tc_fence_after();
+        uint32_t o[NR];
+        tmem_ld16(tbase + lane_off + COL_O, o);
+#pragma unroll
+        for (int r = 0; r < NR; ++r) o[r] = __float_as_uint(__uint_as_float(o[r]) * alpha[r]);
+        tmem_st16(tbase + lane_off + COL_O, o);
+        tmem_st_wait();
+      }
+      // the P^T buffer is free once the P.V of item n - 2 completed
+      if (n >= 2) {
+        const int m = n - 2;
+        ok = wait_bounded(&ctl->pv_done[m & 1], static_cast<uint32_t>((m >> 1) & 1), abort_flag,
+                          p.status, p.timeout_ns, ST_SOFTMAX);
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok) break;
+      }
+      uint8_t* pb = pt + buf * OPB + kh * OPB_HALF + ((kin & 7) << 1);
+#pragma unroll
+      for (int r = 0; r < NR; ++r) {
+        const __nv_bfloat16 v = __float2bfloat16_rn(pv[r]);
+        *reinterpret_cast<__nv_bfloat16*>(pb + r * 128 + (((kin >> 3) ^ (r & 7)) << 4)) = v;
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&ctl->p_full[buf]);
+    }
+
+    // ---- epilogue: partial (m, l, O) of this slice
+    if (ok && N > 0) {
+      ok = wait_bounded(&ctl->o_final, 0u, abort_flag, p.status, p.timeout_ns, ST_SOFTMAX);
+      ok = __all_sync(0xffffffffu, ok);
+    }
+    if (ok) {
+      uint32_t o[NR];
+      if (N > 0) {
+        tc_fence_after();
+        tmem_ld16(tbase + lane_off + COL_O, o);
+      } else {
+#pragma unroll
+        for (int r = 0; r < NR; ++r) o[r] = 0u;
+      }
+      float mine = 0.f, mref_mine = -INFINITY;
+#pragma unroll
+      for (int r = 0; r < NR; ++r) {
+        float v = l_part[r];
+#pragma unroll
+        for (int off = 16; off >= 1; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+        if (lane == r) {
+          mine = v;
+          mref_mine = m_ref[r];
+        }
+      }
+      if (lane < NR) ctl->lsum[warp][lane] = mine;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&ctl->epi_bar);
+      ok = wait_bounded(&ctl->epi_bar, 0u, abort_flag, p.status, p.timeout_ns, ST_SOFTMAX);
+      ok = __all_sync(0xffffffffu, ok);
+      if (ok) {
+        float* po = p.part + static_cast<size_t>(cta) * NR * HD;
+        float* pm = p.part + static_cast<size_t>(p.n_cta) * NR * HD + static_cast<size_t>(cta) * NR;
+        float* pl = pm + static_cast<size_t>(p.n_cta) * NR;
+#pragma unroll
+        for (int r = 0; r < NR; ++r)
+          if (r < n_rows) po[r * HD + tau] = __uint_as_float(o[r]);
+        if (warp == 0 && lane < n_rows) {
+          pm[lane] = (mref_mine == -INFINITY) ? -INFINITY : mref_mine * sc;
+          pl[lane] = ctl->lsum[0][lane] + ctl->lsum[1][lane] + ctl->lsum[2][lane] +
+                     ctl->lsum[3][lane];
+        }
+      }
+    }
+  } else if (warp == WARP_LOAD) {
+    // =========================================================== TMA producer
+    if (lane == 0) {
+      int last_li[NTILE];
+#pragma unroll
+      for (int k = 0; k < NTILE; ++k) last_li[k] = -1;
+      bool ok = true;
+      for (int n = 0; n < N && ok; ++n) {
+        int kt, cls;
+        plan_item(p.plan, it0 + n, kt, cls);
+        for (int which = 0; which < 2; ++which) {  // 0: keys, 1: values
+          const int li = 2 * n + which;
+          const int slot = li % NTILE;
+          const int use = li / NTILE;
+          if (use > 0) {
+            ok = wait_bounded(&ctl->tile_empty[slot], static_cast<uint32_t>((use - 1) & 1),
+                              abort_flag, p.status, p.timeout_ns, ST_LOAD);
+            if (!ok) break;
+          }
+          if ((p.debug & 1) && li == 0) continue;  // test hook: withhold the first key tile
+          uint8_t* dst = tiles + slot * TILE_BYTES;
+          const CUtensorMap* tm = which ? &tm_v : &tm_k;
+          mbar_arrive_expect_tx(&ctl->tile_full[slot], TILE_BYTES);
+          tma_load_3d(dst, tm, &ctl->tile_full[slot], 0, g, kt * BN);
+          tma_load_3d(dst + HALF_BYTES, tm, &ctl->tile_full[slot], 64, g, kt * BN);
+          last_li[slot] = li;
+        }
+      }
+      for (int k = 0; k < NTILE; ++k)
+        if (last_li[k] >= 0)
+          wait_drain(&ctl->tile_full[k], static_cast<uint32_t>((last_li[k] / NTILE) & 1),
+                     p.status, p.timeout_ns, ST_DRAIN);
+    }
+    __syncwarp();
+  } else if (warp == WARP_MMA) {
+    // =========================================================== MMA issuer
+    if (lane == 0) {
+      const uint32_t id_s = idesc_bf16_f32_major(BN, NR, false, false);
+      const uint32_t id_o = idesc_bf16_f32_major(HD, NR, true, false);
+      // Descriptors built once; a k-step or buffer adds its byte offset / 16
+      // to the start-address field (shared addresses stay below 256 KiB).
+      const uint64_t dq0 = sdesc_sw128(smem_u32(qv), 16, 1024);
+      const uint64_t dp0 = sdesc_sw128(smem_u32(pt), 16, 1024);
+      const uint64_t dk0 = sdesc_sw128(smem_u32(tiles), 16, 1024);
+      const uint64_t dv0 = sdesc_sw128(smem_u32(tiles), HALF_BYTES, 1024);
+      auto tile_wait = [&](int li) {
+        return wait_spin(&ctl->tile_full[li % NTILE], static_cast<uint32_t>((li / NTILE) & 1),
+                         abort_flag, p.status, p.timeout_ns, ST_MMA);
+      };
+      bool ok = wait_bounded(&ctl->q_ready, 0u, abort_flag, p.status, p.timeout_ns, ST_MMA);
+      for (int n = 0; n <= N && ok; ++n) {
+        if (n < N) {
+          int kt, cls;
+          plan_item(p.plan, it0 + n, kt, cls);
+          const int li = 2 * n;
+          ok = tile_wait(li);
+          if (!ok) break;
+          if (n >= 2) {
+            ok = wait_spin(&ctl->s_free[n & 1], static_cast<uint32_t>(((n - 2) >> 1) & 1),
+                           abort_flag, p.status, p.timeout_ns, ST_MMA);
+            if (!ok) break;
+          }
+          tc_fence_after();
+          const uint64_t dk = dk0 + static_cast<uint64_t>(((li % NTILE) * TILE_BYTES) >> 4);
+          const uint64_t dq = dq0 + static_cast<uint64_t>((cls * OPB) >> 4);
+#pragma unroll
+          for (int kk = 0; kk < HD / 16; ++kk) {
+            const uint64_t ka = static_cast<uint64_t>(((kk >> 2) * HALF_BYTES + (kk & 3) * 32) >> 4);
+            const uint64_t kb = static_cast<uint64_t>(((kk >> 2) * OPB_HALF + (kk & 3) * 32) >> 4);
+            mma_ss(tbase + static_cast<uint32_t>((n & 1) * 16), dk + ka, dq + kb, id_s,
+                   kk > 0 ? 1u : 0u);
+          }
+          mma_commit(&ctl->s_full[n & 1]);
+          mma_commit(&ctl->tile_empty[li % NTILE]);
+        }
+        if (n >= 1) {
+          const int m = n - 1;
+          const int lv = 2 * m + 1;
+          ok = tile_wait(lv);
+          if (!ok) break;
+          ok = wait_spin(&ctl->p_full[m & 1], static_cast<uint32_t>((m >> 1) & 1), abort_flag,
+                         p.status, p.timeout_ns, ST_MMA);
+          if (!ok) break;
+          tc_fence_after();
+          const uint64_t dv = dv0 + static_cast<uint64_t>(((lv % NTILE) * TILE_BYTES) >> 4);
+          const uint64_t dp = dp0 + static_cast<uint64_t>(((m & 1) * OPB) >> 4);
+#pragma unroll
+          for (int kk = 0; kk < BN / 16; ++kk) {
+            const uint64_t kb = static_cast<uint64_t>(((kk >> 2) * OPB_HALF + (kk & 3) * 32) >> 4);
+            mma_ss(tbase + COL_O, dv + static_cast<uint64_t>((kk * 2048) >> 4), dp + kb, id_o,
+                   (m > 0 || kk > 0) ? 1u : 0u);
+          }
+          mma_commit(&ctl->pv_done[m & 1]);
+          mma_commit(&ctl->tile_empty[lv % NTILE]);
+        }
+      }
+      if (ok && N > 0) mma_commit(&ctl->o_final);
+      // no MMA may still be running when TMEM is released
+      mma_commit(&ctl->drain);
+      wait_drain(&ctl->drain, 0u, p.status, p.timeout_ns, ST_DRAIN);
+    }
+    __syncwarp();
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == WARP_MMA) {
+    tc_fence_after();
+    tmem_dealloc(tbase, TMEM_COLS);
+  }
+}
+
+// Merge the slices of each (token, head) row: with slice maxima m_k (log2
+// units), sums l_k and unnormalised outputs O_k, out = sum_k 2^(m_k - M) O_k /
+// sum_k 2^(m_k - M) l_k with M = max m_k; LSE (natural log) = (M + log2 of the
+// denominator) ln 2.  One CTA per row, one thread per dim.
+__global__ void __launch_bounds__(HD)
+    dca_decode_combine_kernel(const float* __restrict__ part, __nv_bfloat16* __restrict__ out,
+                              float* __restrict__ lse, int Hq, int G, int n_rg, int n_splits,
+                              int n_cta) {
+  const int row = static_cast<int>(blockIdx.x);  // t * Hq + h
+  const int t = row / Hq, h = row % Hq;
+  const int g = h / G;
+  const int rho_g = t * G + (h % G);
+  const int rg = rho_g / NR, rho = rho_g % NR;
+  const int c0 = (g * n_rg + rg) * n_splits;
+  const float* pm = part + static_cast<size_t>(n_cta) * NR * HD;
+  const float* pl = pm + static_cast<size_t>(n_cta) * NR;
+  float M = -INFINITY;
+  for (int k = 0; k < n_splits; ++k) M = fmaxf(M, pm[(c0 + k) * NR + rho]);
+  float L = 0.f, acc = 0.f;
+  for (int k = 0; k < n_splits; ++k) {
+    const float mk = pm[(c0 + k) * NR + rho];
+    if (mk == -INFINITY) continue;
+    const float wk = exp2f(mk - M);
+    L = fmaf(wk, pl[(c0 + k) * NR + rho], L);
+    acc = fmaf(wk, part[(static_cast<size_t>(c0 + k) * NR + rho) * HD + threadIdx.x], acc);
+  }
+  out[static_cast<size_t>(row) * HD + threadIdx.x] = __float2bfloat16_rn(acc / L);
+  if (lse != nullptr && threadIdx.x == 0) lse[row] = (M + log2f(L)) * 0.6931471805599453f;
+}
+
+}  // namespace dec
+
+cudaError_t launch_decode_sm100(const AttnArgs& a, float* part, cudaStream_t st) {
+  using namespace dec;
+  if (a.Lq <= 0) return cudaSuccess;
+  CUtensorMap tm_k, tm_v;
+  if (!encode_kv_map(&tm_k, a.kr, a.Lk, a.Hkv) || !encode_kv_map(&tm_v, a.v, a.Lk, a.Hkv))
+    return cudaErrorInvalidValue;
+  Params p;
+  p.q = static_cast<const __nv_bfloat16*>(a.q);
+  p.tab = a.tab;
+  p.part = part;
+  p.q_start = a.q_start;
+  p.Lq = a.Lq;
+  p.Lk = a.Lk;
+  p.s = a.s;
+  p.w = a.w;
+  p.tab_c1 = a.tab_c1;
+  p.Hq = a.Hq;
+  p.Hkv = a.Hkv;
+  p.G = a.Hq / a.Hkv;
+  p.reading = a.reading;
+  p.scale_log2 = a.scale_log2;
+  p.status = a.status;
+  p.timeout_ns = a.timeout_ns;
+  p.debug = a.debug;
+  const int64_t i_last = a.q_start + a.Lq - 1;
+  p.plan = make_plan(a.q_start, i_last, a.s, a.w, BN, a.reading);
+  p.fullr = make_full_ranges(a.q_start, i_last, a.s, a.w, BN, a.reading);
+  p.n_rg = decode_row_groups(a.Lq, p.G);
+  const int max_splits = decode_max_splits(a.Hkv, p.n_rg);
+  p.n_splits = p.plan.n_items < max_splits ? p.plan.n_items : max_splits;
+  if (p.n_splits < 1) p.n_splits = 1;
+  const int64_t n_cta = static_cast<int64_t>(a.Hkv) * p.n_rg * p.n_splits;
+  if (n_cta > 0x7fffffffLL || a.Lq * a.Hq > 0x7fffffffLL) return cudaErrorInvalidValue;
+  p.n_cta = static_cast<int>(n_cta);
+  cudaError_t e = cudaFuncSetAttribute(dca_decode_kernel,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(SMEM_BYTES));
+  if (e != cudaSuccess) return e;
+  dca_decode_kernel<<<static_cast<unsigned>(n_cta), NUM_THREADS, SMEM_BYTES, st>>>(tm_k, tm_v, p);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  dca_decode_combine_kernel<<<static_cast<unsigned>(a.Lq * a.Hq), HD, 0, st>>>(
+      part, static_cast<__nv_bfloat16*>(a.out), a.lse, a.Hq, p.G, p.n_rg, p.n_splits, p.n_cta);
+  return cudaGetLastError();
+}
+
+}  // namespace dca

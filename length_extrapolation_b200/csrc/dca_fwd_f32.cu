@@ -34,6 +34,7 @@ struct Params {
   int Hq, Hkv, G, n_qtiles;
   int reading;
   float scale_log2;
+  float* lse;  // optional [Lq][Hq] natural-log LSE
 };
 
 __global__ void __launch_bounds__(THREADS) dca_fwd_f32_kernel(const Params p) {
@@ -179,6 +180,9 @@ __global__ void __launch_bounds__(THREADS) dca_fwd_f32_kernel(const Params p) {
     const float inv = 1.f / l_run[a];
 #pragma unroll
     for (int u = 0; u < 8; ++u) orow[cg + 16 * u] = O[a][u] * inv;
+    // p = 2^(S sc - m sc), so ln sum_j e^(z_j) = (m sc + log2 l) ln 2
+    if (p.lse != nullptr && cg == 0)
+      p.lse[(i - p.q_start) * p.Hq + h] = (m_run[a] * sc + log2f(l_run[a])) * 0.6931471805599453f;
   }
 }
 
@@ -205,6 +209,7 @@ cudaError_t launch_attention_f32(const AttnArgs& a, cudaStream_t st) {
   p.n_qtiles = static_cast<int>((a.Lq + BM - 1) / BM);
   p.reading = a.reading;
   p.scale_log2 = a.scale_log2;
+  p.lse = a.lse;
   const int64_t blocks = static_cast<int64_t>(p.n_qtiles) * p.Hq;
   if (blocks > 0x7fffffffLL) return cudaErrorInvalidValue;
   cudaError_t e = cudaFuncSetAttribute(dca_fwd_f32_kernel,

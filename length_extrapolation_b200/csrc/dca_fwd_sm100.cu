@@ -651,6 +651,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   }
 }
 
+}  // namespace sm100
+
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
@@ -672,7 +674,7 @@ static EncodeTiledFn get_encode_fn() {
 
 // [rows][Hkv][128] bf16 as a 3-D tensor (dims, Hkv, rows); boxes of 64 dims x
 // 1 head x 128 rows with 128-byte swizzle; rows >= n_rows read as zeros.
-static bool encode_kv_map(CUtensorMap* m, const void* base, int64_t n_rows, int Hkv) {
+bool encode_kv_map(CUtensorMap* m, const void* base, int64_t n_rows, int Hkv) {
   EncodeTiledFn fn = get_encode_fn();
   if (fn == nullptr) return false;
   const cuuint64_t dims[3] = {128u, static_cast<cuuint64_t>(Hkv), static_cast<cuuint64_t>(n_rows)};
@@ -683,8 +685,6 @@ static bool encode_kv_map(CUtensorMap* m, const void* base, int64_t n_rows, int 
             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
-
-}  // namespace sm100
 
 cudaError_t launch_attention_sm100(const AttnArgs& a, cudaStream_t st) {
   using namespace sm100;

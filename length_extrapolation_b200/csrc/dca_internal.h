@@ -21,17 +21,42 @@ struct AttnArgs {
   unsigned int* status; // device status word (workspace header)
   unsigned long long timeout_ns;
   int debug;
+  float* lse = nullptr;  // optional [Lq][Hq] natural-log LSE (fp32 kernel and decode only)
 };
+
+// Split-KV decode: a few query rows against a long cache.  CTAs per
+// (KV head, row group) and the partial-result scratch they write.
+constexpr int DECODE_ROWS = 16;      // query rows per row group (MMA N)
+constexpr int DECODE_MAX_CTAS = 148; // one CTA per SM of a B200
+inline int decode_row_groups(int64_t Lq, int G) {
+  return static_cast<int>((Lq * G + DECODE_ROWS - 1) / DECODE_ROWS);
+}
+inline int decode_max_splits(int Hkv, int n_rg) {
+  const int per = DECODE_MAX_CTAS / (Hkv * n_rg);
+  return per > 1 ? per : 1;
+}
+// fp32 words of partial results: O [cta][16][128], then m, l [cta][16].
+inline size_t decode_part_floats(int n_cta) {
+  return static_cast<size_t>(n_cta) * DECODE_ROWS * (128 + 2);
+}
 
 cudaError_t launch_rope_table(float2* tab, int64_t T, int64_t n_direct, int64_t c, double base,
                               int d, cudaStream_t st);
 cudaError_t launch_rotate_keys(const void* k, void* kr, const float2* tab, int64_t j_begin,
                                int64_t j_end, int Hkv, int64_t s, int dtype, cudaStream_t st);
 
+// Tensor map of a [rows][Hkv][128] bf16 tensor for boxes of 64 dims x 1 head x
+// 128 rows, 128-byte swizzle, rows >= n_rows read as zeros; false if the
+// driver's encoder is unavailable or rejects the map.
+bool encode_kv_map(CUtensorMap* m, const void* base, int64_t n_rows, int Hkv);
+
 // bf16 tcgen05/TMA kernel; returns a CUDA error or cudaSuccess, or
 // cudaErrorInvalidValue when a tensor map cannot be encoded.
 cudaError_t launch_attention_sm100(const AttnArgs& a, cudaStream_t st);
-// fp32 CUDA-core kernel.
+// fp32 CUDA-core kernel (writes a.lse when set).
 cudaError_t launch_attention_f32(const AttnArgs& a, cudaStream_t st);
+// bf16 split-KV decode (tcgen05) and the combine of its partial results into
+// out (and a.lse when set); `part` holds decode_part_floats(...) words.
+cudaError_t launch_decode_sm100(const AttnArgs& a, float* part, cudaStream_t st);
 
 }  // namespace dca

@@ -49,7 +49,7 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 // Wait for phase `parity` of `bar` to complete.  Gives up (returns false)
 // when another role of the CTA raised `abort`, or after `timeout_ns`, in
 // which case it raises `abort` and ORs `code` into the device status word.
-__device__ __noinline__ bool wait_bounded(uint64_t* bar, uint32_t parity, volatile int* abort,
+static __device__ __noinline__ bool wait_bounded(uint64_t* bar, uint32_t parity, volatile int* abort,
                                           unsigned int* status, uint64_t timeout_ns,
                                           unsigned int code) {
   if (mbar_try_wait(bar, parity)) return true;
@@ -140,7 +140,7 @@ __device__ __forceinline__ bool wait_warp(uint64_t* bar, uint32_t parity, volati
 
 // Same, ignoring the abort flag (used to drain copies and MMAs in flight
 // before the CTA exits); bounded by time only.
-__device__ __noinline__ bool wait_drain(uint64_t* bar, uint32_t parity, unsigned int* status,
+static __device__ __noinline__ bool wait_drain(uint64_t* bar, uint32_t parity, unsigned int* status,
                                         uint64_t timeout_ns, unsigned int code) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
@@ -242,6 +242,36 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool b_mn_ma
          | ((b_mn_major ? 1u : 0u) << 16)           // B major
          | (static_cast<uint32_t>(N >> 3) << 17)    // N / 8
          | (static_cast<uint32_t>(M >> 4) << 24);   // M / 16
+}
+
+// Instruction descriptor for kind::f16 with bf16 A/B, fp32 D and either
+// operand stored MN-major (M- or N-contiguous) instead of K-major.
+__host__ __device__ constexpr uint32_t idesc_bf16_f32_major(int M, int N, bool a_mn_major,
+                                                            bool b_mn_major) {
+  return idesc_bf16_f32(M, N, b_mn_major) | ((a_mn_major ? 1u : 0u) << 15);
+}
+
+// 32 lanes x 16 columns of 32-bit TMEM words -> 16 registers per thread; waits.
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t* r) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];\n\t"
+      "tcgen05.wait::ld.sync.aligned;"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+        "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr)
+      : "memory");
+}
+// r[0..15] -> 16 TMEM columns of this thread's lane (call tmem_st_wait before use).
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t* r) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
+      "r"(r[15])
+      : "memory");
 }
 
 // 32 lanes x 32 columns of 32-bit TMEM words -> 32 registers per thread

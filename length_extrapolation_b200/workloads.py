@@ -106,25 +106,65 @@ def generate(w: Workload, device="cpu", seed: int = 0, L: Optional[int] = None):
     L = w.L if L is None else L
     g = torch.Generator(device=device)
     g.manual_seed(seed)
+    q = _draw(w, g, L, w.Hq, device)
+    k = _draw(w, g, L, w.Hkv, device)
+    v = _draw(w, g, L, w.Hkv, device)
+    _add_sinks(w, g, k, device)
+    return q, k, v
+
+
+def _draw(w: Workload, g, rows: int, H: int, device):
+    """[rows, H, d] i.i.d. normal (scaled by 1/sqrt(d) when the workload says
+    so), drawn in fp32 per slab and rounded to the storage dtype."""
     scale = 1.0 / math.sqrt(w.d) if w.scale_by_sqrt_d else 1.0
-    out = []
-    for H in (w.Hq, w.Hkv, w.Hkv):
-        x = torch.empty((L, H, w.d), dtype=w.torch_dtype, device=device)
-        # draw per slab to bound the fp32 temporary at full size
-        step = max(1, (1 << 27) // max(1, H * w.d))
-        for r0 in range(0, L, step):
-            r1 = min(L, r0 + step)
-            t = torch.randn((r1 - r0, H, w.d), generator=g, device=device, dtype=torch.float32)
-            if scale != 1.0:
-                t.mul_(scale)
-            x[r0:r1] = t.to(w.torch_dtype)
-            del t
-        out.append(x)
-    q, k, v = out
-    n_sinks = int(math.floor(w.sink_fraction * L))
+    x = torch.empty((rows, H, w.d), dtype=w.torch_dtype, device=device)
+    # draw per slab to bound the fp32 temporary at full size
+    step = max(1, (1 << 27) // max(1, H * w.d))
+    for r0 in range(0, rows, step):
+        r1 = min(rows, r0 + step)
+        t = torch.randn((r1 - r0, H, w.d), generator=g, device=device, dtype=torch.float32)
+        if scale != 1.0:
+            t.mul_(scale)
+        x[r0:r1] = t.to(w.torch_dtype)
+        del t
+    return x
+
+
+def _add_sinks(w: Workload, g, k, device):
+    """Scale the keys at the first floor(fraction * rows) entries of a random permutation."""
+    n = k.shape[0]
+    n_sinks = int(math.floor(w.sink_fraction * n))
     if n_sinks > 0:
-        idx = torch.randperm(L, generator=g, device=device)[:n_sinks]
+        idx = torch.randperm(n, generator=g, device=device)[:n_sinks]
         k[idx] = (k[idx].float() * w.sink_scale).to(w.torch_dtype)
+
+
+@dataclasses.dataclass(frozen=True)
+class DecodeWorkload:
+    """A decode step: Lq new query tokens at positions [Lk - Lq, Lk) against a
+    cache of Lk keys, with the DCA parameters and head shapes of `base`."""
+    name: str
+    base: Workload
+    Lk: int
+    Lq: int
+
+    def kv_bytes(self) -> int:
+        """Bytes of rotated keys and values one step streams (all KV heads)."""
+        esize = 2 if self.base.dtype == "bf16" else 4
+        return 2 * self.Lk * self.base.Hkv * self.base.d * esize
+
+
+def generate_decode(dw: DecodeWorkload, device="cpu", seed: int = 0):
+    """Seeded q [Lq,Hq,d] (the new tokens), k, v [Lk,Hkv,d]: the draws of
+    ``generate`` in the same order (q, k, v, sink indices) with q holding only
+    the Lq new rows."""
+    w = dw.base
+    g = torch.Generator(device=device)
+    g.manual_seed(seed)
+    q = _draw(w, g, dw.Lq, w.Hq, device)
+    k = _draw(w, g, dw.Lk, w.Hkv, device)
+    v = _draw(w, g, dw.Lk, w.Hkv, device)
+    _add_sinks(w, g, k, device)
     return q, k, v
 
 
@@ -153,3 +193,16 @@ def sample_heads(w: Workload):
     """Heads 0, G-1, G, Hq-1 (first/last head of the first two KV groups and the last head)."""
     hs = sorted({0, w.G - 1, min(w.G, w.Hq - 1), w.Hq - 1})
     return torch.tensor(hs, dtype=torch.int32)
+
+
+# Decode steps after the prefills above: the next token (Lq = 1), and four
+# tokens at once (e.g. verifying draft tokens), at the full context length.
+DECODE_WORKLOADS = {
+    dw.name: dw
+    for dw in [
+        DecodeWorkload("qwen7b_32k_decode", WORKLOADS["qwen7b_32k"], Lk=32768, Lq=1),
+        DecodeWorkload("qwen7b_256k_decode", WORKLOADS["qwen7b_256k"], Lk=262144, Lq=1),
+        DecodeWorkload("qwen7b_1m_decode", WORKLOADS["qwen7b_1m_chunked"], Lk=1048576, Lq=1),
+        DecodeWorkload("qwen7b_1m_decode_q4", WORKLOADS["qwen7b_1m_chunked"], Lk=1048576, Lq=4),
+    ]
+}
