@@ -133,9 +133,11 @@ bool ptrs_ok(const void* p) { return p != nullptr && aligned(p, 16); }
 // Scratch bytes of a decode call (0 for invalid sizes).
 size_t decode_scratch_bytes(int64_t Lq, int Hq, int Hkv) {
   if (Lq < 1 || Lq > DCA_DECODE_MAX_TOKENS || Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0) return 0;
-  const int n_rg = dca::decode_row_groups(Lq, Hq / Hkv);
+  const int G = Hq / Hkv;
+  const int n_rg = dca::decode_row_groups(Lq, G);
   const int n_cta = Hkv * n_rg * dca::decode_max_splits(Hkv, n_rg);
-  return align_up(dca::decode_part_floats(n_cta) * sizeof(float), 256);
+  return align_up(dca::decode_part_floats(n_cta, dca::decode_group_rows(Lq, G)) * sizeof(float),
+                  256);
 }
 
 // Window reading from the options (NULL = defaults); -1 when invalid.

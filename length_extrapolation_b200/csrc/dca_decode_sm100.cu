@@ -9,20 +9,21 @@
 // whole cache (2 x 256 bytes per key and KV head) and HBM-bound, so the
 // kernel is split-KV: the work list of the query block (dca_plan.cuh) is cut
 // into contiguous slices, one CTA per (KV head, row group, slice), and a
-// combine kernel merges the slices' partial softmax states.
+// merge kernel combines the slices' partial softmax states.
 //
-// One CTA (192 threads):
-//   warps 0-3  softmax: thread t owns key t of the current 128-key tile (TMEM
-//              lane t of S^T) and dim t of O^T
-//   warp 4     TMA producer: K'/V tiles (128 keys x 128 dims, bf16, 128-byte
-//              swizzle) into a ring of six 32 KiB slots (no multicast)
-//   warp 5     MMA issuer: S^T = K' Q_cls^T (M = 128 keys, N = 16 query rows)
-//              and O^T += V^T P^T (M = 128 dims, A = V tile read MN-major,
-//              B = P^T in shared memory), tcgen05.mma kind::f16, fp32 in TMEM
-// The G query heads of a KV head share its K'/V stream: up to 16 (token,
-// head) rows per row group; a row group is one MMA N.  Query rows are
-// rotated once per class at the start (three 4 KiB operand tiles).
-// Online softmax per row: the four softmax warps exchange their per-row tile
+// A row group is NR = 16 or 32 (token, head) rows of one KV head: the MMA N.
+// One CTA (SW = NR/4 softmax warps + 2):
+//   softmax warps  warp w owns TMEM lane quarter w % 4 -- key 32(w%4) + lane
+//                  of the current 128-key tile in S^T, the same dim of O^T --
+//                  and rows 16(w/4) .. +15 of the group
+//   warp SW        TMA producer: K'/V tiles (128 keys x 128 dims, bf16,
+//                  128-byte swizzle) into a ring of 32 KiB slots (no multicast)
+//   warp SW+1      MMA issuer: S^T = K' Q_cls^T (M = 128 keys, N = NR rows)
+//                  and O^T += V^T P^T (M = 128 dims, A = the V tile read
+//                  MN-major, B = P^T in shared memory), tcgen05.mma kind::f16,
+//                  fp32 accumulators in TMEM
+// Query rows are rotated once per class at the start (three operand tiles).
+// Online softmax per row: the four warps of a row half exchange their tile
 // maxima through shared memory; the reference max moves (and O^T, l rescale)
 // only when it grows by more than 2^8, as in the prefill kernel.
 // Every wait is bounded (globaltimer); on timeout the CTA raises its abort
@@ -39,42 +40,52 @@ namespace dca {
 namespace dec {
 
 constexpr int BN = 128;                  // keys per tile (MMA M of S^T)
-constexpr int NR = DECODE_ROWS;          // query rows per CTA (MMA N)
 constexpr int HD = 128;
-constexpr int NTILE = 6;                 // K'/V tile ring
 constexpr int TILE_BYTES = 32768;        // 128 x 128 bf16
 constexpr int HALF_BYTES = 16384;        // 128 rows x 64 bf16 (one swizzle column block)
-constexpr int OPB = NR * HD * 2;         // 4 KiB: a 16-row operand (Q variant or P^T)
-constexpr int OPB_HALF = NR * 128;       // 2 KiB: its 64-column block
-constexpr int NUM_THREADS = 192;
-constexpr int WARP_LOAD = 4;
-constexpr int WARP_MMA = 5;
-constexpr uint32_t TMEM_COLS = 64;       // S^T x2 (16 cols each), O^T (16 cols)
-constexpr uint32_t COL_O = 32;
 constexpr float RESCALE_LOG2 = 8.0f;
 
 constexpr unsigned ST_SOFTMAX = 0x10u, ST_LOAD = 0x100u, ST_MMA = 0x1000u, ST_DRAIN = 0x10000u;
 
+template <int NR>
+struct Cfg {
+  static_assert(NR == 16 || NR == 32, "row group of 16 or 32");
+  static constexpr int SW = NR / 4;                     // softmax warps
+  static constexpr int NTILE = NR == 16 ? 6 : 5;        // K'/V tile ring
+  static constexpr int OPB = NR * HD * 2;               // an NR-row operand (Q variant or P^T)
+  static constexpr int OPB_HALF = NR * 128;             // its 64-column block
+  static constexpr int THREADS = 32 * (SW + 2);
+  static constexpr int WARP_LOAD = SW;
+  static constexpr int WARP_MMA = SW + 1;
+  static constexpr uint32_t TMEM_COLS = NR == 16 ? 64 : 128;  // S^T x2, O^T (NR cols each)
+  static constexpr uint32_t COL_O = 2 * NR;
+};
+
+template <int NR>
 struct SmemCtl {
-  uint64_t tile_full[NTILE];
-  uint64_t tile_empty[NTILE];
+  static constexpr int SW = Cfg<NR>::SW;
+  uint64_t tile_full[Cfg<NR>::NTILE];
+  uint64_t tile_empty[Cfg<NR>::NTILE];
   uint64_t s_full[2];
-  uint64_t s_free[2];   // four softmax warps have read S^T
-  uint64_t p_full[2];   // four softmax warps have written P^T
+  uint64_t s_free[2];   // the softmax warps have read S^T
+  uint64_t p_full[2];   // the softmax warps have written P^T
   uint64_t pv_done[2];  // O^T += V^T P^T of the item with this parity completed
-  uint64_t max_bar[2];  // four warps' row maxima are in wmax
+  uint64_t max_bar[2];  // the warps' row maxima are in wmax
   uint64_t q_ready;
   uint64_t o_final;
   uint64_t epi_bar;
   uint64_t drain;
   uint32_t tmem_base;
   int abort;
-  alignas(16) float wmax[2][4][NR];  // read as float4
-  float lsum[4][NR];
+  alignas(16) float wmax[2][SW][16];  // read as float4
+  float lsum[SW][16];
 };
 
-constexpr size_t SMEM_BYTES = 1024 + NTILE * TILE_BYTES + 3 * OPB + 2 * OPB + sizeof(SmemCtl);
-static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+template <int NR>
+constexpr size_t smem_bytes() {
+  return 1024 + Cfg<NR>::NTILE * TILE_BYTES + 5 * Cfg<NR>::OPB + sizeof(SmemCtl<NR>);
+}
+static_assert(smem_bytes<16>() <= 232448 && smem_bytes<32>() <= 232448, "shared memory budget");
 
 struct Params {
   const __nv_bfloat16* q;   // [Lq][Hq][128]
@@ -100,22 +111,26 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
 }
 
 // Absolute position of row rho of row group rg (padding rows repeat the last row).
+template <int NR>
 __device__ __forceinline__ int64_t row_pos(const Params& p, int rg, int rho) {
   int64_t t = (static_cast<int64_t>(rg) * NR + rho) / p.G;
   if (t > p.Lq - 1) t = p.Lq - 1;
   return p.q_start + t;
 }
 
-__global__ void __launch_bounds__(NUM_THREADS, 1)
+template <int NR>
+__global__ void __launch_bounds__(Cfg<NR>::THREADS, 1)
     dca_decode_kernel(const __grid_constant__ CUtensorMap tm_k,
                       const __grid_constant__ CUtensorMap tm_v, const Params p) {
+  using C = Cfg<NR>;
+  constexpr int SW = C::SW, NTILE = C::NTILE, OPB = C::OPB, OPB_HALF = C::OPB_HALF;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   uint8_t* tiles = smem;
   uint8_t* qv = tiles + NTILE * TILE_BYTES;  // Q variants, indexed by class
   uint8_t* pt = qv + 3 * OPB;                // P^T, two buffers
-  SmemCtl* ctl = reinterpret_cast<SmemCtl*>(pt + 2 * OPB);
+  SmemCtl<NR>* ctl = reinterpret_cast<SmemCtl<NR>*>(pt + 2 * OPB);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -130,10 +145,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const int it0 = static_cast<int>(static_cast<int64_t>(p.plan.n_items) * sp / p.n_splits);
   const int it1 = static_cast<int>(static_cast<int64_t>(p.plan.n_items) * (sp + 1) / p.n_splits);
   const int N = it1 - it0;
-  const int64_t rows_total = p.Lq * p.G;
-  const int n_rows = static_cast<int>(
-      rows_total - static_cast<int64_t>(rg) * NR < NR ? rows_total - static_cast<int64_t>(rg) * NR
-                                                      : NR);
+  const int64_t rows_left = p.Lq * p.G - static_cast<int64_t>(rg) * NR;
+  const int n_rows = static_cast<int>(rows_left < NR ? rows_left : NR);
 
   if (threadIdx.x == 0) {
     for (int k = 0; k < NTILE; ++k) {
@@ -142,23 +155,23 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
     for (int k = 0; k < 2; ++k) {
       mbar_init(&ctl->s_full[k], 1);
-      mbar_init(&ctl->s_free[k], 4);
-      mbar_init(&ctl->p_full[k], 4);
+      mbar_init(&ctl->s_free[k], SW);
+      mbar_init(&ctl->p_full[k], SW);
       mbar_init(&ctl->pv_done[k], 1);
-      mbar_init(&ctl->max_bar[k], 4);
+      mbar_init(&ctl->max_bar[k], SW);
     }
-    mbar_init(&ctl->q_ready, 4);
+    mbar_init(&ctl->q_ready, SW);
     mbar_init(&ctl->o_final, 1);
-    mbar_init(&ctl->epi_bar, 4);
+    mbar_init(&ctl->epi_bar, SW);
     mbar_init(&ctl->drain, 1);
     ctl->abort = 0;
     fence_barrier_init();
   }
-  if (warp == WARP_MMA) {
-    tmem_alloc(&ctl->tmem_base, TMEM_COLS);
+  if (warp == C::WARP_MMA) {
+    tmem_alloc(&ctl->tmem_base, C::TMEM_COLS);
     tmem_relinquish();
   }
-  if (warp == WARP_LOAD && lane == 0) {
+  if (warp == C::WARP_LOAD && lane == 0) {
     tma_prefetch_desc(&tm_k);
     tma_prefetch_desc(&tm_v);
   }
@@ -168,20 +181,22 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const uint32_t tbase = ctl->tmem_base;
   volatile int* abort_flag = &ctl->abort;
 
-  if (warp < 4) {
+  if (warp < SW) {
     // =========================================================== softmax
-    const int tau = warp * 32 + lane;
-    const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+    const int quad = warp & 3;        // TMEM lane quarter: keys / dims 32*quad + lane
+    const int rh = warp >> 2;         // rows 16*rh .. 16*rh + 15 of the group
+    const int tau = quad * 32 + lane;
+    const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
     const float sc = p.scale_log2;
 
-    // The rotated query operands (16 rows x 128 dims, K-major, 128-byte
+    // The rotated query operands (NR rows x 128 dims, K-major, 128-byte
     // swizzle) of the classes in the work list (the RoPE table holds the
     // positions s + r only when the cache extends past the first chunk, which
     // is when the list has successive-chunk items); task = (class, row,
     // 8-dim chunk of each half).
-    for (int task = tau; task < 3 * NR * 8; task += 128) {
-      const int cls = task >> 7;
-      const int rho = (task >> 3) & (NR - 1);
+    for (int task = warp * 32 + lane; task < 3 * NR * 8; task += 32 * SW) {
+      const int cls = task / (NR * 8);
+      const int rho = (task >> 3) % NR;
       const int c = task & 7;
       uint4 oa = make_uint4(0, 0, 0, 0), ob = oa;
       if (rho < n_rows && p.plan.hi[cls] > p.plan.lo[cls]) {
@@ -215,13 +230,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     __syncwarp();
     if (lane == 0) mbar_arrive(&ctl->q_ready);
 
-    // P^T store address of this thread's key for row 0 (rows add 128 bytes
-    // and change the swizzle phase)
+    // P^T store address of this thread's key (rows add 128 bytes and change
+    // the swizzle phase)
     const int kh = tau >> 6, kin = tau & 63;
 
-    float m_ref[NR], l_part[NR];
+    float m_ref[16], l_part[16];
 #pragma unroll
-    for (int r = 0; r < NR; ++r) {
+    for (int r = 0; r < 16; ++r) {
       m_ref[r] = -INFINITY;
       l_part[r] = 0.f;
     }
@@ -237,8 +252,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
       tc_fence_after();
-      uint32_t sv[NR];
-      tmem_ld16(tbase + lane_off + static_cast<uint32_t>(buf * 16), sv);
+      uint32_t sv[16];
+      tmem_ld16(tbase + lane_off + static_cast<uint32_t>(buf * NR + 16 * rh), sv);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&ctl->s_free[buf]);
@@ -247,34 +262,34 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const int64_t j = static_cast<int64_t>(kt) * BN + tau;
         const int64_t nj = j / p.s;
 #pragma unroll
-        for (int r = 0; r < NR; ++r) {
-          const int64_t i = row_pos(p, rg, r);
+        for (int r = 0; r < 16; ++r) {
+          const int64_t i = row_pos<NR>(p, rg, 16 * rh + r);
           const bool valid =
               j <= i && pair_class(i / p.s - nj, i - j, p.w, p.reading) == cls;
           if (!valid) sv[r] = 0xff800000u;  // -inf
         }
       }
 
-      // row maxima over the warp's 32 keys, then over the four warps
+      // row maxima over the warp's 32 keys, then over the row half's four warps
       float mine = -INFINITY;
 #pragma unroll
-      for (int r = 0; r < NR; ++r) {
+      for (int r = 0; r < 16; ++r) {
         const int v = __reduce_max_sync(0xffffffffu, ordered(static_cast<int>(sv[r])));
         if (lane == r) mine = __int_as_float(ordered(v));
       }
-      if (lane < NR) ctl->wmax[buf][warp][lane] = mine;
+      if (lane < 16) ctl->wmax[buf][warp][lane] = mine;
       __syncwarp();
       if (lane == 0) mbar_arrive(&ctl->max_bar[buf]);
       ok = wait_poll(&ctl->max_bar[buf], ph, abort_flag, p.status, p.timeout_ns, ST_SOFTMAX);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
-      float tmax[NR];
+      float tmax[16];
 #pragma unroll
-      for (int r4 = 0; r4 < NR / 4; ++r4) {
-        float4 a = reinterpret_cast<const float4*>(ctl->wmax[buf][0])[r4];
+      for (int r4 = 0; r4 < 4; ++r4) {
+        float4 a = reinterpret_cast<const float4*>(ctl->wmax[buf][4 * rh])[r4];
 #pragma unroll
         for (int wq = 1; wq < 4; ++wq) {
-          const float4 o = reinterpret_cast<const float4*>(ctl->wmax[buf][wq])[r4];
+          const float4 o = reinterpret_cast<const float4*>(ctl->wmax[buf][4 * rh + wq])[r4];
           a.x = fmaxf(a.x, o.x);
           a.y = fmaxf(a.y, o.y);
           a.z = fmaxf(a.z, o.z);
@@ -286,11 +301,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         tmax[4 * r4 + 3] = a.w;
       }
 
-      // reference update (identical in every thread: same maxima, same history)
-      float alpha[NR];
+      // reference update (identical in the four warps of a row half: same
+      // maxima, same history)
+      float alpha[16];
       bool any = false;
 #pragma unroll
-      for (int r = 0; r < NR; ++r) {
+      for (int r = 0; r < 16; ++r) {
         const float m_new = fmaxf(m_ref[r], tmax[r]);
         const bool need =
             (m_new > m_ref[r]) && (m_ref[r] == -INFINITY || (m_new - m_ref[r]) * sc > RESCALE_LOG2);
@@ -302,15 +318,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           any = true;
         }
       }
-      float pv[NR];
+      float pv[16];
 #pragma unroll
-      for (int r = 0; r < NR; ++r) {
+      for (int r = 0; r < 16; ++r) {
         const float mb = (m_ref[r] == -INFINITY) ? 0.f : m_ref[r] * sc;
         pv[r] = ex2_approx(fmaf(__uint_as_float(sv[r]), sc, -mb));
         l_part[r] += pv[r];
       }
 
-      // O^T holds items < n: rescale its columns once the last P.V landed
+      // O^T holds items < n: rescale this row half's columns once the last
+      // P.V landed
       if (any && n > 0) {
         const int m = n - 1;
         ok = wait_bounded(&ctl->pv_done[m & 1], static_cast<uint32_t>((m >> 1) & 1), abort_flag,
@@ -318,11 +335,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         ok = __all_sync(0xffffffffu, ok);
         if (!ok) break;
         tc_fence_after();
-        uint32_t o[NR];
-        tmem_ld16(tbase + lane_off + COL_O, o);
+        uint32_t o[16];
+        const uint32_t t_o = tbase + lane_off + C::COL_O + static_cast<uint32_t>(16 * rh);
+        tmem_ld16(t_o, o);
 #pragma unroll
-        for (int r = 0; r < NR; ++r) o[r] = __float_as_uint(__uint_as_float(o[r]) * alpha[r]);
-        tmem_st16(tbase + lane_off + COL_O, o);
+        for (int r = 0; r < 16; ++r) o[r] = __float_as_uint(__uint_as_float(o[r]) * alpha[r]);
+        tmem_st16(t_o, o);
         tmem_st_wait();
       }
       // the P^T buffer is free once the P.V of item n - 2 completed
@@ -335,9 +353,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       }
       uint8_t* pb = pt + buf * OPB + kh * OPB_HALF + ((kin & 7) << 1);
 #pragma unroll
-      for (int r = 0; r < NR; ++r) {
+      for (int r = 0; r < 16; ++r) {
+        const int row = 16 * rh + r;
         const __nv_bfloat16 v = __float2bfloat16_rn(pv[r]);
-        *reinterpret_cast<__nv_bfloat16*>(pb + r * 128 + (((kin >> 3) ^ (r & 7)) << 4)) = v;
+        *reinterpret_cast<__nv_bfloat16*>(pb + row * 128 + (((kin >> 3) ^ (row & 7)) << 4)) = v;
       }
       fence_proxy_async_smem();
       tc_fence_before();
@@ -351,17 +370,17 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       ok = __all_sync(0xffffffffu, ok);
     }
     if (ok) {
-      uint32_t o[NR];
+      uint32_t o[16];
       if (N > 0) {
         tc_fence_after();
-        tmem_ld16(tbase + lane_off + COL_O, o);
+        tmem_ld16(tbase + lane_off + C::COL_O + static_cast<uint32_t>(16 * rh), o);
       } else {
 #pragma unroll
-        for (int r = 0; r < NR; ++r) o[r] = 0u;
+        for (int r = 0; r < 16; ++r) o[r] = 0u;
       }
       float mine = 0.f, mref_mine = -INFINITY;
 #pragma unroll
-      for (int r = 0; r < NR; ++r) {
+      for (int r = 0; r < 16; ++r) {
         float v = l_part[r];
 #pragma unroll
         for (int off = 16; off >= 1; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
@@ -370,7 +389,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           mref_mine = m_ref[r];
         }
       }
-      if (lane < NR) ctl->lsum[warp][lane] = mine;
+      if (lane < 16) ctl->lsum[warp][lane] = mine;
       __syncwarp();
       if (lane == 0) mbar_arrive(&ctl->epi_bar);
       ok = wait_bounded(&ctl->epi_bar, 0u, abort_flag, p.status, p.timeout_ns, ST_SOFTMAX);
@@ -380,16 +399,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         float* pm = p.part + static_cast<size_t>(p.n_cta) * NR * HD + static_cast<size_t>(cta) * NR;
         float* pl = pm + static_cast<size_t>(p.n_cta) * NR;
 #pragma unroll
-        for (int r = 0; r < NR; ++r)
-          if (r < n_rows) po[r * HD + tau] = __uint_as_float(o[r]);
-        if (warp == 0 && lane < n_rows) {
-          pm[lane] = (mref_mine == -INFINITY) ? -INFINITY : mref_mine * sc;
-          pl[lane] = ctl->lsum[0][lane] + ctl->lsum[1][lane] + ctl->lsum[2][lane] +
-                     ctl->lsum[3][lane];
+        for (int r = 0; r < 16; ++r)
+          if (16 * rh + r < n_rows) po[(16 * rh + r) * HD + tau] = __uint_as_float(o[r]);
+        if (quad == 0 && lane < 16 && 16 * rh + lane < n_rows) {
+          pm[16 * rh + lane] = (mref_mine == -INFINITY) ? -INFINITY : mref_mine * sc;
+          pl[16 * rh + lane] = ctl->lsum[warp][lane] + ctl->lsum[warp + 1][lane] +
+                               ctl->lsum[warp + 2][lane] + ctl->lsum[warp + 3][lane];
         }
       }
     }
-  } else if (warp == WARP_LOAD) {
+  } else if (warp == C::WARP_LOAD) {
     // =========================================================== TMA producer
     if (lane == 0) {
       int last_li[NTILE];
@@ -423,7 +442,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                      p.status, p.timeout_ns, ST_DRAIN);
     }
     __syncwarp();
-  } else if (warp == WARP_MMA) {
+  } else if (warp == C::WARP_MMA) {
     // =========================================================== MMA issuer
     if (lane == 0) {
       const uint32_t id_s = idesc_bf16_f32_major(BN, NR, false, false);
@@ -458,7 +477,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           for (int kk = 0; kk < HD / 16; ++kk) {
             const uint64_t ka = static_cast<uint64_t>(((kk >> 2) * HALF_BYTES + (kk & 3) * 32) >> 4);
             const uint64_t kb = static_cast<uint64_t>(((kk >> 2) * OPB_HALF + (kk & 3) * 32) >> 4);
-            mma_ss(tbase + static_cast<uint32_t>((n & 1) * 16), dk + ka, dq + kb, id_s,
+            mma_ss(tbase + static_cast<uint32_t>((n & 1) * NR), dk + ka, dq + kb, id_s,
                    kk > 0 ? 1u : 0u);
           }
           mma_commit(&ctl->s_full[n & 1]);
@@ -478,7 +497,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 #pragma unroll
           for (int kk = 0; kk < BN / 16; ++kk) {
             const uint64_t kb = static_cast<uint64_t>(((kk >> 2) * OPB_HALF + (kk & 3) * 32) >> 4);
-            mma_ss(tbase + COL_O, dv + static_cast<uint64_t>((kk * 2048) >> 4), dp + kb, id_o,
+            mma_ss(tbase + C::COL_O, dv + static_cast<uint64_t>((kk * 2048) >> 4), dp + kb, id_o,
                    (m > 0 || kk > 0) ? 1u : 0u);
           }
           mma_commit(&ctl->pv_done[m & 1]);
@@ -495,40 +514,87 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 
   tc_fence_before();
   __syncthreads();
-  if (warp == WARP_MMA) {
+  if (warp == C::WARP_MMA) {
     tc_fence_after();
-    tmem_dealloc(tbase, TMEM_COLS);
+    tmem_dealloc(tbase, C::TMEM_COLS);
   }
 }
 
 // Merge the slices of each (token, head) row: with slice maxima m_k (log2
 // units), sums l_k and unnormalised outputs O_k, out = sum_k 2^(m_k - M) O_k /
 // sum_k 2^(m_k - M) l_k with M = max m_k; LSE (natural log) = (M + log2 of the
-// denominator) ln 2.  One CTA per row, one thread per dim.
+// denominator) ln 2.  One CTA per row, one thread per dim: the slices'
+// (m, l) are fetched in parallel into shared memory, then each thread streams
+// its dim of the O_k with independent loads.
+constexpr int MERGE_MAX_SPLITS = DECODE_MAX_CTAS;
+
 __global__ void __launch_bounds__(HD)
     dca_decode_combine_kernel(const float* __restrict__ part, __nv_bfloat16* __restrict__ out,
-                              float* __restrict__ lse, int Hq, int G, int n_rg, int n_splits,
-                              int n_cta) {
+                              float* __restrict__ lse, int Hq, int G, int nr, int n_rg,
+                              int n_splits, int n_cta) {
+  __shared__ float wk[MERGE_MAX_SPLITS];
+  __shared__ float lk[MERGE_MAX_SPLITS];
+  __shared__ float red[HD / 32];
   const int row = static_cast<int>(blockIdx.x);  // t * Hq + h
   const int t = row / Hq, h = row % Hq;
   const int g = h / G;
   const int rho_g = t * G + (h % G);
-  const int rg = rho_g / NR, rho = rho_g % NR;
+  const int rg = rho_g / nr, rho = rho_g % nr;
   const int c0 = (g * n_rg + rg) * n_splits;
-  const float* pm = part + static_cast<size_t>(n_cta) * NR * HD;
-  const float* pl = pm + static_cast<size_t>(n_cta) * NR;
-  float M = -INFINITY;
-  for (int k = 0; k < n_splits; ++k) M = fmaxf(M, pm[(c0 + k) * NR + rho]);
-  float L = 0.f, acc = 0.f;
-  for (int k = 0; k < n_splits; ++k) {
-    const float mk = pm[(c0 + k) * NR + rho];
-    if (mk == -INFINITY) continue;
-    const float wk = exp2f(mk - M);
-    L = fmaf(wk, pl[(c0 + k) * NR + rho], L);
-    acc = fmaf(wk, part[(static_cast<size_t>(c0 + k) * NR + rho) * HD + threadIdx.x], acc);
+  const float* pm = part + static_cast<size_t>(n_cta) * nr * HD;
+  const float* pl = pm + static_cast<size_t>(n_cta) * nr;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+
+  float mx = -INFINITY;
+  for (int k = tid; k < n_splits; k += HD) {
+    const float m = pm[(c0 + k) * nr + rho];
+    wk[k] = m;
+    lk[k] = pl[(c0 + k) * nr + rho];
+    mx = fmaxf(mx, m);
   }
-  out[static_cast<size_t>(row) * HD + threadIdx.x] = __float2bfloat16_rn(acc / L);
-  if (lse != nullptr && threadIdx.x == 0) lse[row] = (M + log2f(L)) * 0.6931471805599453f;
+#pragma unroll
+  for (int off = 16; off >= 1; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+  if (lane == 0) red[warp] = mx;
+  __syncthreads();
+  const float M = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
+  float lsum = 0.f;
+  for (int k = tid; k < n_splits; k += HD) {
+    const float w = (wk[k] == -INFINITY) ? 0.f : exp2f(wk[k] - M);
+    wk[k] = w;
+    lsum = fmaf(w, lk[k], lsum);
+  }
+#pragma unroll
+  for (int off = 16; off >= 1; off >>= 1) lsum += __shfl_xor_sync(0xffffffffu, lsum, off);
+  __syncthreads();  // wk complete; red reused below
+  if (lane == 0) red[warp] = lsum;
+  __syncthreads();
+  const float L = red[0] + red[1] + red[2] + red[3];
+
+  const float* po = part + (static_cast<size_t>(c0) * nr + rho) * HD + tid;
+  const size_t stride = static_cast<size_t>(nr) * HD;
+  float acc[4] = {0.f, 0.f, 0.f, 0.f};
+  int k = 0;
+  for (; k + 4 <= n_splits; k += 4) {
+#pragma unroll
+    for (int u = 0; u < 4; ++u) acc[u] = fmaf(wk[k + u], po[(k + u) * stride], acc[u]);
+  }
+  for (; k < n_splits; ++k) acc[0] = fmaf(wk[k], po[k * stride], acc[0]);
+  const float o = (acc[0] + acc[1]) + (acc[2] + acc[3]);
+  out[static_cast<size_t>(row) * HD + tid] = __float2bfloat16_rn(o / L);
+  if (lse != nullptr && tid == 0) lse[row] = (M + log2f(L)) * 0.6931471805599453f;
+}
+
+template <int NR>
+cudaError_t launch(const CUtensorMap& tm_k, const CUtensorMap& tm_v, const Params& p,
+                   cudaStream_t st) {
+  constexpr size_t smem = smem_bytes<NR>();
+  cudaError_t e = cudaFuncSetAttribute(dca_decode_kernel<NR>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  dca_decode_kernel<NR><<<static_cast<unsigned>(p.n_cta), Cfg<NR>::THREADS, smem, st>>>(tm_k,
+                                                                                         tm_v, p);
+  return cudaGetLastError();
 }
 
 }  // namespace dec
@@ -560,6 +626,7 @@ cudaError_t launch_decode_sm100(const AttnArgs& a, float* part, cudaStream_t st)
   const int64_t i_last = a.q_start + a.Lq - 1;
   p.plan = make_plan(a.q_start, i_last, a.s, a.w, BN, a.reading);
   p.fullr = make_full_ranges(a.q_start, i_last, a.s, a.w, BN, a.reading);
+  const int nr = decode_group_rows(a.Lq, p.G);
   p.n_rg = decode_row_groups(a.Lq, p.G);
   const int max_splits = decode_max_splits(a.Hkv, p.n_rg);
   p.n_splits = p.plan.n_items < max_splits ? p.plan.n_items : max_splits;
@@ -567,15 +634,11 @@ cudaError_t launch_decode_sm100(const AttnArgs& a, float* part, cudaStream_t st)
   const int64_t n_cta = static_cast<int64_t>(a.Hkv) * p.n_rg * p.n_splits;
   if (n_cta > 0x7fffffffLL || a.Lq * a.Hq > 0x7fffffffLL) return cudaErrorInvalidValue;
   p.n_cta = static_cast<int>(n_cta);
-  cudaError_t e = cudaFuncSetAttribute(dca_decode_kernel,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(SMEM_BYTES));
-  if (e != cudaSuccess) return e;
-  dca_decode_kernel<<<static_cast<unsigned>(n_cta), NUM_THREADS, SMEM_BYTES, st>>>(tm_k, tm_v, p);
-  e = cudaGetLastError();
+  cudaError_t e = nr == 16 ? launch<16>(tm_k, tm_v, p, st) : launch<32>(tm_k, tm_v, p, st);
   if (e != cudaSuccess) return e;
   dca_decode_combine_kernel<<<static_cast<unsigned>(a.Lq * a.Hq), HD, 0, st>>>(
-      part, static_cast<__nv_bfloat16*>(a.out), a.lse, a.Hq, p.G, p.n_rg, p.n_splits, p.n_cta);
+      part, static_cast<__nv_bfloat16*>(a.out), a.lse, a.Hq, p.G, nr, p.n_rg, p.n_splits,
+      p.n_cta);
   return cudaGetLastError();
 }
 

@@ -25,19 +25,22 @@ struct AttnArgs {
 };
 
 // Split-KV decode: a few query rows against a long cache.  CTAs per
-// (KV head, row group) and the partial-result scratch they write.
-constexpr int DECODE_ROWS = 16;      // query rows per row group (MMA N)
+// (KV head, row group, slice) and the partial-result scratch they write.
+// A row group is 16 (token, head) rows when the query block has at most 16
+// rows per KV head, otherwise 32 (the MMA N of the decode kernel).
 constexpr int DECODE_MAX_CTAS = 148; // one CTA per SM of a B200
+inline int decode_group_rows(int64_t Lq, int G) { return Lq * G <= 16 ? 16 : 32; }
 inline int decode_row_groups(int64_t Lq, int G) {
-  return static_cast<int>((Lq * G + DECODE_ROWS - 1) / DECODE_ROWS);
+  const int nr = decode_group_rows(Lq, G);
+  return static_cast<int>((Lq * G + nr - 1) / nr);
 }
 inline int decode_max_splits(int Hkv, int n_rg) {
   const int per = DECODE_MAX_CTAS / (Hkv * n_rg);
   return per > 1 ? per : 1;
 }
-// fp32 words of partial results: O [cta][16][128], then m, l [cta][16].
-inline size_t decode_part_floats(int n_cta) {
-  return static_cast<size_t>(n_cta) * DECODE_ROWS * (128 + 2);
+// fp32 words of partial results: O [cta][nr][128], then m, l [cta][nr].
+inline size_t decode_part_floats(int n_cta, int nr) {
+  return static_cast<size_t>(n_cta) * nr * (128 + 2);
 }
 
 cudaError_t launch_rope_table(float2* tab, int64_t T, int64_t n_direct, int64_t c, double base,

@@ -33,11 +33,14 @@ def lib():
 
 
 def test_scratch_size_rule(lib):
-    # (Hkv * row groups * slices) CTAs, each 16 rows x (128 + 2) fp32 words
+    # (Hkv * row groups * slices) CTAs, each nr rows x (128 + 2) fp32 words;
+    # a row group holds 16 (token, head) rows, or 32 when a KV head has more
     def expect(Lq, Hq, Hkv):
-        n_rg = -(-Lq * (Hq // Hkv) // 16)
+        rows = Lq * (Hq // Hkv)
+        nr = 16 if rows <= 16 else 32
+        n_rg = -(-rows // nr)
         n_cta = Hkv * n_rg * max(1, 148 // (Hkv * n_rg))
-        return -(-n_cta * 16 * 130 * 4 // 256) * 256
+        return -(-n_cta * nr * 130 * 4 // 256) * 256
     for Lq, Hq, Hkv in [(1, 28, 4), (4, 28, 4), (256, 28, 4), (1, 8, 8), (3, 40, 8), (1, 1, 1)]:
         assert lib.dca_decode_scratch_size(Lq, Hq, Hkv) == expect(Lq, Hq, Hkv)
     assert lib.dca_decode_scratch_size(0, 28, 4) == 0
@@ -81,7 +84,9 @@ CASES = [
     dec("far_r", 5000, 1, 28, 4, 1024, 128, 2048),                 # r_i >= w: SUCC at c - 1
     dec("near_r", 4147, 1, 28, 4, 1024, 128, 2048, yarn=4.0),      # r_i = 50 < w: SUCC at s + r_i
     dec("straddle", 4098, 3, 28, 4, 1024, 128, 2048),              # rows 4095..4097 cross a chunk
-    dec("rowgroups", 3000, 5, 28, 4, 512, 64, 1024, yarn=2.0),     # 35 rows: 3 row groups
+    dec("rowgroups", 3000, 5, 28, 4, 512, 64, 1024, yarn=2.0),     # 35 rows: 2 groups of 32
+    dec("group32", 4147, 4, 28, 4, 1024, 128, 2048),              # 28 rows: one group of 32
+    dec("group16_full", 2000, 2, 16, 2, 512, 64, 1024),           # exactly 16 rows
     dec("single_chunk", 700, 2, 8, 2, 1024, 64, 2048),
     dec("tiny_chunks", 300, 2, 2, 1, 3, 2, 5),
     dec("w0", 2500, 1, 4, 2, 256, 0, 256),
