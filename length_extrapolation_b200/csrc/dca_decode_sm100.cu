@@ -51,7 +51,10 @@ template <int NR>
 struct Cfg {
   static_assert(NR == 16 || NR == 32, "row group of 16 or 32");
   static constexpr int SW = NR / 4;                     // softmax warps
-  static constexpr int NTILE = NR == 16 ? 6 : 5;        // K'/V tile ring
+  // K'/V tile ring: 3 items in flight for 16 rows, 2.5 for 32 (shared-memory
+  // budget; a 6-slot ring with one P^T buffer measured no faster for 32)
+  static constexpr int NTILE = NR == 16 ? 6 : 5;
+  static constexpr int NPB = 2;                         // P^T buffers
   static constexpr int OPB = NR * HD * 2;               // an NR-row operand (Q variant or P^T)
   static constexpr int OPB_HALF = NR * 128;             // its 64-column block
   static constexpr int THREADS = 32 * (SW + 2);
@@ -83,7 +86,8 @@ struct SmemCtl {
 
 template <int NR>
 constexpr size_t smem_bytes() {
-  return 1024 + Cfg<NR>::NTILE * TILE_BYTES + 5 * Cfg<NR>::OPB + sizeof(SmemCtl<NR>);
+  return 1024 + Cfg<NR>::NTILE * TILE_BYTES + (3 + Cfg<NR>::NPB) * Cfg<NR>::OPB +
+         sizeof(SmemCtl<NR>);
 }
 static_assert(smem_bytes<16>() <= 232448 && smem_bytes<32>() <= 232448, "shared memory budget");
 
@@ -124,13 +128,14 @@ __global__ void __launch_bounds__(Cfg<NR>::THREADS, 1)
                       const __grid_constant__ CUtensorMap tm_v, const Params p) {
   using C = Cfg<NR>;
   constexpr int SW = C::SW, NTILE = C::NTILE, OPB = C::OPB, OPB_HALF = C::OPB_HALF;
+  constexpr int NPB = C::NPB;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   uint8_t* tiles = smem;
   uint8_t* qv = tiles + NTILE * TILE_BYTES;  // Q variants, indexed by class
-  uint8_t* pt = qv + 3 * OPB;                // P^T, two buffers
-  SmemCtl<NR>* ctl = reinterpret_cast<SmemCtl<NR>*>(pt + 2 * OPB);
+  uint8_t* pt = qv + 3 * OPB;                // P^T, NPB buffers
+  SmemCtl<NR>* ctl = reinterpret_cast<SmemCtl<NR>*>(pt + NPB * OPB);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -283,39 +288,54 @@ __global__ void __launch_bounds__(Cfg<NR>::THREADS, 1)
       ok = wait_poll(&ctl->max_bar[buf], ph, abort_flag, p.status, p.timeout_ns, ST_SOFTMAX);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
-      float tmax[16];
-#pragma unroll
-      for (int r4 = 0; r4 < 4; ++r4) {
-        float4 a = reinterpret_cast<const float4*>(ctl->wmax[buf][4 * rh])[r4];
-#pragma unroll
-        for (int wq = 1; wq < 4; ++wq) {
-          const float4 o = reinterpret_cast<const float4*>(ctl->wmax[buf][4 * rh + wq])[r4];
-          a.x = fmaxf(a.x, o.x);
-          a.y = fmaxf(a.y, o.y);
-          a.z = fmaxf(a.z, o.z);
-          a.w = fmaxf(a.w, o.w);
-        }
-        tmax[4 * r4 + 0] = a.x;
-        tmax[4 * r4 + 1] = a.y;
-        tmax[4 * r4 + 2] = a.z;
-        tmax[4 * r4 + 3] = a.w;
-      }
-
       // reference update (identical in the four warps of a row half: same
-      // maxima, same history)
-      float alpha[16];
-      bool any = false;
+      // maxima, same history); O^T holds items < n, so when a reference
+      // moves its columns are rescaled once the last P.V landed
+      {
+        float alpha[16];
+        bool any = false;
 #pragma unroll
-      for (int r = 0; r < 16; ++r) {
-        const float m_new = fmaxf(m_ref[r], tmax[r]);
-        const bool need =
-            (m_new > m_ref[r]) && (m_ref[r] == -INFINITY || (m_new - m_ref[r]) * sc > RESCALE_LOG2);
-        alpha[r] = 1.f;
-        if (need) {
-          alpha[r] = (m_ref[r] == -INFINITY) ? 0.f : ex2_approx((m_ref[r] - m_new) * sc);
-          m_ref[r] = m_new;
-          l_part[r] *= alpha[r];
-          any = true;
+        for (int r4 = 0; r4 < 4; ++r4) {
+          // tile maxima of rows 4 r4 .. 4 r4 + 3 over the row half's four warps
+          float4 t = reinterpret_cast<const float4*>(ctl->wmax[buf][4 * rh])[r4];
+#pragma unroll
+          for (int wq = 1; wq < 4; ++wq) {
+            const float4 o = reinterpret_cast<const float4*>(ctl->wmax[buf][4 * rh + wq])[r4];
+            t.x = fmaxf(t.x, o.x);
+            t.y = fmaxf(t.y, o.y);
+            t.z = fmaxf(t.z, o.z);
+            t.w = fmaxf(t.w, o.w);
+          }
+          const float tm[4] = {t.x, t.y, t.z, t.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int r = 4 * r4 + e;
+            const float m_new = fmaxf(m_ref[r], tm[e]);
+            const bool need = (m_new > m_ref[r]) &&
+                              (m_ref[r] == -INFINITY || (m_new - m_ref[r]) * sc > RESCALE_LOG2);
+            alpha[r] = 1.f;
+            if (need) {
+              alpha[r] = (m_ref[r] == -INFINITY) ? 0.f : ex2_approx((m_ref[r] - m_new) * sc);
+              m_ref[r] = m_new;
+              l_part[r] *= alpha[r];
+              any = true;
+            }
+          }
+        }
+        if (any && n > 0) {
+          const int m = n - 1;
+          ok = wait_bounded(&ctl->pv_done[m & 1], static_cast<uint32_t>((m >> 1) & 1),
+                            abort_flag, p.status, p.timeout_ns, ST_SOFTMAX);
+          ok = __all_sync(0xffffffffu, ok);
+          if (!ok) break;
+          tc_fence_after();
+          uint32_t o[16];
+          const uint32_t t_o = tbase + lane_off + C::COL_O + static_cast<uint32_t>(16 * rh);
+          tmem_ld16(t_o, o);
+#pragma unroll
+          for (int r = 0; r < 16; ++r) o[r] = __float_as_uint(__uint_as_float(o[r]) * alpha[r]);
+          tmem_st16(t_o, o);
+          tmem_st_wait();
         }
       }
       float pv[16];
@@ -325,33 +345,15 @@ __global__ void __launch_bounds__(Cfg<NR>::THREADS, 1)
         pv[r] = ex2_approx(fmaf(__uint_as_float(sv[r]), sc, -mb));
         l_part[r] += pv[r];
       }
-
-      // O^T holds items < n: rescale this row half's columns once the last
-      // P.V landed
-      if (any && n > 0) {
-        const int m = n - 1;
-        ok = wait_bounded(&ctl->pv_done[m & 1], static_cast<uint32_t>((m >> 1) & 1), abort_flag,
-                          p.status, p.timeout_ns, ST_SOFTMAX);
-        ok = __all_sync(0xffffffffu, ok);
-        if (!ok) break;
-        tc_fence_after();
-        uint32_t o[16];
-        const uint32_t t_o = tbase + lane_off + C::COL_O + static_cast<uint32_t>(16 * rh);
-        tmem_ld16(t_o, o);
-#pragma unroll
-        for (int r = 0; r < 16; ++r) o[r] = __float_as_uint(__uint_as_float(o[r]) * alpha[r]);
-        tmem_st16(t_o, o);
-        tmem_st_wait();
-      }
-      // the P^T buffer is free once the P.V of item n - 2 completed
-      if (n >= 2) {
-        const int m = n - 2;
+      // the P^T buffer is free once the P.V of item n - NPB completed
+      if (n >= NPB) {
+        const int m = n - NPB;
         ok = wait_bounded(&ctl->pv_done[m & 1], static_cast<uint32_t>((m >> 1) & 1), abort_flag,
                           p.status, p.timeout_ns, ST_SOFTMAX);
         ok = __all_sync(0xffffffffu, ok);
         if (!ok) break;
       }
-      uint8_t* pb = pt + buf * OPB + kh * OPB_HALF + ((kin & 7) << 1);
+      uint8_t* pb = pt + (n % NPB) * OPB + kh * OPB_HALF + ((kin & 7) << 1);
 #pragma unroll
       for (int r = 0; r < 16; ++r) {
         const int row = 16 * rh + r;
@@ -493,7 +495,7 @@ __global__ void __launch_bounds__(Cfg<NR>::THREADS, 1)
           if (!ok) break;
           tc_fence_after();
           const uint64_t dv = dv0 + static_cast<uint64_t>(((lv % NTILE) * TILE_BYTES) >> 4);
-          const uint64_t dp = dp0 + static_cast<uint64_t>(((m & 1) * OPB) >> 4);
+          const uint64_t dp = dp0 + static_cast<uint64_t>(((m % NPB) * OPB) >> 4);
 #pragma unroll
           for (int kk = 0; kk < BN / 16; ++kk) {
             const uint64_t kb = static_cast<uint64_t>(((kk >> 2) * OPB_HALF + (kk & 3) * 32) >> 4);
