@@ -37,6 +37,11 @@ MUTATIONS = {
     "noncausal_diag": 8,
     "gqa_interleaved": 9,
     "theta_d": 10,
+    # sparse variant
+    "sp_no_dedup": 11,
+    "sp_vert_acausal": 12,
+    "sp_offset_off1": 13,
+    "sp_no_self": 14,
 }
 
 
@@ -65,6 +70,10 @@ def _load():
             vp, vp, vp, i32, i64, i64, i64, i32, i32, i32, i64, i64, i64, dbl, dbl,
             i32, i32, vp, i64, vp, i32, vp, vp, i32]
         lib.dca_oracle_attention_mut.restype = i32
+        lib.dca_oracle_sparse_attention.argtypes = [
+            vp, vp, vp, i32, i64, i64, i64, i32, i32, i32, i64, i64, i64, dbl, dbl,
+            i32, i32, vp, vp, vp, vp, vp, i64, vp, i32, vp, vp, i32]
+        lib.dca_oracle_sparse_attention.restype = i32
         lib.dca_oracle_position.argtypes = [i64, i64, i64, i64, i64, i32, i32,
                                             ctypes.POINTER(i64), ctypes.POINTER(i64)]
         lib.dca_oracle_position.restype = i32
@@ -142,6 +151,60 @@ def attention(q, k, v, *, chunk_size, local_window, pretrain_window,
         Hkv, d, int(chunk_size), int(local_window), int(pretrain_window),
         float(rope_base), float(yarn_scale), int(reading), int(mutation),
         rows.ctypes.data, len(rows), heads.ctypes.data, len(heads), out.ctypes.data,
+        lse.ctypes.data if lse is not None else None, int(n_threads))
+    if rc != 0:
+        raise ValueError(f"oracle returned {rc}")
+    return (out, lse) if return_lse else out
+
+
+def csr(lists, Lk):
+    """Per-head index lists -> (ptr int64 [H+1], idx int64), each list sorted,
+    without repeats, inside [0, Lk)."""
+    ptr = [0]
+    flat = []
+    for a in lists:
+        a = np.asarray(a, dtype=np.int64).ravel()
+        if a.size and (np.any(np.diff(a) <= 0) or a[0] < 0 or a[-1] >= Lk):
+            raise ValueError("index lists must be sorted, unique and inside [0, Lk)")
+        flat.append(a)
+        ptr.append(ptr[-1] + a.size)
+    idx = np.concatenate(flat) if flat else np.zeros(0, np.int64)
+    return np.asarray(ptr, dtype=np.int64), np.ascontiguousarray(idx, dtype=np.int64)
+
+
+def sparse_attention(q, k, v, *, vertical, slash, chunk_size, local_window, pretrain_window,
+                     rope_base=1e7, yarn_scale=1.0, q_start=0, rows=None, heads=None,
+                     reading=0, mutation=0, n_threads=None, return_lse=False):
+    """Vertical-slash sparse DCA attention in fp64 (definition in dca_oracle.c).
+
+    vertical[h], slash[h]: sorted key indices / diagonal offsets of query head
+    h.  Row i of head h attends keys {j <= i in vertical[h]} U {i - o : o in
+    slash[h], o <= i} U {i}.  Other arguments as ``attention``.
+    """
+    qa, dt = _as_input(q)
+    ka, dtk = _as_input(k)
+    va, dtv = _as_input(v)
+    if not (dt == dtk == dtv):
+        raise TypeError("q, k, v must share a dtype")
+    Lq, Hq, d = qa.shape
+    Lk, Hkv, dk = ka.shape
+    if va.shape != ka.shape or dk != d or len(vertical) != Hq or len(slash) != Hq:
+        raise ValueError("shape mismatch")
+    v_ptr, v_idx = csr(vertical, Lk)
+    s_ptr, s_off = csr(slash, Lk)
+    rows = np.arange(Lq, dtype=np.int64) if rows is None else np.ascontiguousarray(rows, dtype=np.int64)
+    heads = np.arange(Hq, dtype=np.int32) if heads is None else np.ascontiguousarray(heads, dtype=np.int32)
+    out = np.zeros((len(rows), len(heads), d), dtype=np.float64)
+    lse = np.zeros((len(rows), len(heads)), dtype=np.float64) if return_lse else None
+    if n_threads is None:
+        n_threads = os.cpu_count() or 1
+    rc = _load().dca_oracle_sparse_attention(
+        qa.ctypes.data, ka.ctypes.data, va.ctypes.data, dt, int(q_start), Lq, Lk, Hq, Hkv, d,
+        int(chunk_size), int(local_window), int(pretrain_window), float(rope_base),
+        float(yarn_scale), int(reading), int(mutation), v_ptr.ctypes.data,
+        v_idx.ctypes.data if v_idx.size else None, s_ptr.ctypes.data,
+        s_off.ctypes.data if s_off.size else None, rows.ctypes.data, len(rows),
+        heads.ctypes.data, len(heads), out.ctypes.data,
         lse.ctypes.data if lse is not None else None, int(n_threads))
     if rc != 0:
         raise ValueError(f"oracle returned {rc}")

@@ -44,6 +44,17 @@
  *      q_start attends to a KV cache of Lk rows; the formula above is applied
  *      to absolute indices, so block results equal the one-shot rows. [MIZ Chunked Prefill]
  *
+ * Sparse variant (dca_oracle_sparse_attention): the vertical-slash sparse
+ * attention that the Qwen2.5-1M framework runs on top of DCA ("Qwen2.5-1M
+ * 不重训外推 1M", sections "跟 NSA / 其他稀疏注意力的区别" and "稀疏注意力 +
+ * 核优化": a few key columns draw most of the attention, per-head sparse
+ * configurations are searched offline, and at inference only the selected
+ * keys are attended).  For query head h with vertical key set V_h and slash
+ * offset set S_h, row i attends exactly the member keys
+ *      M_h(i) = { j <= i : j in V_h }  U  { i - o : o in S_h, o <= i }  U  { i }
+ * (each key once; the row's own key always, so no row is empty), with the
+ * DCA logits above and a softmax over M_h(i).
+ *
  * The oracle also carries a `mutation` argument used only by tests that
  * check that the pins catch plausible mistakes (each value plants one known
  * mistake).  mutation = 0 is the oracle proper.
@@ -70,6 +81,11 @@
 #define MUT_NONCAUSAL_DIAG 8  /* diagonal j = i excluded                        */
 #define MUT_GQA_INTERLEAVED 9 /* head h reads KV head h % Hkv                   */
 #define MUT_THETA_D 10        /* theta_k = base^(-k/d)                          */
+/* sparse variant */
+#define MUT_SP_NO_DEDUP 11    /* a key that is vertical and on a slash counted twice */
+#define MUT_SP_VERT_ACAUSAL 12/* vertical keys j > i included                   */
+#define MUT_SP_OFFSET_OFF1 13 /* slash offset o selects j = i - o - 1            */
+#define MUT_SP_NO_SELF 14     /* the row's own key not added                      */
 
 static double to_f64(const void* p, int dtype, int64_t idx) {
   if (dtype == ORACLE_DT_BF16) {
@@ -151,6 +167,9 @@ typedef struct {
   int n_heads;
   double* out;
   double* lse;
+  /* sparse pattern (NULL v_ptr: dense) -- CSR per query head, sorted lists */
+  const int64_t *v_ptr, *v_idx, *s_ptr, *s_off;
+  int64_t krot_rows;  /* rows of krot (keys 0 .. krot_rows - 1 are rotated) */
   /* shared state */
   const double* theta;
   const double* krot; /* rotated keys of the current KV head: [jmax+1][d] */
@@ -230,12 +249,95 @@ static void one_row(job_t* J, int64_t ridx, int hidx, double* scratch) {
   if (J->lse) J->lse[ridx * J->n_heads + hidx] = mx + log(sum);
 }
 
+static int cmp_i64(const void* a, const void* b) {
+  int64_t x = *(const int64_t*)a, y = *(const int64_t*)b;
+  return (x > y) - (x < y);
+}
+
+/* One (row, head) output of the sparse variant: the member set written out,
+ * then the same logits and softmax as one_row over those keys only. */
+static void one_row_sparse(job_t* J, int64_t ridx, int hidx, double* scratch, int64_t* cand) {
+  const int d = J->d;
+  const int64_t t = J->rows[ridx];
+  const int64_t i = J->q_start + t;
+  const int h = J->heads[hidx];
+  /* member keys */
+  int64_t n = 0;
+  for (int64_t e = J->v_ptr[h]; e < J->v_ptr[h + 1]; ++e) {
+    int64_t j = J->v_idx[e];
+    if (j <= i || (J->mutation == MUT_SP_VERT_ACAUSAL && j < J->krot_rows)) cand[n++] = j;
+  }
+  for (int64_t e = J->s_ptr[h]; e < J->s_ptr[h + 1]; ++e) {
+    int64_t o = J->s_off[e];
+    int64_t j = (J->mutation == MUT_SP_OFFSET_OFF1) ? i - o - 1 : i - o;
+    if (o <= i && j >= 0) cand[n++] = j;
+  }
+  if (J->mutation != MUT_SP_NO_SELF) cand[n++] = i;
+  qsort(cand, (size_t)n, sizeof(int64_t), cmp_i64);
+  int64_t m = 0;
+  for (int64_t e = 0; e < n; ++e)
+    if (J->mutation == MUT_SP_NO_DEDUP || m == 0 || cand[e] != cand[m - 1]) cand[m++] = cand[e];
+
+  double* logit = scratch;          /* [m] */
+  double* qraw = scratch + m;       /* [d] */
+  double* qvar = qraw + d;          /* [3][d] */
+  int64_t qpos_cached[3] = {-1, -1, -1};
+  double scale = (1.0 / sqrt((double)d)) * dca_oracle_mscale(J->yarn) * dca_oracle_mscale(J->yarn);
+  for (int e = 0; e < d; ++e)
+    qraw[e] = to_f64(J->q, J->dtype, (t * J->Hq + h) * (int64_t)d + e);
+  double mx = -INFINITY;
+  for (int64_t e = 0; e < m; ++e) {
+    int64_t j = cand[e], pq, pk;
+    int cls = dca_oracle_position(i, j, J->s, J->w, J->c, J->reading, MUT_NONE, &pq, &pk);
+    double* qv = qvar + cls * d;
+    if (qpos_cached[cls] != pq) {
+      rotate(qraw, qv, d, pq, J->theta, MUT_NONE);
+      qpos_cached[cls] = pq;
+    }
+    const double* kr = J->krot + j * (int64_t)d;
+    double dot = 0.0;
+    for (int c2 = 0; c2 < d; ++c2) dot += qv[c2] * kr[c2];
+    logit[e] = scale * dot;
+    if (logit[e] > mx) mx = logit[e];
+  }
+  double* o = J->out + (ridx * J->n_heads + hidx) * (int64_t)d;
+  for (int e = 0; e < d; ++e) o[e] = 0.0;
+  if (m == 0) {
+    if (J->lse) J->lse[ridx * J->n_heads + hidx] = -INFINITY;
+    return;
+  }
+  double sum = 0.0;
+  for (int64_t e = 0; e < m; ++e) {
+    double p = exp(logit[e] - mx);
+    sum += p;
+    for (int c2 = 0; c2 < d; ++c2)
+      o[c2] += p * to_f64(J->v, J->dtype, (cand[e] * J->Hkv + J->kv_head) * (int64_t)d + c2);
+  }
+  for (int e = 0; e < d; ++e) o[e] /= sum;
+  if (J->lse) J->lse[ridx * J->n_heads + hidx] = mx + log(sum);
+}
+
 static void* worker(void* arg) {
   job_t* J = (job_t*)arg;
   int64_t imax = 0;
   for (int64_t r = 0; r < J->n_rows; ++r)
     if (J->q_start + J->rows[r] > imax) imax = J->q_start + J->rows[r];
-  double* scratch = (double*)malloc(sizeof(double) * (size_t)(imax + 1 + 4 * J->d));
+  int64_t most = 0; /* candidate keys of a sparse row (before removing repeats) */
+  if (J->v_ptr)
+    for (int hh = 0; hh < J->Hq; ++hh) {
+      int64_t c2 = (J->v_ptr[hh + 1] - J->v_ptr[hh]) + (J->s_ptr[hh + 1] - J->s_ptr[hh]) + 1;
+      if (c2 > most) most = c2;
+    }
+  int64_t nlog = imax + 1 > most ? imax + 1 : most;
+  double* scratch = (double*)malloc(sizeof(double) * (size_t)(nlog + 4 * J->d));
+  int64_t* cand = NULL;
+  if (J->v_ptr) {
+    cand = (int64_t*)malloc(sizeof(int64_t) * (size_t)(most + 1));
+    if (!cand) {
+      free(scratch);
+      scratch = NULL;
+    }
+  }
   if (!scratch) {
     pthread_mutex_lock(&J->mu);
     J->status = -3;
@@ -247,9 +349,13 @@ static void* worker(void* arg) {
     int64_t w = J->next++;
     pthread_mutex_unlock(&J->mu);
     if (w >= J->n_work) break;
-    one_row(J, J->work[2 * w], (int)J->work[2 * w + 1], scratch);
+    if (J->v_ptr)
+      one_row_sparse(J, J->work[2 * w], (int)J->work[2 * w + 1], scratch, cand);
+    else
+      one_row(J, J->work[2 * w], (int)J->work[2 * w + 1], scratch);
   }
   free(scratch);
+  free(cand);
   return NULL;
 }
 
@@ -281,12 +387,14 @@ static void* rot_worker(void* arg) {
  *   out  [n_rows][n_heads][d] fp64,  lse [n_rows][n_heads] (natural log) or NULL
  * Returns 0 on success, -1 on a bad argument, -3 on allocation failure.
  */
-int dca_oracle_attention_mut(const void* q, const void* k, const void* v, int dtype,
-                             int64_t q_start, int64_t Lq, int64_t Lk, int Hq, int Hkv,
-                             int d, int64_t s, int64_t w, int64_t c, double base,
-                             double yarn, int reading, int mutation,
-                             const int64_t* rows, int64_t n_rows, const int* heads,
-                             int n_heads, double* out, double* lse, int n_threads) {
+static int attention_impl(const void* q, const void* k, const void* v, int dtype,
+                          int64_t q_start, int64_t Lq, int64_t Lk, int Hq, int Hkv,
+                          int d, int64_t s, int64_t w, int64_t c, double base,
+                          double yarn, int reading, int mutation,
+                          const int64_t* v_ptr, const int64_t* v_idx,
+                          const int64_t* s_ptr, const int64_t* s_off,
+                          const int64_t* rows, int64_t n_rows, const int* heads,
+                          int n_heads, double* out, double* lse, int n_threads) {
   if (!q || !k || !v || !out || !rows || !heads) return -1;
   if (dtype < 0 || dtype > 2 || d <= 0 || d % 2 || d > 1024) return -1;
   if (Hq <= 0 || Hkv <= 0 || Hq % Hkv) return -1;
@@ -313,11 +421,15 @@ int dca_oracle_attention_mut(const void* q, const void* k, const void* v, int dt
   J.reading = reading; J.mutation = mutation;
   J.rows = rows; J.n_rows = n_rows; J.heads = heads; J.n_heads = n_heads;
   J.out = out; J.lse = lse; J.theta = theta;
+  J.v_ptr = v_ptr; J.v_idx = v_idx; J.s_ptr = s_ptr; J.s_off = s_off;
   pthread_mutex_init(&J.mu, NULL);
 
   int64_t imax = -1;
   for (int64_t r = 0; r < n_rows; ++r)
     if (q_start + rows[r] > imax) imax = q_start + rows[r];
+  /* keys 0 .. imax are rotated; the acausal-vertical mutation reaches up to Lk - 1 */
+  if (v_ptr && mutation == MUT_SP_VERT_ACAUSAL && imax >= 0) imax = Lk - 1;
+  J.krot_rows = imax + 1;
 
   int64_t* work = (int64_t*)malloc(sizeof(int64_t) * 2 * (size_t)(n_rows * n_heads + 1));
   double* krot = (double*)malloc(sizeof(double) * (size_t)(imax + 1) * d + 8);
@@ -363,6 +475,44 @@ int dca_oracle_attention_mut(const void* q, const void* k, const void* v, int dt
   free(theta);
   pthread_mutex_destroy(&J.mu);
   return status;
+}
+
+int dca_oracle_attention_mut(const void* q, const void* k, const void* v, int dtype,
+                             int64_t q_start, int64_t Lq, int64_t Lk, int Hq, int Hkv,
+                             int d, int64_t s, int64_t w, int64_t c, double base,
+                             double yarn, int reading, int mutation,
+                             const int64_t* rows, int64_t n_rows, const int* heads,
+                             int n_heads, double* out, double* lse, int n_threads) {
+  return attention_impl(q, k, v, dtype, q_start, Lq, Lk, Hq, Hkv, d, s, w, c, base, yarn,
+                        reading, mutation, NULL, NULL, NULL, NULL, rows, n_rows, heads,
+                        n_heads, out, lse, n_threads);
+}
+
+/*
+ * Sparse variant.  v_ptr, s_ptr [Hq + 1] (CSR offsets), v_idx [v_ptr[Hq]]
+ * vertical key indices in [0, Lk) and s_off [s_ptr[Hq]] slash offsets in
+ * [0, Lk), each head's list sorted ascending without repeats.  Other
+ * arguments and outputs as dca_oracle_attention_mut.
+ */
+int dca_oracle_sparse_attention(const void* q, const void* k, const void* v, int dtype,
+                                int64_t q_start, int64_t Lq, int64_t Lk, int Hq, int Hkv,
+                                int d, int64_t s, int64_t w, int64_t c, double base,
+                                double yarn, int reading, int mutation,
+                                const int64_t* v_ptr, const int64_t* v_idx,
+                                const int64_t* s_ptr, const int64_t* s_off,
+                                const int64_t* rows, int64_t n_rows, const int* heads,
+                                int n_heads, double* out, double* lse, int n_threads) {
+  if (!v_ptr || !s_ptr || Hq <= 0) return -1;
+  for (int h = 0; h < Hq; ++h) {
+    if (v_ptr[h + 1] < v_ptr[h] || s_ptr[h + 1] < s_ptr[h]) return -1;
+    for (int64_t e = v_ptr[h]; e < v_ptr[h + 1]; ++e)
+      if (v_idx[e] < 0 || v_idx[e] >= Lk || (e > v_ptr[h] && v_idx[e] <= v_idx[e - 1])) return -1;
+    for (int64_t e = s_ptr[h]; e < s_ptr[h + 1]; ++e)
+      if (s_off[e] < 0 || s_off[e] >= Lk || (e > s_ptr[h] && s_off[e] <= s_off[e - 1])) return -1;
+  }
+  return attention_impl(q, k, v, dtype, q_start, Lq, Lk, Hq, Hkv, d, s, w, c, base, yarn,
+                        reading, mutation, v_ptr, v_idx, s_ptr, s_off, rows, n_rows, heads,
+                        n_heads, out, lse, n_threads);
 }
 
 int dca_oracle_attention(const void* q, const void* k, const void* v, int dtype,
