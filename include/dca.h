@@ -190,6 +190,67 @@ int dca_decode(const void* q_block, const void* v_cache, void* out_block, float*
                size_t ws_bytes, void* scratch, size_t scratch_bytes, void* cuda_stream);
 
 /*
+ * Vertical-slash sparse DCA ("Qwen2.5-1M 不重训外推 1M", sections
+ * "跟 NSA / 其他稀疏注意力的区别" and "稀疏注意力 + 核优化": per query head a few key
+ * columns and diagonals carry the attention; per-head sparse patterns are
+ * chosen offline and only the selected keys are attended).  For query head h
+ * with vertical keys V_h and slash offsets S_h, row i attends exactly
+ *     { j <= i : j in V_h } U { i - o : o in S_h, o <= i } U { i }
+ * (each key once) with the DCA logits, softmax over those keys.
+ *
+ * dca_sparse_config fixes the sparse workspace layout: the key capacity its
+ * bitmaps cover and the most vertical keys / slash offsets of any head.
+ * Each head's slash offsets may form at most DCA_SPARSE_MAX_RUNS runs of
+ * consecutive values.
+ *
+ * dca_sparse_prepare takes the patterns as HOST arrays in CSR form (v_ptr,
+ * s_ptr [Hq + 1] offsets; v_idx, s_off the per-head lists, each sorted
+ * ascending without repeats, inside [0, Lk)) and the DCA sizes of the
+ * workspace (chunk_size, local_window, pretrain_window), copies them into the sparse
+ * workspace, builds membership bitmaps and gathers the vertical keys' rotated
+ * rows (from `workspace`, prepared by dca_prepare for rows [0, Lk)) and value
+ * rows (from v_cache) into it.  The host arrays may be freed on return.  A
+ * chunked prefill calls it again when the cache grows (vertical keys past Lk
+ * are not gathered: pass the lists restricted to keys < Lk).
+ * dca_sparse_attend then runs the sparse kernel for a query block (rows
+ * q_start .., keys [0, Lk)).  bf16 only (DCA_ERR_UNSUPPORTED otherwise).
+ * Argument and pattern errors are DCA_ERR_ARG, before any copy or launch;
+ * a too-small sparse workspace is DCA_ERR_WORKSPACE.
+ */
+#define DCA_SPARSE_MAX_RUNS 1023
+typedef struct {
+  int64_t kv_capacity;  /* keys the bitmaps cover (>= every Lk used) */
+  int64_t max_vertical; /* most vertical keys of a head */
+  int64_t max_slash;    /* most slash offsets of a head */
+} dca_sparse_config;
+size_t dca_sparse_workspace_size(const dca_sparse_config* cfg, int Hq);
+int dca_sparse_prepare(const dca_sparse_config* cfg, const int64_t* v_ptr, const int32_t* v_idx,
+                       const int64_t* s_ptr, const int32_t* s_off, int64_t Lk, int Hq, int Hkv,
+                       int d, int64_t chunk_size, int64_t local_window, int64_t pretrain_window,
+                       int dtype, const void* v_cache, const void* workspace, size_t ws_bytes,
+                       void* sparse_ws, size_t sparse_bytes, void* cuda_stream);
+int dca_sparse_attend(const dca_sparse_config* cfg, const void* q_block, const void* v_cache,
+                      void* out_block, int64_t q_start, int64_t Lq, int64_t Lk, int Hq, int Hkv,
+                      int d, int64_t chunk_size, int64_t local_window, int64_t pretrain_window,
+                      double yarn_scale, int dtype, const dca_options* opts, void* workspace,
+                      size_t ws_bytes, const void* sparse_ws, size_t sparse_bytes,
+                      void* cuda_stream);
+
+/*
+ * Host-side introspection of the sparse kernel's work list (no GPU needed):
+ * for the query tile whose rows are [i0, i0 + 128) (i0 a multiple of 128) with
+ * real rows up to i_last, and one head's sorted vertical keys / slash offsets
+ * (host arrays), writes up to max_items triples (src, tile, class): src 0 = a
+ * 128-key tile of the head's gathered vertical keys (list positions
+ * 128*tile ..), src 1 = cache k-tile `tile` crossed by a slash diagonal or by
+ * the diagonal j = i; class as in dca_plan_items.  Returns the number of
+ * items (which may exceed max_items) or DCA_ERR_ARG.
+ */
+int dca_sparse_plan_items(const int32_t* v_idx, int64_t n_v, const int32_t* s_off, int64_t n_s,
+                          int64_t i0, int64_t i_last, int64_t chunk_size, int64_t local_window,
+                          int window_reading, int32_t* items, int max_items);
+
+/*
  * Device-side status: synchronises `cuda_stream`, reads and clears the status
  * word that kernels set when a bounded wait gave up.  Returns DCA_OK,
  * DCA_ERR_TIMEOUT or DCA_ERR_CUDA.

@@ -6,6 +6,8 @@ does not load the library; the first call does, and fails loudly if it was not
 built.
 """
 from .api import (  # noqa: F401
+    SparsePattern,
+    SparseWorkspace,
     Workspace,
     attend,
     decode,
@@ -17,11 +19,15 @@ from .api import (  # noqa: F401
     prefill_host,
     prepare,
     set_debug_flags,
+    sparse_attend,
+    sparse_prefill,
+    sparse_prepare,
     set_wait_timeout_ns,
     workspace_size,
 )
 
 __all__ = [
-    "Workspace", "attend", "decode", "decode_scratch_size", "decode_step", "host_arena_size", "prefill", "prefill_chunked", "prefill_host",
-    "prepare", "set_debug_flags", "set_wait_timeout_ns", "workspace_size",
+    "SparsePattern", "SparseWorkspace", "Workspace", "attend", "decode", "decode_scratch_size", "decode_step", "host_arena_size", "prefill", "prefill_chunked", "prefill_host",
+    "prepare", "set_debug_flags", "set_wait_timeout_ns", "sparse_attend", "sparse_prefill", "sparse_prepare",
+    "workspace_size",
 ]

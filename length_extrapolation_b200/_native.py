@@ -47,6 +47,13 @@ SIGNATURES = {
     "dca_decode_scratch_size": (_sz, [_i64, _i32, _i32]),
     "dca_decode": (_i32, [_vp, _vp, _vp, _vp, _i64, _i64, _i64, _i32, _i32, _i32, _i64, _i64,
                           _i64, _dbl, _i32, _vp, _vp, _sz, _vp, _sz, _vp]),
+    "dca_sparse_workspace_size": (_sz, [_vp, _i32]),
+    "dca_sparse_prepare": (_i32, [_vp, _vp, _vp, _vp, _vp, _i64, _i32, _i32, _i32, _i64, _i64,
+                                  _i64, _i32, _vp, _vp, _sz, _vp, _sz, _vp]),
+    "dca_sparse_attend": (_i32, [_vp, _vp, _vp, _vp, _i64, _i64, _i64, _i32, _i32, _i32, _i64,
+                                 _i64, _i64, _dbl, _i32, _vp, _vp, _sz, _vp, _sz, _vp]),
+    "dca_sparse_plan_items": (_i32, [_vp, _i64, _vp, _i64, _i64, _i64, _i64, _i64, _i32, _vp,
+                                     _i32]),
     "dca_set_wait_timeout_ns": (None, [_i64]),
     "dca_set_debug_flags": (None, [_i32]),
 }
@@ -56,6 +63,15 @@ _lib = None
 
 
 DCA_DECODE_MAX_TOKENS = 256
+
+
+DCA_SPARSE_MAX_RUNS = 1023
+
+
+class DCASparseConfig(ctypes.Structure):
+    """Mirror of dca_sparse_config (include/dca.h)."""
+    _fields_ = [("kv_capacity", ctypes.c_int64), ("max_vertical", ctypes.c_int64),
+                ("max_slash", ctypes.c_int64)]
 
 
 class DCAOptions(ctypes.Structure):

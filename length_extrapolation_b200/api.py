@@ -201,6 +201,112 @@ def decode_step(q_new, k_cache, v_cache, *, kv_len, chunk_size, local_window, pr
                   window_reading=window_reading)
 
 
+class SparsePattern:
+    """Per-query-head vertical keys and slash offsets (host CSR arrays) for
+    the vertical-slash sparse attention.  Lists are sorted, without repeats."""
+
+    def __init__(self, vertical, slash):
+        import numpy as np
+        if len(vertical) != len(slash):
+            raise ValueError("one vertical and one slash list per query head")
+        self.Hq = len(vertical)
+
+        def csr(lists):
+            ptr = np.zeros(len(lists) + 1, dtype=np.int64)
+            arrs = [np.asarray(a, dtype=np.int64).ravel() for a in lists]
+            for h, a in enumerate(arrs):
+                ptr[h + 1] = ptr[h] + a.size
+            idx = np.concatenate(arrs).astype(np.int32) if ptr[-1] else np.zeros(1, np.int32)
+            return ptr, np.ascontiguousarray(idx)
+
+        self.v_ptr, self.v_idx = csr(vertical)
+        self.s_ptr, self.s_off = csr(slash)
+        self.vertical = [np.asarray(a, dtype=np.int64) for a in vertical]
+        self.slash = [np.asarray(a, dtype=np.int64) for a in slash]
+
+    def max_vertical(self):
+        return int((self.v_ptr[1:] - self.v_ptr[:-1]).max())
+
+    def max_slash(self):
+        return int((self.s_ptr[1:] - self.s_ptr[:-1]).max())
+
+    def restricted(self, Lk):
+        """The pattern with vertical keys and slash offsets below Lk."""
+        return SparsePattern([a[a < Lk] for a in self.vertical], [a[a < Lk] for a in self.slash])
+
+
+class SparseWorkspace:
+    """Device memory for the sparse index structures (bitmaps, gathered
+    vertical rows); its layout is fixed by (kv_capacity, max_vertical,
+    max_slash, Hq)."""
+
+    def __init__(self, kv_capacity, Hq, max_vertical, max_slash, device="cuda"):
+        self.cfg = N.DCASparseConfig(int(kv_capacity), int(max_vertical), int(max_slash))
+        n = N.lib().dca_sparse_workspace_size(ctypes.byref(self.cfg), int(Hq))
+        if n == 0:
+            raise N.DCAError(N.DCA_ERR_ARG, "dca_sparse_workspace_size")
+        # 1 KiB alignment for the gathered rows' tensor maps
+        self.raw = torch.empty(n + 1024, dtype=torch.uint8, device=device)
+        off = (-self.raw.data_ptr()) % 1024
+        self.buf = self.raw[off:off + n]
+        self.nbytes = n
+        self.device = self.buf.device
+
+    @property
+    def ptr(self) -> int:
+        return self.buf.data_ptr()
+
+
+def sparse_prepare(pattern: SparsePattern, v_cache, *, kv_len, chunk_size, local_window,
+                   pretrain_window, workspace: Workspace, sparse: SparseWorkspace):
+    """Copy the pattern (restricted to keys < kv_len), build the bitmaps and
+    gather the vertical rows from the rotated keys in `workspace`."""
+    _check_cuda(v_cache)
+    pat = pattern.restricted(kv_len)
+    rc = N.lib().dca_sparse_prepare(
+        ctypes.byref(sparse.cfg), pat.v_ptr.ctypes.data, pat.v_idx.ctypes.data,
+        pat.s_ptr.ctypes.data, pat.s_off.ctypes.data, int(kv_len), pattern.Hq,
+        v_cache.shape[1], v_cache.shape[2], int(chunk_size), int(local_window),
+        int(pretrain_window), _dtype_code(v_cache), v_cache.data_ptr(), workspace.ptr,
+        workspace.nbytes, sparse.ptr, sparse.nbytes, _stream_ptr(v_cache.device))
+    N.check(rc, "dca_sparse_prepare")
+
+
+def sparse_attend(q_block, v_cache, out=None, *, q_start, kv_len, chunk_size, local_window,
+                  pretrain_window, yarn_scale=1.0, workspace: Workspace, sparse: SparseWorkspace,
+                  window_reading="query_offset"):
+    """Sparse DCA attention of a query block over the prepared structures."""
+    _check_cuda(q_block, v_cache)
+    Lq, Hq, d = q_block.shape
+    if out is None:
+        out = torch.empty_like(q_block)
+    opts = _options(window_reading)
+    rc = N.lib().dca_sparse_attend(
+        ctypes.byref(sparse.cfg), q_block.data_ptr(), v_cache.data_ptr(), out.data_ptr(),
+        int(q_start), Lq, int(kv_len), Hq, v_cache.shape[1], d, int(chunk_size),
+        int(local_window), int(pretrain_window), float(yarn_scale), _dtype_code(q_block),
+        ctypes.byref(opts), workspace.ptr, workspace.nbytes, sparse.ptr, sparse.nbytes,
+        _stream_ptr(q_block.device))
+    N.check(rc, "dca_sparse_attend")
+    return out
+
+
+def sparse_prefill(q, k, v, pattern: SparsePattern, *, chunk_size, local_window,
+                   pretrain_window, rope_base=1e7, yarn_scale=1.0, out=None,
+                   window_reading="query_offset"):
+    """One-shot sparse DCA prefill: rotate the keys, prepare the pattern, attend."""
+    L, Hq, d = q.shape
+    ws = Workspace(L, Hq, k.shape[1], d, chunk_size, local_window, pretrain_window, q.dtype,
+                   q.device)
+    kw = dict(chunk_size=chunk_size, local_window=local_window, pretrain_window=pretrain_window)
+    prepare(k, kv_len=L, k_rows_valid=0, rope_base=rope_base, workspace=ws, **kw)
+    sp = SparseWorkspace(L, Hq, max(1, pattern.max_vertical()), max(1, pattern.max_slash()),
+                         q.device)
+    sparse_prepare(pattern, v, kv_len=L, workspace=ws, sparse=sp, **kw)
+    return sparse_attend(q, v, out, q_start=0, kv_len=L, yarn_scale=yarn_scale, workspace=ws,
+                         sparse=sp, window_reading=window_reading, **kw)
+
+
 def host_arena_size(L, block, Hq, Hkv, d, chunk_size, local_window, pretrain_window, dtype):
     code = _DTYPES[dtype] if isinstance(dtype, torch.dtype) else int(dtype)
     n = N.lib().dca_host_arena_size(int(L), int(block), int(Hq), int(Hkv), int(d),

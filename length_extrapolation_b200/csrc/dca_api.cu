@@ -6,10 +6,12 @@
 #include <stdint.h>
 
 #include <atomic>
+#include <vector>
 
 #include "../../include/dca.h"
 #include "dca_internal.h"
 #include "dca_plan.cuh"
+#include "dca_sparse_plan.cuh"
 
 namespace {
 
@@ -149,6 +151,81 @@ int reading_of(const dca_options* opts) {
   for (int k = 0; k < 7; ++k)
     if (opts->reserved[k] != 0) return -1;
   return opts->window_reading;
+}
+
+// Sparse workspace: the host-copied prefix (counts, runs, lists), the
+// bitmaps, then the gathered vertical rows (1 KiB aligned for TMA).
+struct SparseLayout {
+  int64_t cap = 0, nv_cap = 0, s_cap = 0, wpr = 0;
+  size_t nv_off = 0, ns_off = 0, nruns_off = 0, runs_off = 0, vidx_off = 0, soff_off = 0;
+  size_t host_bytes = 0, vbit_off = 0, sbit_off = 0, gk_off = 0, gv_off = 0, total = 0;
+};
+
+bool sparse_cfg_ok(const dca_sparse_config* cfg) {
+  return cfg != nullptr && cfg->kv_capacity >= 1 && cfg->kv_capacity <= (1LL << 31) - 1 &&
+         cfg->max_vertical >= 0 && cfg->max_vertical <= (1LL << 31) - 1 && cfg->max_slash >= 0 &&
+         cfg->max_slash <= (1LL << 31) - 1;
+}
+
+SparseLayout make_sparse_layout(const dca_sparse_config* cfg, int Hq) {
+  SparseLayout S;
+  S.cap = cfg->kv_capacity;
+  S.nv_cap = (cfg->max_vertical + 127) / 128 * 128;
+  if (S.nv_cap < 128) S.nv_cap = 128;
+  S.s_cap = cfg->max_slash > 0 ? cfg->max_slash : 1;
+  S.wpr = S.cap / 32 + 8;  // bits 0 .. cap + 127 are readable (row padding)
+  size_t o = 0;
+  S.nv_off = o;
+  o = align_up(o + sizeof(int32_t) * Hq, 256);
+  S.ns_off = o;
+  o = align_up(o + sizeof(int32_t) * Hq, 256);
+  S.nruns_off = o;
+  o = align_up(o + sizeof(int32_t) * Hq, 256);
+  S.runs_off = o;
+  o = align_up(o + sizeof(int2) * static_cast<size_t>(Hq) * dca::SPARSE_MAX_RUNS, 256);
+  S.vidx_off = o;
+  o = align_up(o + sizeof(int32_t) * static_cast<size_t>(Hq) * S.nv_cap, 256);
+  S.soff_off = o;
+  o = align_up(o + sizeof(int32_t) * static_cast<size_t>(Hq) * S.s_cap, 256);
+  S.host_bytes = o;
+  S.vbit_off = o;
+  o = align_up(o + sizeof(uint32_t) * static_cast<size_t>(Hq) * S.wpr, 256);
+  S.sbit_off = o;
+  o = align_up(o + sizeof(uint32_t) * static_cast<size_t>(Hq) * S.wpr, 1024);
+  S.gk_off = o;
+  o = align_up(o + static_cast<size_t>(S.nv_cap) * Hq * 128 * 2, 1024);
+  S.gv_off = o;
+  o = align_up(o + static_cast<size_t>(S.nv_cap) * Hq * 128 * 2, 1024);
+  S.total = o;
+  return S;
+}
+
+dca::SparseArgs sparse_args(const SparseLayout& S, const void* sws) {
+  const uint8_t* b = static_cast<const uint8_t*>(sws);
+  dca::SparseArgs a;
+  a.vidx = reinterpret_cast<const int32_t*>(b + S.vidx_off);
+  a.nv = reinterpret_cast<const int32_t*>(b + S.nv_off);
+  a.runs = reinterpret_cast<const int2*>(b + S.runs_off);
+  a.nruns = reinterpret_cast<const int32_t*>(b + S.nruns_off);
+  a.vbit = reinterpret_cast<const uint32_t*>(b + S.vbit_off);
+  a.sbit = reinterpret_cast<const uint32_t*>(b + S.sbit_off);
+  a.gk = b + S.gk_off;
+  a.gv = b + S.gv_off;
+  a.wpr = S.wpr;
+  a.nv_cap = S.nv_cap;
+  return a;
+}
+
+// Checks one head's list: sorted, no repeats, inside [0, Lk); returns its
+// number of runs of consecutive values, or -1.
+int64_t list_runs(const int32_t* a, int64_t n, int64_t Lk) {
+  int64_t runs = 0;
+  for (int64_t e = 0; e < n; ++e) {
+    if (a[e] < 0 || a[e] >= Lk) return -1;
+    if (e > 0 && a[e] <= a[e - 1]) return -1;
+    if (e == 0 || a[e] != a[e - 1] + 1) ++runs;
+  }
+  return runs;
 }
 
 }  // namespace
@@ -426,5 +503,159 @@ void dca_set_wait_timeout_ns(int64_t ns) {
 }
 
 void dca_set_debug_flags(int flags) { g_debug_flags.store(flags); }
+
+size_t dca_sparse_workspace_size(const dca_sparse_config* cfg, int Hq) {
+  if (!sparse_cfg_ok(cfg) || Hq <= 0) return 0;
+  return make_sparse_layout(cfg, Hq).total;
+}
+
+int dca_sparse_prepare(const dca_sparse_config* cfg, const int64_t* v_ptr, const int32_t* v_idx,
+                       const int64_t* s_ptr, const int32_t* s_off, int64_t Lk, int Hq, int Hkv,
+                       int d, int64_t chunk_size, int64_t local_window, int64_t pretrain_window,
+                       int dtype, const void* v_cache, const void* workspace, size_t ws_bytes,
+                       void* sparse_ws, size_t sparse_bytes, void* cuda_stream) {
+  if (!sparse_cfg_ok(cfg) || v_ptr == nullptr || s_ptr == nullptr) return DCA_ERR_ARG;
+  // the dense workspace holds the rotated keys [0, Lk)
+  Layout L;
+  int rc = check_common(0, 0, Lk, Hq, Hkv, d, chunk_size, local_window, pretrain_window, 1.0,
+                        dtype, workspace, ws_bytes, &L);
+  if (rc != DCA_OK) return rc;
+  if (dtype != DCA_BF16) return DCA_ERR_UNSUPPORTED;
+  if (Lk < 1 || Lk > cfg->kv_capacity || !ptrs_ok(v_cache)) return DCA_ERR_ARG;
+  if (sparse_ws == nullptr || !aligned(sparse_ws, 1024)) return DCA_ERR_WORKSPACE;
+  const SparseLayout S = make_sparse_layout(cfg, Hq);
+  if (sparse_bytes < S.total) return DCA_ERR_WORKSPACE;
+  // host-side pattern checks and the copied prefix
+  std::vector<uint8_t> blob(S.host_bytes, 0);
+  int32_t* nv = reinterpret_cast<int32_t*>(blob.data() + S.nv_off);
+  int32_t* ns = reinterpret_cast<int32_t*>(blob.data() + S.ns_off);
+  int32_t* nr = reinterpret_cast<int32_t*>(blob.data() + S.nruns_off);
+  int2* runs = reinterpret_cast<int2*>(blob.data() + S.runs_off);
+  int32_t* vi = reinterpret_cast<int32_t*>(blob.data() + S.vidx_off);
+  int32_t* so = reinterpret_cast<int32_t*>(blob.data() + S.soff_off);
+  if (v_ptr[0] != 0 || s_ptr[0] != 0) return DCA_ERR_ARG;
+  for (int h = 0; h < Hq; ++h) {
+    const int64_t n_v = v_ptr[h + 1] - v_ptr[h], n_s = s_ptr[h + 1] - s_ptr[h];
+    if (n_v < 0 || n_v > cfg->max_vertical || n_s < 0 || n_s > cfg->max_slash) return DCA_ERR_ARG;
+    if ((n_v > 0 && v_idx == nullptr) || (n_s > 0 && s_off == nullptr)) return DCA_ERR_ARG;
+    if (n_v > 0 && list_runs(v_idx + v_ptr[h], n_v, Lk) < 0) return DCA_ERR_ARG;
+    const int64_t r = n_s > 0 ? list_runs(s_off + s_ptr[h], n_s, Lk) : 0;
+    if (r < 0 || r > dca::SPARSE_MAX_RUNS) return DCA_ERR_ARG;
+    nv[h] = static_cast<int32_t>(n_v);
+    ns[h] = static_cast<int32_t>(n_s);
+    nr[h] = static_cast<int32_t>(r);
+    for (int64_t e = 0; e < n_v; ++e) vi[h * S.nv_cap + e] = v_idx[v_ptr[h] + e];
+    int k = -1;
+    for (int64_t e = 0; e < n_s; ++e) {
+      const int32_t o = s_off[s_ptr[h] + e];
+      so[h * S.s_cap + e] = o;
+      if (e == 0 || o != s_off[s_ptr[h] + e - 1] + 1)
+        runs[h * dca::SPARSE_MAX_RUNS + (++k)] = make_int2(o, o + 1);
+      else
+        runs[h * dca::SPARSE_MAX_RUNS + k].y = o + 1;
+    }
+  }
+  cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
+  uint8_t* sb = static_cast<uint8_t*>(sparse_ws);
+  if (cudaMemcpyAsync(sb, blob.data(), S.host_bytes, cudaMemcpyHostToDevice, st) != cudaSuccess)
+    return DCA_ERR_CUDA;
+  if (cudaMemsetAsync(sb + S.vbit_off, 0, S.gk_off - S.vbit_off, st) != cudaSuccess)
+    return DCA_ERR_CUDA;
+  const dca::SparseArgs a = sparse_args(S, sparse_ws);
+  cudaError_t e = dca::launch_sparse_bits(a.vidx, a.nv, S.nv_cap,
+                                          reinterpret_cast<const int32_t*>(sb + S.soff_off),
+                                          reinterpret_cast<const int32_t*>(sb + S.ns_off), S.s_cap,
+                                          reinterpret_cast<uint32_t*>(sb + S.vbit_off),
+                                          reinterpret_cast<uint32_t*>(sb + S.sbit_off), S.wpr, Hq,
+                                          st);
+  if (e == cudaSuccess) {
+    const uint8_t* wb = static_cast<const uint8_t*>(workspace);
+    e = dca::launch_sparse_gather(a.vidx, a.nv, S.nv_cap, wb + L.kr_off, v_cache, sb + S.gk_off,
+                                  sb + S.gv_off, Hq, Hkv, st);
+  }
+  return e == cudaSuccess ? DCA_OK : DCA_ERR_CUDA;
+}
+
+int dca_sparse_attend(const dca_sparse_config* cfg, const void* q_block, const void* v_cache,
+                      void* out_block, int64_t q_start, int64_t Lq, int64_t Lk, int Hq, int Hkv,
+                      int d, int64_t chunk_size, int64_t local_window, int64_t pretrain_window,
+                      double yarn_scale, int dtype, const dca_options* opts, void* workspace,
+                      size_t ws_bytes, const void* sparse_ws, size_t sparse_bytes,
+                      void* cuda_stream) {
+  const int reading = reading_of(opts);
+  if (reading < 0 || !sparse_cfg_ok(cfg)) return DCA_ERR_ARG;
+  Layout L;
+  int rc = check_common(q_start, Lq, Lk, Hq, Hkv, d, chunk_size, local_window, pretrain_window,
+                        yarn_scale, dtype, workspace, ws_bytes, &L);
+  if (rc != DCA_OK) return rc;
+  if (dtype != DCA_BF16) return DCA_ERR_UNSUPPORTED;
+  if (Lk > cfg->kv_capacity) return DCA_ERR_ARG;
+  if (sparse_ws == nullptr || !aligned(sparse_ws, 1024)) return DCA_ERR_WORKSPACE;
+  const SparseLayout S = make_sparse_layout(cfg, Hq);
+  if (sparse_bytes < S.total) return DCA_ERR_WORKSPACE;
+  if (Lq == 0) return DCA_OK;
+  if (!ptrs_ok(q_block) || !ptrs_ok(v_cache) || !ptrs_ok(out_block)) return DCA_ERR_ARG;
+  uint8_t* base = static_cast<uint8_t*>(workspace);
+  dca::AttnArgs a;
+  a.q = q_block;
+  a.kr = base + L.kr_off;
+  a.v = v_cache;
+  a.out = out_block;
+  a.tab = reinterpret_cast<const float2*>(base + L.tab_off);
+  a.q_start = q_start;
+  a.Lq = Lq;
+  a.Lk = Lk;
+  a.s = chunk_size;
+  a.w = local_window;
+  a.tab_c1 = L.T - 1;
+  a.Hq = Hq;
+  a.Hkv = Hkv;
+  a.reading = reading;
+  a.scale_log2 = logit_scale_log2(yarn_scale, d);
+  a.status = reinterpret_cast<unsigned int*>(base);
+  a.timeout_ns = static_cast<unsigned long long>(g_timeout_ns.load());
+  a.debug = g_debug_flags.exchange(0);
+  const cudaError_t e = dca::launch_sparse_sm100(a, sparse_args(S, sparse_ws),
+                                                 static_cast<cudaStream_t>(cuda_stream));
+  return e == cudaSuccess ? DCA_OK : DCA_ERR_CUDA;
+}
+
+int dca_sparse_plan_items(const int32_t* v_idx, int64_t n_v, const int32_t* s_off, int64_t n_s,
+                          int64_t i0, int64_t i_last, int64_t chunk_size, int64_t local_window,
+                          int window_reading, int32_t* items, int max_items) {
+  if (chunk_size < 1 || local_window < 0 || local_window > chunk_size) return DCA_ERR_ARG;
+  if (window_reading != DCA_WINDOW_QUERY_OFFSET && window_reading != DCA_WINDOW_TRUE_DISTANCE)
+    return DCA_ERR_ARG;
+  if (i0 < 0 || i_last < i0 || i_last - i0 >= 128 || (i0 % 128) != 0) return DCA_ERR_ARG;
+  if (n_v < 0 || n_s < 0 || (n_v > 0 && !v_idx) || (n_s > 0 && !s_off) || max_items < 0 ||
+      (max_items > 0 && !items))
+    return DCA_ERR_ARG;
+  const int64_t lim = (1LL << 31) - 1;
+  if ((n_v > 0 && list_runs(v_idx, n_v, lim) < 0)) return DCA_ERR_ARG;
+  const int64_t nr = n_s > 0 ? list_runs(s_off, n_s, lim) : 0;
+  if (nr < 0 || nr > dca::SPARSE_MAX_RUNS) return DCA_ERR_ARG;
+  std::vector<int2> runs;
+  for (int64_t e = 0; e < n_s; ++e) {
+    if (e == 0 || s_off[e] != s_off[e - 1] + 1)
+      runs.push_back(make_int2(s_off[e], s_off[e] + 1));
+    else
+      runs.back().y = s_off[e] + 1;
+  }
+  std::vector<dca::SparsePlan> P(1);
+  dca::sparse_plan_build(P[0], v_idx, static_cast<int>(n_v), runs.data(), static_cast<int>(nr), i0,
+                         i_last, chunk_size, local_window, window_reading, 128);
+  dca::SparseIter it;
+  dca::sparse_iter_init(it);
+  int n = 0, src, tile, cls;
+  while (dca::sparse_iter_next(it, P[0], src, tile, cls)) {
+    if (n < max_items) {
+      items[3 * n] = src;
+      items[3 * n + 1] = tile;
+      items[3 * n + 2] = cls;
+    }
+    ++n;
+  }
+  return n;
+}
 
 }  // extern "C"

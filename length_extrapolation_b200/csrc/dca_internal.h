@@ -53,6 +53,21 @@ cudaError_t launch_rotate_keys(const void* k, void* kr, const float2* tab, int64
 // driver's encoder is unavailable or rejects the map.
 bool encode_kv_map(CUtensorMap* m, const void* base, int64_t n_rows, int Hkv);
 
+// Vertical-slash sparse attention: the index structures built by
+// dca_sparse_prepare in the sparse workspace.
+constexpr int SPARSE_MAX_RUNS = 1023;  // runs of consecutive slash offsets per head
+struct SparseArgs {
+  const int32_t* vidx;   // [Hq][nv_cap] sorted vertical keys
+  const int32_t* nv;     // [Hq]
+  const int2* runs;      // [Hq][SPARSE_MAX_RUNS] slash offset runs [x, y)
+  const int32_t* nruns;  // [Hq]
+  const uint32_t* vbit;  // [Hq][wpr]
+  const uint32_t* sbit;  // [Hq][wpr]
+  const void* gk;        // [nv_cap][Hq][128] gathered rotated keys
+  const void* gv;        // [nv_cap][Hq][128] gathered values
+  int64_t wpr, nv_cap;
+};
+
 // bf16 tcgen05/TMA kernel; returns a CUDA error or cudaSuccess, or
 // cudaErrorInvalidValue when a tensor map cannot be encoded.
 cudaError_t launch_attention_sm100(const AttnArgs& a, cudaStream_t st);
@@ -61,5 +76,16 @@ cudaError_t launch_attention_f32(const AttnArgs& a, cudaStream_t st);
 // bf16 split-KV decode (tcgen05) and the combine of its partial results into
 // out (and a.lse when set); `part` holds decode_part_floats(...) words.
 cudaError_t launch_decode_sm100(const AttnArgs& a, float* part, cudaStream_t st);
+// Sparse attention kernel over the structures of `sa` (bf16).
+cudaError_t launch_sparse_sm100(const AttnArgs& a, const SparseArgs& sa, cudaStream_t st);
+// Preparation: membership bitmaps from the per-head lists (zeroed before),
+// and the gathered vertical rows of the rotated keys and values.
+cudaError_t launch_sparse_bits(const int32_t* vidx, const int32_t* nv, int64_t nv_cap,
+                               const int32_t* soff, const int32_t* ns, int64_t s_cap,
+                               uint32_t* vbit, uint32_t* sbit, int64_t wpr, int Hq,
+                               cudaStream_t st);
+cudaError_t launch_sparse_gather(const int32_t* vidx, const int32_t* nv, int64_t nv_cap,
+                                 const void* kr, const void* v, void* gk, void* gv, int Hq,
+                                 int Hkv, cudaStream_t st);
 
 }  // namespace dca

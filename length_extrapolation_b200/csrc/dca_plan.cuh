@@ -92,6 +92,32 @@ DCA_HD TilePlan make_plan(int64_t i0, int64_t i_last, int64_t s, int64_t w, int 
   return P;
 }
 
+// Key ranges [lo, hi) of the three classes for the query rows [i0, i_last]
+// (the unions over the rows; the k-tile ranges of make_plan are these ranges
+// rounded out to tiles).  A pair (i, j) of class c has j inside range c.
+DCA_HD void class_key_ranges(int64_t i0, int64_t i_last, int64_t s, int64_t w, int reading,
+                             int64_t lo[3], int64_t hi[3]) {
+  const int64_t n0 = i0 / s, n1 = i_last / s;
+  int64_t inter_end = (n1 >= 2) ? s * (n1 - 1) : 0;
+  if (reading == READING_B && n1 >= 1) {
+    const int64_t far_end = (s * n1 < i_last - w + 1) ? s * n1 : i_last - w + 1;
+    if (far_end > inter_end) inter_end = far_end;
+  }
+  lo[CLS_INTER] = 0;
+  hi[CLS_INTER] = inter_end;
+  if (n1 >= 1 && (reading == READING_A || w > 0)) {
+    int64_t a = s * (n0 >= 1 ? n0 - 1 : 0);
+    const int64_t b = s * n1;
+    if (reading == READING_B && i0 - w + 1 > a) a = i0 - w + 1;
+    lo[CLS_SUCC] = a;
+    hi[CLS_SUCC] = a < b ? b : a;
+  } else {
+    lo[CLS_SUCC] = hi[CLS_SUCC] = 0;
+  }
+  lo[CLS_INTRA] = s * n0;
+  hi[CLS_INTRA] = i_last + 1;
+}
+
 // Item n of the work list -> (k-tile, class).  Order: INTER, SUCC, INTRA.
 DCA_HD void plan_item(const TilePlan& P, int n, int& kt, int& cls) {
   const int c2 = P.hi[CLS_INTER] - P.lo[CLS_INTER];

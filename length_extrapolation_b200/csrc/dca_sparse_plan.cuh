@@ -1,0 +1,169 @@
+// dca_sparse_plan.cuh -- the work list of one (128-row query tile, query
+// head) of the vertical-slash sparse attention, shared by the kernel (which
+// keeps the plan in shared memory) and the host introspection entry point.
+//
+// Items are 128-key tiles, visited class by class (INTER, SUCC, INTRA; see
+// dca_plan.cuh); within a class first the tiles of the head's gathered
+// vertical keys whose positions fall in the class's key range, then the
+// cache k-tiles that a slash diagonal (or the diagonal j = i) crosses for some
+// row of the tile, clipped to the class's k-tile range.  A tile shared by two
+// classes appears once per class; the kernel masks each item to its class.
+#pragma once
+#include <stdint.h>
+#include <vector_types.h>
+
+#include "dca_plan.cuh"
+
+namespace dca {
+
+constexpr int SPARSE_IV_MAX = 1024;  // slash runs per head (1023) + the diagonal j = i
+
+struct SparsePlan {
+  int n_items;
+  int n_iv;            // merged slash key-tile intervals
+  int nv_eff;          // vertical keys <= the tile's last row
+  int vt[3][2];        // vertical (gathered) tile range per class (indexed by CLS_*)
+  int ktr[3][2];       // cache k-tile range per class
+  int qbuf_of[3];      // query operand tile of each class, -1 if absent
+  int third_cls;       // class that reuses operand tile 0 (-1 if fewer than three)
+  int2 iv[SPARSE_IV_MAX];  // [x, y) k-tile intervals, ascending
+};
+
+DCA_HD int sparse_class_at(int ci) {  // visiting order INTER, SUCC, INTRA
+  return ci == 0 ? CLS_INTER : (ci == 1 ? CLS_SUCC : CLS_INTRA);
+}
+
+struct SparseIter {
+  int ci, phase;  // class index in visiting order; -1 start, 0 vertical, 1 slash
+  int t, t_end;   // current tile and the end of the current range
+  int iv;         // slash interval index
+};
+
+DCA_HD void sparse_iter_init(SparseIter& it) {
+  it.ci = 0;
+  it.phase = -1;
+  it.t = it.t_end = 0;
+  it.iv = 0;
+}
+
+// Next item: src 0 = vertical (gathered tile index), 1 = slash (cache k-tile).
+DCA_HD bool sparse_iter_next(SparseIter& it, const SparsePlan& P, int& src, int& tile, int& cls) {
+  for (;;) {
+    if (it.phase >= 0 && it.t < it.t_end) {
+      src = it.phase;
+      tile = it.t++;
+      cls = sparse_class_at(it.ci);
+      return true;
+    }
+    if (it.phase == 1) {
+      const int c = sparse_class_at(it.ci);
+      const int clo = P.ktr[c][0], chi = P.ktr[c][1];
+      while (it.iv < P.n_iv) {
+        const int2 r = P.iv[it.iv];
+        if (r.x >= chi) break;
+        ++it.iv;
+        const int a = r.x > clo ? r.x : clo;
+        const int b = r.y < chi ? r.y : chi;
+        if (a < b) {
+          it.t = a;
+          it.t_end = b;
+          break;
+        }
+      }
+      if (it.t < it.t_end) continue;
+      ++it.ci;
+      it.phase = -1;
+    }
+    if (it.ci >= 3) return false;
+    const int c = sparse_class_at(it.ci);
+    if (it.phase == -1) {
+      it.phase = 0;
+      it.t = P.vt[c][0];
+      it.t_end = P.vt[c][1];
+      continue;
+    }
+    // vertical tiles done: slash intervals from the first that reaches the class
+    it.phase = 1;
+    it.iv = 0;
+    while (it.iv < P.n_iv && P.iv[it.iv].y <= P.ktr[c][0]) ++it.iv;
+    it.t = it.t_end = 0;
+  }
+}
+
+// Builds the plan of the query rows [i0, i_last] for a head with nvh sorted
+// vertical keys vk and nr slash runs (offset ranges [x, y), ascending, at most
+// SPARSE_IV_MAX - 1).  bn = 128.
+DCA_HD void sparse_plan_build(SparsePlan& P, const int32_t* vk, int nvh, const int2* runs, int nr,
+                              int64_t i0, int64_t i_last, int64_t s, int64_t w, int reading,
+                              int bn) {
+  int64_t klo[3], khi[3];
+  class_key_ranges(i0, i_last, s, w, reading, klo, khi);
+  for (int c = 0; c < 3; ++c) {
+    P.ktr[c][0] = static_cast<int>(klo[c] / bn);
+    P.ktr[c][1] = khi[c] > klo[c] ? static_cast<int>(cdiv64(khi[c], bn)) : P.ktr[c][0];
+  }
+  // vertical tile ranges per class: positions of the class's key range
+  auto lower = [&](int64_t key) {
+    int lo = 0, hi = nvh;
+    while (lo < hi) {
+      const int mid = (lo + hi) >> 1;
+      if (vk[mid] < key) lo = mid + 1; else hi = mid;
+    }
+    return lo;
+  };
+  P.nv_eff = lower(i_last + 1);
+  for (int c = 0; c < 3; ++c) {
+    int a = 0, b = 0;
+    if (khi[c] > klo[c]) {
+      a = lower(klo[c]);
+      b = lower(khi[c]);
+      if (b > P.nv_eff) b = P.nv_eff;
+    }
+    P.vt[c][0] = a / bn;
+    P.vt[c][1] = b > a ? (b + bn - 1) / bn : a / bn;
+  }
+  // slash intervals: runs from the largest offsets down (ascending keys),
+  // the diagonal j = i always included, merged
+  int n_iv = 0;
+  for (int r = nr; r >= 0; --r) {
+    int64_t oa, ob;
+    if (r == 0) {
+      oa = 0;
+      ob = 1;
+    } else {
+      oa = runs[r - 1].x;
+      ob = runs[r - 1].y;
+    }
+    if (oa > i_last) continue;
+    int64_t ka = i0 - (ob - 1);
+    if (ka < 0) ka = 0;
+    const int64_t kb = i_last - oa;
+    const int ta = static_cast<int>(ka / bn), tb = static_cast<int>(kb / bn) + 1;
+    if (n_iv > 0 && ta <= P.iv[n_iv - 1].y) {
+      if (tb > P.iv[n_iv - 1].y) P.iv[n_iv - 1].y = tb;
+      if (ta < P.iv[n_iv - 1].x) P.iv[n_iv - 1].x = ta;
+    } else {
+      P.iv[n_iv].x = ta;
+      P.iv[n_iv].y = tb;
+      ++n_iv;
+    }
+  }
+  P.n_iv = n_iv;
+  // item count; operand tiles alternate between the classes in order of appearance
+  for (int c = 0; c < 3; ++c) P.qbuf_of[c] = -1;
+  P.third_cls = -1;
+  SparseIter it;
+  sparse_iter_init(it);
+  int n_items = 0, src, tile, cls, seen = 0;
+  while (sparse_iter_next(it, P, src, tile, cls)) {
+    if (P.qbuf_of[cls] < 0) {
+      P.qbuf_of[cls] = seen & 1;
+      if (seen == 2) P.third_cls = cls;
+      ++seen;
+    }
+    ++n_items;
+  }
+  P.n_items = n_items;
+}
+
+}  // namespace dca

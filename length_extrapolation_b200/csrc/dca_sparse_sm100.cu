@@ -1,0 +1,561 @@
+// dca_sparse_sm100.cu -- vertical-slash sparse Dual Chunk Attention for sm_100a.
+//
+// The Qwen2.5-1M framework runs MInference's vertical-slash sparse attention
+// on top of DCA ("Qwen2.5-1M 不重训外推 1M", sections "跟 NSA / 其他稀疏注意力的
+// 区别" and "稀疏注意力 + 核优化"): per query head, a few key columns (vertical
+// lines) and a few diagonals (slash lines) carry the attention, and only
+// those keys are attended.  For head h with vertical keys V_h and slash
+// offsets S_h, row i attends exactly
+//     M_h(i) = { j <= i : j in V_h } U { i - o : o in S_h, o <= i } U { i }
+// (each key once) with the DCA logits of the dense kernel and a softmax over
+// M_h(i).
+//
+// One CTA = one 128-row query tile of one query head (patterns are per head).
+// Its work list has two kinds of 128-key items, visited class by class
+// (INTER, SUCC, INTRA; dca_plan.cuh):
+//   vertical items  tiles of the head's gathered vertical keys (rotated keys
+//                   and values copied into a compact [n][Hq][128] array by
+//                   the preparation kernels), masked to j <= i and the class;
+//   slash items     K'/V tiles of the cache that a slash diagonal (or the
+//                   diagonal j = i) crosses for some row of the tile, masked
+//                   per element to the member pairs not already counted as
+//                   vertical, and to the class.
+// The slash tiles come from the head's runs of consecutive offsets, merged
+// into key-tile intervals once per CTA in shared memory.
+//
+// Warp roles as in the dense kernel (320 threads): warps 0-7 softmax (warp w
+// and w+4 split each row's 128 keys), warp 8 TMA producer (4-slot K/V ring,
+// no multicast), warp 9 MMA issuer.  With one head per CTA the two TMEM S
+// buffers alternate between consecutive items, so S(n+1) runs on the tensor
+// cores while the softmax warps work on S(n); P(n) overwrites the first 64
+// columns of its S buffer and feeds O += P V from TMEM.  Two query operand
+// tiles alternate between the classes in the order they appear (the third
+// class rewrites the first tile after the first class's last item).
+// Every wait is bounded; on timeout the CTA raises its abort flag, ORs a code
+// into the device status word, drains its copies and MMAs and exits.
+#include <cuda_bf16.h>
+#include <math.h>
+
+#include "dca_internal.h"
+#include "dca_plan.cuh"
+#include "dca_softmax.cuh"
+#include "dca_sparse_plan.cuh"
+#include "sm100_ptx.cuh"
+
+namespace dca {
+namespace sp {
+
+using namespace attn;
+
+constexpr int BM = 128, BN = 128, HD = 128;
+constexpr int NSLOT = 4;
+constexpr int TILE_BYTES = 32768;
+constexpr int NUM_THREADS = 320;
+constexpr int WARP_LOAD = 8, WARP_MMA = 9;
+constexpr float RESCALE_LOG2 = 8.0f;
+
+constexpr unsigned ST_SOFTMAX = 0x10u, ST_LOAD = 0x100u, ST_MMA = 0x1000u, ST_DRAIN = 0x10000u;
+
+struct SmemCtl {
+  uint64_t slot_full[NSLOT];
+  uint64_t slot_empty[NSLOT];
+  uint64_t s_full[2];
+  uint64_t p_full[2];
+  uint64_t pv_done[2];
+  uint64_t q_ready;
+  uint64_t o_final;
+  uint64_t drain;
+  uint64_t pair_bar[4];
+  uint32_t tmem_base;
+  int abort;
+  float xval[2][2][128];
+  SparsePlan plan;
+};
+
+constexpr size_t SMEM_BYTES = 1024 + 2 * TILE_BYTES + NSLOT * TILE_BYTES + sizeof(SmemCtl);
+static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+
+struct Params {
+  const __nv_bfloat16* q;
+  __nv_bfloat16* out;
+  const float2* tab;
+  const int32_t* vidx;    // [Hq][nv_cap] sorted vertical keys
+  const int32_t* nv;      // [Hq] vertical key counts
+  const int2* runs;       // [Hq][SPARSE_MAX_RUNS] slash offset runs [x, y), ascending
+  const int32_t* nruns;   // [Hq]
+  const uint32_t* vbit;   // [Hq][wpr] vertical membership bits (bit j)
+  const uint32_t* sbit;   // [Hq][wpr] slash offset bits (bit o)
+  int64_t wpr;            // words per head row of the bitmaps (>= cap/32 + 2)
+  int64_t nv_cap;
+  int64_t q_start, Lq, Lk;
+  int64_t s, w, tab_c1;
+  int Hq, Hkv, G, n_qtiles;
+  int reading;
+  float scale_log2;
+  unsigned int* status;
+  unsigned long long timeout_ns;
+};
+
+// 64 bits of a bitmap starting at bit `lo` (bits below 0 read as 0); the
+// bitmap row is padded with two zero words past its last bit.
+__device__ __forceinline__ uint64_t bits64(const uint32_t* row, int64_t lo) {
+  if (lo <= -64) return 0ull;
+  const int64_t base = lo < 0 ? 0 : lo;
+  const int64_t wd = base >> 5;
+  const int sh = static_cast<int>(base & 31);
+  const uint64_t w0 = row[wd], w1 = row[wd + 1], w2 = row[wd + 2];
+  uint64_t v = (w0 | (w1 << 32)) >> sh;
+  if (sh) v |= w2 << (64 - sh);
+  if (lo < 0) v <<= static_cast<int>(-lo);
+  return v;
+}
+
+// True when every bit of [lo, hi] (0 <= lo <= hi) is set.
+__device__ __forceinline__ bool all_bits(const uint32_t* row, int64_t lo, int64_t hi) {
+  for (int64_t b = lo; b <= hi; b += 64) {
+    const int64_t n = hi - b + 1 < 64 ? hi - b + 1 : 64;
+    const uint64_t want = n == 64 ? ~0ull : ((1ull << n) - 1);
+    if ((bits64(row, b) & want) != want) return false;
+  }
+  return true;
+}
+
+// One online-softmax step for half of a query row (see the dense kernel):
+// mask (when the item is not full) by causality, class and membership,
+// half-row max exchanged with the partner thread, exponentials into P (bf16,
+// first 64 columns of the S buffer), O rescaled when the reference moves
+// (after the previous item's P.V completed).
+__device__ __forceinline__ bool sparse_half_step(
+    uint32_t tS, uint32_t tO, int n, bool full, int src, int tile, int cls, int64_t i,
+    const Params& p, int h, float sc, int64_t nb, int64_t pb, float& m_ref, float& l_sum,
+    PairCtx& pc, SmemCtl* ctl, volatile int* abort, unsigned int* status) {
+  const int half = pc.half;
+  uint32_t sv[64];
+  tmem_ld64(tS + 64u * half, sv);
+  if (!full) {
+    const uint32_t NEG_INF = 0xff800000u;
+    if (src == 1) {
+      const int64_t j0 = static_cast<int64_t>(tile) * BN + 64 * half;
+      mask_cols<64>(sv, i, j0, cls, p.s, p.w, p.reading);
+      const uint32_t* vrow = p.vbit + static_cast<int64_t>(h) * p.wpr;
+      const uint32_t* srow = p.sbit + static_cast<int64_t>(h) * p.wpr;
+      const uint64_t vm = bits64(vrow, j0);
+      const int64_t base = i - j0;  // offset of key e is base - e
+      uint64_t sm = __brevll(bits64(srow, base - 63));
+      if (base >= 0 && base < 64) sm |= 1ull << base;
+      const uint64_t mem = sm & ~vm;
+#pragma unroll
+      for (int e = 0; e < 64; ++e)
+        if (!((mem >> e) & 1ull)) sv[e] = NEG_INF;
+    } else {
+      const int64_t pos0 = static_cast<int64_t>(tile) * BN + 64 * half;
+      const int nv = ctl->plan.nv_eff;
+      const int32_t* vk = p.vidx + static_cast<int64_t>(h) * p.nv_cap + pos0;
+#pragma unroll
+      for (int e4 = 0; e4 < 16; ++e4) {
+        int4 jj = make_int4(0x7fffffff, 0x7fffffff, 0x7fffffff, 0x7fffffff);
+        if (pos0 + 4 * e4 + 3 < nv) {
+          jj = *reinterpret_cast<const int4*>(vk + 4 * e4);
+        } else {
+          if (pos0 + 4 * e4 + 0 < nv) jj.x = vk[4 * e4 + 0];
+          if (pos0 + 4 * e4 + 1 < nv) jj.y = vk[4 * e4 + 1];
+          if (pos0 + 4 * e4 + 2 < nv) jj.z = vk[4 * e4 + 2];
+        }
+        const int js[4] = {jj.x, jj.y, jj.z, jj.w};
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int64_t j = js[u];
+          int c;
+          if (j >= nb) c = CLS_INTRA;
+          else if (j >= pb && (p.reading == READING_A || i - j < p.w)) c = CLS_SUCC;
+          else c = CLS_INTER;
+          if (j > i || c != cls) sv[4 * e4 + u] = NEG_INF;
+        }
+      }
+    }
+  }
+  float mx = max64(sv);
+  float mx_other = -INFINITY;
+  if (!pair_exchange(pc, mx, mx_other, abort, status, p.timeout_ns, ST_SOFTMAX)) return false;
+  mx = fmaxf(mx, mx_other);
+
+  const float m_new = fmaxf(m_ref, mx);
+  const bool need =
+      (m_new > m_ref) && (m_ref == -INFINITY || (m_new - m_ref) * sc > RESCALE_LOG2);
+  float alpha = 1.f;
+  if (need) {
+    alpha = (m_ref == -INFINITY) ? 0.f : ex2_approx((m_ref - m_new) * sc);
+    m_ref = m_new;
+    l_sum *= alpha;
+  }
+  uint32_t pk[32];
+  l_sum += exp_pack64(sv, sc, (m_ref == -INFINITY) ? 0.f : m_ref * sc, pk);
+  tmem_st32(tS + 32u * half, pk);
+  // O holds items < n; the P.V of item n - 1 must have landed before a rescale
+  if (n > 0 && __any_sync(0xffffffffu, need)) {
+    const int m = n - 1;
+    bool ok = wait_bounded(&ctl->pv_done[m & 1], static_cast<uint32_t>((m >> 1) & 1), abort,
+                           status, p.timeout_ns, ST_SOFTMAX);
+    if (!__all_sync(0xffffffffu, ok)) return false;
+    tc_fence_after();
+#pragma unroll
+    for (int c = 0; c < 2; ++c) {
+      uint32_t o[32];
+      tmem_ld32(tO + 64u * half + 32u * c, o);
+#pragma unroll
+      for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+      tmem_st32(tO + 64u * half + 32u * c, o);
+    }
+  }
+  tmem_st_wait();
+  return true;
+}
+
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+    dca_sparse_kernel(const __grid_constant__ CUtensorMap tm_k,
+                      const __grid_constant__ CUtensorMap tm_v,
+                      const __grid_constant__ CUtensorMap tm_gk,
+                      const __grid_constant__ CUtensorMap tm_gv, const Params p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint8_t* q_buf[2] = {smem, smem + TILE_BYTES};
+  uint8_t* slots = smem + 2 * TILE_BYTES;
+  SmemCtl* ctl = reinterpret_cast<SmemCtl*>(slots + NSLOT * TILE_BYTES);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  // ---- work unit: the G heads of a KV group next to each other (they cross
+  // the same slash tiles of the cache), longest query tiles first
+  const int qt = p.n_qtiles - 1 - static_cast<int>(blockIdx.x / p.Hq);
+  const int h = static_cast<int>(blockIdx.x % p.Hq);
+  const int g = h / p.G;
+  const int64_t i0 = p.q_start + static_cast<int64_t>(qt) * BM;
+  const int64_t q_end = p.q_start + p.Lq;
+  const int64_t i_last = (i0 + BM - 1 < q_end - 1) ? i0 + BM - 1 : q_end - 1;
+  const int64_t i_hi = i0 + BM - 1;
+
+  if (threadIdx.x == 0) {
+    for (int k = 0; k < NSLOT; ++k) {
+      mbar_init(&ctl->slot_full[k], 1);
+      mbar_init(&ctl->slot_empty[k], 1);
+    }
+    for (int st = 0; st < 2; ++st) {
+      mbar_init(&ctl->s_full[st], 1);
+      mbar_init(&ctl->p_full[st], 8);
+      mbar_init(&ctl->pv_done[st], 1);
+    }
+    mbar_init(&ctl->q_ready, 8);
+    mbar_init(&ctl->o_final, 1);
+    mbar_init(&ctl->drain, 1);
+    for (int k = 0; k < 4; ++k) mbar_init(&ctl->pair_bar[k], 2);
+    ctl->abort = 0;
+    fence_barrier_init();
+
+    // ---- the CTA's work list
+    sparse_plan_build(ctl->plan, p.vidx + static_cast<int64_t>(h) * p.nv_cap, p.nv[h],
+                      p.runs + static_cast<int64_t>(h) * SPARSE_MAX_RUNS, p.nruns[h], i0, i_last,
+                      p.s, p.w, p.reading, BN);
+  }
+  if (warp == WARP_MMA) {
+    tmem_alloc(&ctl->tmem_base, 512);
+    tmem_relinquish();
+  }
+  if (warp == WARP_LOAD && lane == 0) {
+    tma_prefetch_desc(&tm_k);
+    tma_prefetch_desc(&tm_v);
+    tma_prefetch_desc(&tm_gk);
+    tma_prefetch_desc(&tm_gv);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tbase = ctl->tmem_base;
+  volatile int* abort_flag = &ctl->abort;
+  const SparsePlan& plan = ctl->plan;
+  const int N = plan.n_items;
+
+  if (warp < 8) {
+    // =========================================================== softmax
+    const int half = warp >> 2;
+    const int sub = warp & 3;
+    const int r = sub * 32 + lane;
+    PairCtx pc;
+    pc.xval = &ctl->xval[0][0][0];
+    pc.bar = &ctl->pair_bar[sub];
+    pc.ph = 0;
+    pc.half = half;
+    pc.r = r;
+    pc.lane = lane;
+    const int64_t i = i0 + r;
+    const bool real = i <= i_last;
+    const uint32_t lane_off = static_cast<uint32_t>(sub * 32) << 16;
+    const float sc = p.scale_log2;
+    const __nv_bfloat16* qrow =
+        real ? p.q + ((i - p.q_start) * p.Hq + h) * static_cast<int64_t>(HD) : nullptr;
+    const int c0 = 4 * half, c1 = 4 * half + 4;
+    const int64_t nb = (i / p.s) * p.s, pb = nb - p.s;  // chunk start of row i, and the previous
+    // query operands of the first two classes
+#pragma unroll
+    for (int c = 0; c < 3; ++c) {
+      const int b = plan.qbuf_of[c];
+      if (b < 0 || c == plan.third_cls) continue;
+      const float2* trow = real ? p.tab + query_table_row(i, c, p.s, p.w, p.tab_c1) * 64 : nullptr;
+      write_q_row(q_buf[b], r, qrow, trow, c0, c1);
+    }
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&ctl->q_ready);
+
+    SparseIter it;
+    sparse_iter_init(it);
+    float m_ref = -INFINITY, l_sum = 0.f;
+    bool ok = true;
+    int src, tile, cls;
+    for (int n = 0; n < N && ok; ++n) {
+      sparse_iter_next(it, plan, src, tile, cls);
+      // full item: every pair causal, of this class and a member
+      bool full;
+      if (src == 1) {
+        const int64_t j0 = static_cast<int64_t>(tile) * BN, j1 = j0 + BN - 1;
+        full = item_is_full(i0, i_hi, j0, j1, p.s, p.w, cls, p.reading);
+        if (full) {
+          const uint32_t* vrow = p.vbit + static_cast<int64_t>(h) * p.wpr;
+          full = (bits64(vrow, j0) | bits64(vrow, j0 + 64)) == 0ull;
+        }
+        if (full) full = i0 - j1 >= 0 &&
+                         all_bits(p.sbit + static_cast<int64_t>(h) * p.wpr, i0 - j1, i_hi - j0);
+      } else {
+        const int64_t pos0 = static_cast<int64_t>(tile) * BN;
+        full = pos0 + BN <= plan.nv_eff;
+        if (full) {
+          const int32_t* vk = p.vidx + static_cast<int64_t>(h) * p.nv_cap;
+          const int64_t ja = vk[pos0], jb = vk[pos0 + BN - 1];
+          full = jb <= i0 && item_is_full(i0, i_hi, ja, jb, p.s, p.w, cls, p.reading);
+        }
+      }
+      const int st = n & 1;
+      ok = wait_poll(&ctl->s_full[st], static_cast<uint32_t>((n >> 1) & 1), abort_flag, p.status,
+                     p.timeout_ns, ST_SOFTMAX);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      tc_fence_after();
+      const uint32_t tS = tbase + lane_off + static_cast<uint32_t>(st * 128);
+      const uint32_t tO = tbase + lane_off + 256u;
+      ok = sparse_half_step(tS, tO, n, full, src, tile, cls, i, p, h, sc, nb, pb, m_ref, l_sum,
+                            pc, ctl, abort_flag, p.status);
+      if (!ok) break;
+      // the first class ends: its operand tile becomes the third class's
+      if (plan.third_cls >= 0 && plan.qbuf_of[cls] == 0 && cls != plan.third_cls) {
+        SparseIter peek = it;
+        int s2, t2, c2;
+        if (n + 1 < N && sparse_iter_next(peek, plan, s2, t2, c2) && c2 != cls) {
+          const float2* trow =
+              real ? p.tab + query_table_row(i, plan.third_cls, p.s, p.w, p.tab_c1) * 64 : nullptr;
+          write_q_row(q_buf[0], r, qrow, trow, c0, c1);
+          fence_proxy_async_smem();
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&ctl->p_full[st]);
+    }
+    // epilogue: O / (l_half0 + l_half1) -> bf16 -> out
+    if (ok && N > 0) {
+      ok = wait_bounded(&ctl->o_final, 0u, abort_flag, p.status, p.timeout_ns, ST_SOFTMAX);
+      ok = __all_sync(0xffffffffu, ok);
+    }
+    float l_other = 0.f;
+    if (ok) ok = pair_exchange(pc, l_sum, l_other, abort_flag, p.status, p.timeout_ns, ST_SOFTMAX);
+    if (ok && N > 0) {
+      const float l_tot = l_sum + l_other;
+      tc_fence_after();
+      const uint32_t tO = tbase + lane_off + 256u + 64u * half;
+      const float inv = 1.f / l_tot;
+      __nv_bfloat16* orow =
+          real ? p.out + ((i - p.q_start) * p.Hq + h) * static_cast<int64_t>(HD) + 64 * half
+               : nullptr;
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        uint32_t o[32];
+        tmem_ld32(tO + 32u * c, o);
+        if (real) {
+#pragma unroll
+          for (int v4 = 0; v4 < 4; ++v4) {
+            uint4 w4;
+            w4.x = pack_bf16(__uint_as_float(o[8 * v4 + 0]) * inv, __uint_as_float(o[8 * v4 + 1]) * inv);
+            w4.y = pack_bf16(__uint_as_float(o[8 * v4 + 2]) * inv, __uint_as_float(o[8 * v4 + 3]) * inv);
+            w4.z = pack_bf16(__uint_as_float(o[8 * v4 + 4]) * inv, __uint_as_float(o[8 * v4 + 5]) * inv);
+            w4.w = pack_bf16(__uint_as_float(o[8 * v4 + 6]) * inv, __uint_as_float(o[8 * v4 + 7]) * inv);
+            *reinterpret_cast<uint4*>(orow + 32 * c + 8 * v4) = w4;
+          }
+        }
+      }
+    }
+  } else if (warp == WARP_LOAD) {
+    // =========================================================== TMA producer
+    if (lane == 0) {
+      int last_li[NSLOT];
+#pragma unroll
+      for (int k = 0; k < NSLOT; ++k) last_li[k] = -1;
+      SparseIter it;
+      sparse_iter_init(it);
+      bool ok = true;
+      int src, tile, cls;
+      for (int n = 0; n < N && ok; ++n) {
+        sparse_iter_next(it, plan, src, tile, cls);
+        for (int which = 0; which < 2; ++which) {  // 0: keys, 1: values
+          const int li = 2 * n + which;
+          const int slot = li % NSLOT;
+          const int use = li / NSLOT;
+          if (use > 0) {
+            ok = wait_bounded(&ctl->slot_empty[slot], static_cast<uint32_t>((use - 1) & 1),
+                              abort_flag, p.status, p.timeout_ns, ST_LOAD);
+            if (!ok) break;
+          }
+          uint8_t* dst = slots + slot * TILE_BYTES;
+          const CUtensorMap* tm = src == 1 ? (which ? &tm_v : &tm_k) : (which ? &tm_gv : &tm_gk);
+          const int head_coord = src == 1 ? g : h;
+          mbar_arrive_expect_tx(&ctl->slot_full[slot], TILE_BYTES);
+          tma_load_3d(dst, tm, &ctl->slot_full[slot], 0, head_coord, tile * BN);
+          tma_load_3d(dst + HALF_BYTES, tm, &ctl->slot_full[slot], 64, head_coord, tile * BN);
+          last_li[slot] = li;
+        }
+      }
+      for (int k = 0; k < NSLOT; ++k)
+        if (last_li[k] >= 0)
+          wait_drain(&ctl->slot_full[k], static_cast<uint32_t>((last_li[k] / NSLOT) & 1),
+                     p.status, p.timeout_ns, ST_DRAIN);
+    }
+    __syncwarp();
+  } else if (warp == WARP_MMA) {
+    // =========================================================== MMA issuer
+    if (lane == 0) {
+      const uint32_t id_s = idesc_bf16_f32(BM, BN, false);
+      const uint32_t id_o = idesc_bf16_f32(BM, HD, true);
+      const uint64_t dq[2] = {sdesc_sw128(smem_u32(q_buf[0]), 16, 1024),
+                              sdesc_sw128(smem_u32(q_buf[1]), 16, 1024)};
+      const uint64_t dk0 = sdesc_sw128(smem_u32(slots), 16, 1024);
+      const uint64_t dv0 = sdesc_sw128(smem_u32(slots), HALF_BYTES, 1024);
+      auto full_wait = [&](int li) {
+        return wait_spin(&ctl->slot_full[li % NSLOT], static_cast<uint32_t>((li / NSLOT) & 1),
+                         abort_flag, p.status, p.timeout_ns, ST_MMA);
+      };
+      SparseIter it;
+      sparse_iter_init(it);
+      int src, tile, cls;
+      // S(n) into buffer n & 1 with the class's query operand
+      auto issue_s = [&](int n) {
+        const int li = 2 * n;
+        const uint64_t dk = dk0 + static_cast<uint64_t>(((li % NSLOT) * TILE_BYTES) >> 4);
+        const uint64_t dqc = dq[plan.qbuf_of[cls]];
+#pragma unroll
+        for (int kk = 0; kk < HD / 16; ++kk) {
+          const uint64_t off = static_cast<uint64_t>(((kk >> 2) * HALF_BYTES + (kk & 3) * 32) >> 4);
+          mma_ss(tbase + static_cast<uint32_t>((n & 1) * 128), dqc + off, dk + off, id_s,
+                 kk > 0 ? 1u : 0u);
+        }
+        mma_commit(&ctl->s_full[n & 1]);
+        mma_commit(&ctl->slot_empty[li % NSLOT]);
+      };
+      bool ok = wait_bounded(&ctl->q_ready, 0u, abort_flag, p.status, p.timeout_ns, ST_MMA);
+      int issued = 0;  // S issued for items < issued
+      for (int k = 0; k < 2 && k < N && ok; ++k) {
+        sparse_iter_next(it, plan, src, tile, cls);
+        ok = full_wait(2 * k);
+        if (!ok) break;
+        tc_fence_after();
+        issue_s(k);
+        ++issued;
+      }
+      for (int n = 0; n < N && ok; ++n) {
+        const int lv = 2 * n + 1;
+        ok = full_wait(lv);
+        if (!ok) break;
+        ok = wait_spin(&ctl->p_full[n & 1], static_cast<uint32_t>((n >> 1) & 1), abort_flag,
+                       p.status, p.timeout_ns, ST_MMA);
+        if (!ok) break;
+        tc_fence_after();
+        const uint64_t dv = dv0 + static_cast<uint64_t>(((lv % NSLOT) * TILE_BYTES) >> 4);
+#pragma unroll
+        for (int kk = 0; kk < BN / 16; ++kk) {
+          mma_ts(tbase + 256u, tbase + static_cast<uint32_t>((n & 1) * 128 + kk * 8),
+                 dv + static_cast<uint64_t>((kk * 2048) >> 4), id_o, (n > 0 || kk > 0) ? 1u : 0u);
+        }
+        mma_commit(&ctl->pv_done[n & 1]);
+        mma_commit(&ctl->slot_empty[lv % NSLOT]);
+        if (issued < N) {  // S(n + 2) reuses buffer n & 1 after P.V(n) (in issue order)
+          sparse_iter_next(it, plan, src, tile, cls);
+          ok = full_wait(2 * issued);
+          if (!ok) break;
+          // the query operand of a class that reuses tile 0 is written by the
+          // softmax warps before they release P(n); P.V(n) waited for that
+          tc_fence_after();
+          issue_s(issued);
+          ++issued;
+        }
+      }
+      if (ok && N > 0) mma_commit(&ctl->o_final);
+      mma_commit(&ctl->drain);
+      wait_drain(&ctl->drain, 0u, p.status, p.timeout_ns, ST_DRAIN);
+    }
+    __syncwarp();
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == WARP_MMA) {
+    tc_fence_after();
+    tmem_dealloc(tbase, 512);
+  }
+}
+
+}  // namespace sp
+
+cudaError_t launch_sparse_sm100(const AttnArgs& a, const SparseArgs& sa, cudaStream_t st) {
+  using namespace sp;
+  if (a.Lq <= 0) return cudaSuccess;
+  CUtensorMap tm_k, tm_v, tm_gk, tm_gv;
+  if (!encode_kv_map(&tm_k, a.kr, a.Lk, a.Hkv) || !encode_kv_map(&tm_v, a.v, a.Lk, a.Hkv) ||
+      !encode_kv_map(&tm_gk, sa.gk, sa.nv_cap, a.Hq) ||
+      !encode_kv_map(&tm_gv, sa.gv, sa.nv_cap, a.Hq))
+    return cudaErrorInvalidValue;
+  Params p;
+  p.q = static_cast<const __nv_bfloat16*>(a.q);
+  p.out = static_cast<__nv_bfloat16*>(a.out);
+  p.tab = a.tab;
+  p.vidx = sa.vidx;
+  p.nv = sa.nv;
+  p.runs = sa.runs;
+  p.nruns = sa.nruns;
+  p.vbit = sa.vbit;
+  p.sbit = sa.sbit;
+  p.wpr = sa.wpr;
+  p.nv_cap = sa.nv_cap;
+  p.q_start = a.q_start;
+  p.Lq = a.Lq;
+  p.Lk = a.Lk;
+  p.s = a.s;
+  p.w = a.w;
+  p.tab_c1 = a.tab_c1;
+  p.Hq = a.Hq;
+  p.Hkv = a.Hkv;
+  p.G = a.Hq / a.Hkv;
+  p.n_qtiles = static_cast<int>((a.Lq + BM - 1) / BM);
+  p.reading = a.reading;
+  p.scale_log2 = a.scale_log2;
+  p.status = a.status;
+  p.timeout_ns = a.timeout_ns;
+  const int64_t blocks = static_cast<int64_t>(p.n_qtiles) * p.Hq;
+  if (blocks > 0x7fffffffLL) return cudaErrorInvalidValue;
+  cudaError_t e = cudaFuncSetAttribute(dca_sparse_kernel,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(SMEM_BYTES));
+  if (e != cudaSuccess) return e;
+  dca_sparse_kernel<<<static_cast<unsigned>(blocks), NUM_THREADS, SMEM_BYTES, st>>>(
+      tm_k, tm_v, tm_gk, tm_gv, p);
+  return cudaGetLastError();
+}
+
+}  // namespace dca

@@ -206,3 +206,55 @@ DECODE_WORKLOADS = {
         DecodeWorkload("qwen7b_1m_decode_q4", WORKLOADS["qwen7b_1m_chunked"], Lk=1048576, Lq=4),
     ]
 }
+
+
+def sparse_pattern(L: int, Hq: int, n_vertical: int, n_band: int, n_far: int, n_init: int = 4,
+                   seed: int = 0):
+    """Seeded synthetic vertical-slash pattern per query head (lists of sorted
+    key indices and diagonal offsets in [0, L)).  Vertical keys: the first
+    n_init tokens plus uniform random others; slash offsets: the band
+    0 .. n_band - 1 (local diagonals) plus n_far uniform random far offsets.
+    The real per-head patterns are searched offline on calibration data."""
+    import numpy as np
+    rng = np.random.default_rng(seed + 1000)
+    vertical, slash = [], []
+    for _ in range(Hq):
+        nv = min(n_vertical, L)
+        init = np.arange(min(n_init, nv))
+        rest = rng.choice(np.arange(len(init), L), size=max(0, min(nv - len(init), L - len(init))),
+                          replace=False) if nv > len(init) else np.zeros(0, np.int64)
+        vertical.append(np.unique(np.concatenate([init, rest])).astype(np.int64))
+        band = np.arange(min(n_band, L))
+        far = rng.choice(np.arange(len(band), L), size=max(0, min(n_far, L - len(band))),
+                         replace=False) if L > len(band) and n_far > 0 else np.zeros(0, np.int64)
+        slash.append(np.unique(np.concatenate([band, far])).astype(np.int64))
+    return vertical, slash
+
+
+@dataclasses.dataclass(frozen=True)
+class SparseWorkload:
+    """A vertical-slash sparse prefill: the DCA parameters, shapes and query
+    blocks of `base`, and per query head n_vertical vertical keys (the first
+    4 tokens plus random others), a band of n_band local diagonals and n_far
+    random far diagonals."""
+    name: str
+    base: Workload
+    n_vertical: int
+    n_band: int
+    n_far: int
+
+
+def generate_sparse(sw: SparseWorkload, seed: int = 0):
+    """The workload's seeded per-head (vertical, slash) lists."""
+    return sparse_pattern(sw.base.L, sw.base.Hq, sw.n_vertical, sw.n_band, sw.n_far, seed=seed)
+
+
+# Pattern sizes in the range the sparse-attention literature uses at these
+# lengths (about a thousand key columns and a few thousand diagonals per head).
+SPARSE_WORKLOADS = {
+    sw.name: sw
+    for sw in [
+        SparseWorkload("qwen7b_256k_sparse", WORKLOADS["qwen7b_256k"], 1000, 4096, 64),
+        SparseWorkload("qwen7b_1m_sparse", WORKLOADS["qwen7b_1m_chunked"], 1000, 4096, 64),
+    ]
+}
