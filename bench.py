@@ -38,11 +38,13 @@ if ROOT not in sys.path:
 
 import torch  # noqa: E402
 
-from length_extrapolation_b200.workloads import (DECODE_WORKLOADS, WORKLOADS,  # noqa: E402
-                                                 generate, generate_decode, sample_heads)
+from length_extrapolation_b200.workloads import (DECODE_WORKLOADS, SPARSE_WORKLOADS,  # noqa: E402
+                                                 WORKLOADS, generate, generate_decode,
+                                                 generate_sparse, sample_heads)
 
 METRIC = "DCA prefill tokens/s and attention TFLOP/s (fraction of B200 bf16 peak)"
 DECODE_METRIC = "DCA decode tokens/s (KV-cache stream, fraction of B200 HBM bandwidth)"
+SPARSE_METRIC = "vertical-slash sparse DCA prefill tokens/s (member-pair TFLOP/s)"
 UNIT = "tokens/s"
 
 
@@ -53,7 +55,7 @@ def parse_args(argv=None):
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="qwen7b_1m_chunked",
-                    choices=sorted(WORKLOADS) + sorted(DECODE_WORKLOADS),
+                    choices=sorted(WORKLOADS) + sorted(DECODE_WORKLOADS) + sorted(SPARSE_WORKLOADS),
                     help="a prefill workload, or a decode step (*_decode*: the new tokens "
                          "against a full cache)")
     ap.add_argument("--e2e-steps", type=int, default=2)
@@ -532,9 +534,168 @@ def run_decode_bench(args, dw, world, rank, local, dist):
     return 0
 
 
+# ----------------------------------------------------------------------------- sparse
+def member_pairs(V, S, L, rows=None):
+    """Sum over query heads and rows i of |{j <= i in V_h} U {i - o : o in S_h,
+    o <= i} U {i}| (the sparse variant's attended pairs), in closed form:
+    sum_v (L - v) + sum_o (L - o) - #{(v, o) : v + o < L} + the rows whose
+    own key is in neither set.  `rows` = (r0, r1) restricts to rows [r0, r1)."""
+    import numpy as np
+    r0, r1 = (0, L) if rows is None else rows
+    tot = 0
+    for Vh, Sh in zip(V, S):
+        Vh = np.asarray(Vh, dtype=np.int64)
+        Sh = np.asarray(Sh, dtype=np.int64)
+        a = np.clip(r1 - np.maximum(Vh, r0), 0, None).sum()
+        b = np.clip(r1 - np.maximum(Sh, r0), 0, None).sum()
+        both = np.add.outer(Vh, Sh)
+        ov = np.count_nonzero((both >= r0) & (both < r1))
+        own = 0 if (Sh.size and Sh[0] == 0) else (r1 - r0) - np.count_nonzero((Vh >= r0) & (Vh < r1))
+        tot += int(a + b - ov + own)
+    return tot
+
+
+def sparse_config(sw):
+    w = sw.base
+    return {**workload_config(w), "workload": sw.name, "n_vertical": sw.n_vertical,
+            "n_band": sw.n_band, "n_far": sw.n_far}
+
+
+def run_sparse_bench(args, sw, world, rank, local, dist):
+    """One step = one whole chunked sparse prefill: per query block, rotate
+    the block's keys, prepare the pattern for the grown cache (copy, bitmaps,
+    gather of the vertical rows), run the sparse attention kernel."""
+    import numpy as np
+    w = sw.base
+    V, S = generate_sparse(sw)
+    pairs = member_pairs(V, S, w.L)
+    flops = 4.0 * w.d * pairs
+    if args.impl == "reference" or (rank == 0 and world == 1 and not args.no_cpu_baseline):
+        import oracle
+        qc, kc, vc = generate(w, device="cpu")
+        q0, lq, _ = w.blocks()[-1]
+        heads = sample_heads(w).numpy()
+        threads = os.cpu_count() or 1
+        rows = np.arange(lq - 64, lq)
+        t0 = time.perf_counter()
+        oracle.sparse_attention(qc[q0:q0 + lq], kc, vc, vertical=V, slash=S, q_start=q0,
+                                rows=rows, heads=heads, n_threads=threads, **w.params())
+        dt = time.perf_counter() - t0
+        done = member_pairs([V[h] for h in heads], [S[h] for h in heads], w.L,
+                            rows=(q0 + lq - 64, q0 + lq))
+        t_full = dt * pairs / done
+        cpu = {"value": w.L / t_full, "unit": UNIT, "cores": threads, "kind": "oracle",
+               "sample": f"64 rows x {len(heads)} heads of the last block ({done:.3e} member "
+                         f"pairs in {dt:.1f} s); extrapolated by member pairs"}
+        if args.impl == "reference":
+            if rank == 0:
+                print(json.dumps({
+                    "impl": "reference", "metric": SPARSE_METRIC, "value": cpu["value"],
+                    "unit": UNIT, "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+                    "ms_per_step": t_full * 1e3, "higher_is_better": True, "scaling": "weak",
+                    "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+                    "config": sparse_config(sw), "cpu_baseline": cpu,
+                    "e2e": {"value": cpu["value"], "unit": UNIT, "h2d_bytes_per_step": 0,
+                            "d2h_bytes_per_step": 0}}), flush=True)
+            return 0
+        del qc, kc, vc
+    else:
+        cpu = None
+
+    import length_extrapolation_b200 as dca
+    from length_extrapolation_b200 import _native as N
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    peaks = load_peaks()
+    q, k, v = generate(w, device=dev, seed=0)
+    out = torch.empty_like(q)
+    pat = dca.SparsePattern(V, S)
+    kw = dict(chunk_size=w.chunk_size, local_window=w.local_window,
+              pretrain_window=w.pretrain_window)
+    ws = dca.Workspace(w.L, w.Hq, w.Hkv, w.d, w.chunk_size, w.local_window, w.pretrain_window,
+                       q.dtype, dev)
+    sp = dca.SparseWorkspace(w.L, w.Hq, pat.max_vertical(), pat.max_slash(), dev)
+    blocks = w.blocks()
+    # the pattern restricted to each block's cache, built once (host lists)
+    pats = [pat.restricted(lk) for _, _, lk in blocks]
+
+    def step(evs=None):
+        for b, (q0, lq, lk) in enumerate(blocks):
+            dca.prepare(k, kv_len=lk, k_rows_valid=q0, rope_base=w.rope_base, workspace=ws, **kw)
+            dca.sparse_prepare(pats[b], v, kv_len=lk, workspace=ws, sparse=sp, **kw)
+            if evs is not None:
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record()
+            dca.sparse_attend(q[q0:q0 + lq], v, out[q0:q0 + lq], q_start=q0, kv_len=lk,
+                              yarn_scale=w.yarn_scale, workspace=ws, sparse=sp, **kw)
+            if evs is not None:
+                e1.record()
+                evs.append((e0, e1))
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if ws.status() != N.DCA_OK:
+        raise RuntimeError("device status after warm-up")
+    clocks = ClockSampler(dev.index).start()
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    evs = []
+    t0.record()
+    for _ in range(args.steps):
+        step(evs)
+    t1.record()
+    torch.cuda.synchronize()
+    if dist is not None:
+        dist.barrier()
+    clk = clocks.stop()
+    if ws.status() != N.DCA_OK:
+        raise RuntimeError("device status after timing")
+    ms, attn_ms = max_over_ranks([t0.elapsed_time(t1), sum(a.elapsed_time(b) for a, b in evs)],
+                                 dist, dev)
+    ms_per_step = ms / args.steps
+    # processed tiles: items x 128 x 128 pairs (host plan of every query tile and head)
+    achieved = flops * args.steps / (attn_ms / 1e3) / 1e12
+    roofline = {
+        "kernel": "dca_sparse_kernel (tcgen05, vertical-slash)", "bound": "tensor",
+        "achieved": achieved, "peak": peaks["bf16_tflops_sustained"], "unit": "TFLOP/s",
+        "frac": achieved / peaks["bf16_tflops_sustained"],
+        "peak_kind": f"{peaks['source']} sustained bf16 (cuBLAS, power-capped loop)",
+        "algorithmic_flops_per_step": flops, "member_pairs_per_step": pairs,
+        "dense_causal_pairs_per_step": total_pair_heads(w),
+        "traffic": None, "launches_per_step": len(blocks),
+        "avg_launch_ms": attn_ms / (args.steps * len(blocks)),
+    }
+    line = {
+        "metric": SPARSE_METRIC, "value": whole_job_rate(w.L, world, ms_per_step), "unit": UNIT,
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": w.dtype,
+        "data": "synthetic",
+        "config": {**sparse_config(sw), "parallelism": f"replicas x{world}" if world > 1 else "1 GPU"},
+        "tflops_member_pairs": world * flops / (ms_per_step / 1e3) / 1e12,
+        "roofline": roofline, "e2e": None, "cpu_baseline": cpu, "clocks": clk,
+        "gpu_launches": args.steps * len(blocks) * 5,  # rotate, 2 prep kernels, attend (+ memset)
+        "peaks_source": peaks["source"],
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
 # ----------------------------------------------------------------------------- our arm
 def main(argv=None):
     args = parse_args(argv)
+    if args.workload in SPARSE_WORKLOADS:
+        world = int(os.environ.get("WORLD_SIZE", "1"))
+        rank = int(os.environ.get("RANK", "0"))
+        local = int(os.environ.get("LOCAL_RANK", "0"))
+        dist = init_dist(world, local)
+        return run_sparse_bench(args, SPARSE_WORKLOADS[args.workload], world, rank, local, dist)
     if args.workload in DECODE_WORKLOADS:
         world = int(os.environ.get("WORLD_SIZE", "1"))
         rank = int(os.environ.get("RANK", "0"))

@@ -254,6 +254,7 @@ def generate_sparse(sw: SparseWorkload, seed: int = 0):
 SPARSE_WORKLOADS = {
     sw.name: sw
     for sw in [
+        SparseWorkload("qwen7b_32k_sparse", WORKLOADS["qwen7b_32k"], 1000, 4096, 64),
         SparseWorkload("qwen7b_256k_sparse", WORKLOADS["qwen7b_256k"], 1000, 4096, 64),
         SparseWorkload("qwen7b_1m_sparse", WORKLOADS["qwen7b_1m_chunked"], 1000, 4096, 64),
     ]
