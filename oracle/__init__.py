@@ -74,6 +74,11 @@ def _load():
             vp, vp, vp, i32, i64, i64, i64, i32, i32, i32, i64, i64, i64, dbl, dbl,
             i32, i32, vp, vp, vp, vp, vp, i64, vp, i32, vp, vp, i32]
         lib.dca_oracle_sparse_attention.restype = i32
+        lib.dca_oracle_vs_scores.argtypes = [vp, vp, i32, i64, i64, i64, i32, i32, i32, i64, i64,
+                                             i64, dbl, dbl, i32, i64, i32, vp, vp, i32]
+        lib.dca_oracle_vs_scores.restype = i32
+        lib.dca_oracle_topk.argtypes = [vp, i64, i64, vp]
+        lib.dca_oracle_topk.restype = i32
         lib.dca_oracle_position.argtypes = [i64, i64, i64, i64, i64, i32, i32,
                                             ctypes.POINTER(i64), ctypes.POINTER(i64)]
         lib.dca_oracle_position.restype = i32
@@ -209,3 +214,36 @@ def sparse_attention(q, k, v, *, vertical, slash, chunk_size, local_window, pret
     if rc != 0:
         raise ValueError(f"oracle returned {rc}")
     return (out, lse) if return_lse else out
+
+
+def vs_scores(q, k, *, chunk_size, local_window, pretrain_window, rope_base=1e7, yarn_scale=1.0,
+              q_start=0, kv_len=None, n_last=64, continuous=False, reading=0, n_threads=None):
+    """Key-selection scores (definition in dca_oracle.c): vertical [Hq, Lk]
+    and slash [Hq, Lk] fp64 from the last n_last rows of the query block,
+    with DCA logits or (continuous=True) RoPE logits at the true positions."""
+    qa, dt = _as_input(q)
+    ka, dtk = _as_input(k)
+    if dt != dtk:
+        raise TypeError("q, k must share a dtype")
+    Lq, Hq, d = qa.shape
+    Lk = ka.shape[0] if kv_len is None else int(kv_len)
+    vert = np.zeros((Hq, Lk), dtype=np.float64)
+    slash = np.zeros((Hq, Lk), dtype=np.float64)
+    rc = _load().dca_oracle_vs_scores(
+        qa.ctypes.data, ka.ctypes.data, dt, int(q_start), Lq, Lk, Hq, ka.shape[1], d,
+        int(chunk_size), int(local_window), int(pretrain_window), float(rope_base),
+        float(yarn_scale), int(reading), int(n_last), 1 if continuous else 0, vert.ctypes.data,
+        slash.ctypes.data, int(n_threads or os.cpu_count() or 1))
+    if rc != 0:
+        raise ValueError(f"oracle returned {rc}")
+    return vert, slash
+
+
+def topk(score, n):
+    """The n indices of largest score (ties: smaller index), ascending."""
+    score = np.ascontiguousarray(score, dtype=np.float64)
+    out = np.zeros(max(1, n), dtype=np.int64)
+    m = _load().dca_oracle_topk(score.ctypes.data, score.size, int(n), out.ctypes.data)
+    if m != n:
+        raise ValueError("bad top-k arguments")
+    return out[:n]

@@ -55,6 +55,17 @@
  * (each key once; the row's own key always, so no row is empty), with the
  * DCA logits above and a softmax over M_h(i).
  *
+ * Key selection for the sparse variant (dca_oracle_vs_scores): the estimate
+ * from which the per-head vertical and slash sets are chosen.  For the last
+ * n_last rows i of the query block and query head h, p_ij is the softmax over
+ * keys j <= i of the logits, either the DCA logits above or -- the
+ * refinement of "稀疏注意力 + 核优化", which restores continuous relative
+ * positions at this stage -- plain RoPE logits with the true positions
+ * (query rotated by i, key by j).  Then
+ *      vertical_h[j] = sum_rows p_ij,   slash_h[o] = sum_rows p_{i, i-o}.
+ * The n_v keys and n_s offsets of largest score (ties: the smaller index)
+ * form the head's pattern (dca_oracle_topk).
+ *
  * The oracle also carries a `mutation` argument used only by tests that
  * check that the pins catch plausible mistakes (each value plants one known
  * mistake).  mutation = 0 is the oracle proper.
@@ -513,6 +524,153 @@ int dca_oracle_sparse_attention(const void* q, const void* k, const void* v, int
   return attention_impl(q, k, v, dtype, q_start, Lq, Lk, Hq, Hkv, d, s, w, c, base, yarn,
                         reading, mutation, v_ptr, v_idx, s_ptr, s_off, rows, n_rows, heads,
                         n_heads, out, lse, n_threads);
+}
+
+/*
+ * Vertical / slash scores of the key selection (definition in the header).
+ * q [Lq][Hq][d] query block (row t at absolute index q_start + t), k
+ * [Lk][Hkv][d]; the last n_last rows of the block are the estimate's rows.
+ * continuous = 0: DCA logits; 1: RoPE logits at the true positions.
+ * vert, slash [Hq][Lk] fp64 outputs.  Returns 0, -1 on bad arguments,
+ * -3 on allocation failure.  Single-threaded per head, parallel over heads.
+ */
+typedef struct {
+  const void *q, *k;
+  int dtype;
+  int64_t q_start, Lq, Lk, n_last;
+  int Hq, Hkv, d;
+  int64_t s, w, c;
+  double base, yarn;
+  int reading, continuous;
+  const double* theta;
+  double *vert, *slash;
+  int next;
+  pthread_mutex_t mu;
+  int status;
+} vs_job_t;
+
+static void vs_head(vs_job_t* J, int h) {
+  const int d = J->d;
+  const int G = J->Hq / J->Hkv, g = h / G;
+  double* logit = (double*)malloc(sizeof(double) * (size_t)J->Lk);
+  double* kraw = (double*)malloc(sizeof(double) * (size_t)d);
+  double* kr = (double*)malloc(sizeof(double) * (size_t)d);
+  double* qraw = (double*)malloc(sizeof(double) * (size_t)d);
+  double* qv = (double*)malloc(sizeof(double) * (size_t)d);
+  if (!logit || !kraw || !kr || !qraw || !qv) {
+    pthread_mutex_lock(&J->mu);
+    J->status = -3;
+    pthread_mutex_unlock(&J->mu);
+    free(logit); free(kraw); free(kr); free(qraw); free(qv);
+    return;
+  }
+  double scale = (1.0 / sqrt((double)d)) * dca_oracle_mscale(J->yarn) * dca_oracle_mscale(J->yarn);
+  double* vert = J->vert + (int64_t)h * J->Lk;
+  double* slash = J->slash + (int64_t)h * J->Lk;
+  for (int64_t j = 0; j < J->Lk; ++j) vert[j] = slash[j] = 0.0;
+  for (int64_t t = J->Lq - J->n_last; t < J->Lq; ++t) {
+    const int64_t i = J->q_start + t;
+    for (int e = 0; e < d; ++e) qraw[e] = to_f64(J->q, J->dtype, (t * J->Hq + h) * (int64_t)d + e);
+    double mx = -INFINITY;
+    for (int64_t j = 0; j <= i; ++j) {
+      int64_t pq, pk;
+      if (J->continuous) {
+        pq = i;
+        pk = j;
+      } else {
+        dca_oracle_position(i, j, J->s, J->w, J->c, J->reading, MUT_NONE, &pq, &pk);
+      }
+      rotate(qraw, qv, d, pq, J->theta, MUT_NONE);
+      for (int e = 0; e < d; ++e) kraw[e] = to_f64(J->k, J->dtype, (j * J->Hkv + g) * (int64_t)d + e);
+      rotate(kraw, kr, d, pk, J->theta, MUT_NONE);
+      double dot = 0.0;
+      for (int e = 0; e < d; ++e) dot += qv[e] * kr[e];
+      logit[j] = scale * dot;
+      if (logit[j] > mx) mx = logit[j];
+    }
+    double sum = 0.0;
+    for (int64_t j = 0; j <= i; ++j) sum += exp(logit[j] - mx);
+    for (int64_t j = 0; j <= i; ++j) {
+      const double p = exp(logit[j] - mx) / sum;
+      vert[j] += p;
+      slash[i - j] += p;
+    }
+  }
+  free(logit); free(kraw); free(kr); free(qraw); free(qv);
+}
+
+static void* vs_worker(void* arg) {
+  vs_job_t* J = (vs_job_t*)arg;
+  for (;;) {
+    pthread_mutex_lock(&J->mu);
+    int h = J->next++;
+    pthread_mutex_unlock(&J->mu);
+    if (h >= J->Hq) break;
+    vs_head(J, h);
+  }
+  return NULL;
+}
+
+int dca_oracle_vs_scores(const void* q, const void* k, int dtype, int64_t q_start, int64_t Lq,
+                         int64_t Lk, int Hq, int Hkv, int d, int64_t s, int64_t w, int64_t c,
+                         double base, double yarn, int reading, int64_t n_last, int continuous,
+                         double* vert, double* slash, int n_threads) {
+  if (!q || !k || !vert || !slash) return -1;
+  if (dtype < 0 || dtype > 2 || d <= 0 || d % 2 || Hq <= 0 || Hkv <= 0 || Hq % Hkv) return -1;
+  if (s < 1 || w < 0 || c < 1 || q_start < 0 || Lq < 1 || Lk < q_start + Lq) return -1;
+  if (n_last < 1 || n_last > Lq) return -1;
+  if (n_threads < 1) n_threads = 1;
+  double* theta = (double*)malloc(sizeof(double) * (size_t)(d / 2));
+  pthread_t* th = (pthread_t*)malloc(sizeof(pthread_t) * (size_t)n_threads);
+  if (!theta || !th) {
+    free(theta);
+    free(th);
+    return -3;
+  }
+  for (int kk = 0; kk < d / 2; ++kk) theta[kk] = pow(base, -2.0 * kk / d);
+  vs_job_t J;
+  memset(&J, 0, sizeof J);
+  J.q = q; J.k = k; J.dtype = dtype; J.q_start = q_start; J.Lq = Lq; J.Lk = Lk;
+  J.n_last = n_last; J.Hq = Hq; J.Hkv = Hkv; J.d = d; J.s = s; J.w = w; J.c = c;
+  J.base = base; J.yarn = yarn; J.reading = reading; J.continuous = continuous;
+  J.theta = theta; J.vert = vert; J.slash = slash;
+  pthread_mutex_init(&J.mu, NULL);
+  for (int t = 0; t < n_threads; ++t) pthread_create(&th[t], NULL, vs_worker, &J);
+  for (int t = 0; t < n_threads; ++t) pthread_join(th[t], NULL);
+  pthread_mutex_destroy(&J.mu);
+  free(theta);
+  free(th);
+  return J.status;
+}
+
+/* The n indices of largest score among score[0 .. len) (ties: the smaller
+ * index), written ascending to out[0 .. n): sort by (score descending,
+ * index ascending), keep the first n, sort those by index.  Returns n, or -1. */
+typedef struct {
+  double v;
+  int64_t j;
+} sj_t;
+
+static int cmp_score_desc(const void* a, const void* b) {
+  const sj_t* x = (const sj_t*)a;
+  const sj_t* y = (const sj_t*)b;
+  if (x->v != y->v) return x->v > y->v ? -1 : 1;
+  return (x->j > y->j) - (x->j < y->j);
+}
+
+int dca_oracle_topk(const double* score, int64_t len, int64_t n, int64_t* out) {
+  if (!score || !out || n < 0 || n > len) return -1;
+  sj_t* a = (sj_t*)malloc(sizeof(sj_t) * (size_t)(len > 0 ? len : 1));
+  if (!a) return -1;
+  for (int64_t j = 0; j < len; ++j) {
+    a[j].v = score[j];
+    a[j].j = j;
+  }
+  qsort(a, (size_t)len, sizeof(sj_t), cmp_score_desc);
+  for (int64_t r = 0; r < n; ++r) out[r] = a[r].j;
+  qsort(out, (size_t)n, sizeof(int64_t), cmp_i64);
+  free(a);
+  return (int)n;
 }
 
 int dca_oracle_attention(const void* q, const void* k, const void* v, int dtype,
