@@ -237,6 +237,41 @@ int dca_sparse_attend(const dca_sparse_config* cfg, const void* q_block, const v
                       void* cuda_stream);
 
 /*
+ * Online key selection ("稀疏注意力 + 核优化": the fix restores continuous
+ * relative positions at the key-selection stage, because DCA's remapped
+ * positions break the diagonal pattern).  From the last n_last (1..64) rows
+ * i of the query block (absolute rows q_start + Lq - n_last ..), per query
+ * head: p_ij = softmax over keys j <= i of the logits -- the DCA logits, or
+ * with continuous_positions = 1 RoPE logits at the true positions i and j --
+ * vertical score of key j = sum_rows p_ij, slash score of offset o =
+ * sum_rows p_{i, i-o}; the n_vertical keys and n_slash offsets of largest
+ * score (ties: the smaller index) become the head's pattern in sparse_ws,
+ * with its bitmaps and gathered vertical rows, ready for dca_sparse_attend
+ * (no host round trip).  Requires the rotated keys [0, Lk) in `workspace`
+ * (dca_prepare), n_vertical <= cfg->max_vertical, n_slash <= min(cfg->max_slash,
+ * DCA_SPARSE_MAX_RUNS), bf16.  scratch: dca_sparse_select_scratch_size bytes,
+ * 256-byte aligned.
+ */
+size_t dca_sparse_select_scratch_size(int64_t Lk, int Hq, int64_t chunk_size);
+int dca_sparse_select(const dca_sparse_config* cfg, const void* q_block, const void* v_cache,
+                      int64_t q_start, int64_t Lq, int64_t Lk, int Hq, int Hkv, int d,
+                      int64_t chunk_size, int64_t local_window, int64_t pretrain_window,
+                      double rope_base, double yarn_scale, int dtype, const dca_options* opts,
+                      int n_last, int continuous_positions, int64_t n_vertical, int64_t n_slash,
+                      void* workspace, size_t ws_bytes, void* sparse_ws, size_t sparse_bytes,
+                      void* scratch, size_t scratch_bytes, void* cuda_stream);
+
+/*
+ * Copies the pattern held by sparse_ws to host memory (synchronises the
+ * stream): per head the count and sorted list of vertical keys
+ * (v_counts [Hq], v_idx [Hq][cfg->max_vertical]) and of slash offsets
+ * (s_counts [Hq], s_off [Hq][cfg->max_slash]).
+ */
+int dca_sparse_pattern_get(const dca_sparse_config* cfg, int Hq, const void* sparse_ws,
+                           size_t sparse_bytes, int32_t* v_counts, int32_t* v_idx,
+                           int32_t* s_counts, int32_t* s_off, void* cuda_stream);
+
+/*
  * Host-side introspection of the sparse kernel's work list (no GPU needed):
  * for the query tile whose rows are [i0, i0 + 128) (i0 a multiple of 128) with
  * real rows up to i_last, and one head's sorted vertical keys / slash offsets

@@ -20,14 +20,17 @@ from .api import (  # noqa: F401
     prepare,
     set_debug_flags,
     sparse_attend,
+    sparse_pattern_get,
     sparse_prefill,
     sparse_prepare,
+    sparse_select,
     set_wait_timeout_ns,
     workspace_size,
 )
 
 __all__ = [
     "SparsePattern", "SparseWorkspace", "Workspace", "attend", "decode", "decode_scratch_size", "decode_step", "host_arena_size", "prefill", "prefill_chunked", "prefill_host",
-    "prepare", "set_debug_flags", "set_wait_timeout_ns", "sparse_attend", "sparse_prefill", "sparse_prepare",
+    "prepare", "set_debug_flags", "set_wait_timeout_ns", "sparse_attend", "sparse_pattern_get", "sparse_prefill",
+    "sparse_prepare", "sparse_select",
     "workspace_size",
 ]

@@ -54,6 +54,11 @@ SIGNATURES = {
                                  _i64, _i64, _dbl, _i32, _vp, _vp, _sz, _vp, _sz, _vp]),
     "dca_sparse_plan_items": (_i32, [_vp, _i64, _vp, _i64, _i64, _i64, _i64, _i64, _i32, _vp,
                                      _i32]),
+    "dca_sparse_select_scratch_size": (_sz, [_i64, _i32, _i64]),
+    "dca_sparse_select": (_i32, [_vp, _vp, _vp, _i64, _i64, _i64, _i32, _i32, _i32, _i64, _i64,
+                                 _i64, _dbl, _dbl, _i32, _vp, _i32, _i32, _i64, _i64, _vp, _sz,
+                                 _vp, _sz, _vp, _sz, _vp]),
+    "dca_sparse_pattern_get": (_i32, [_vp, _i32, _vp, _sz, _vp, _vp, _vp, _vp, _vp]),
     "dca_set_wait_timeout_ns": (None, [_i64]),
     "dca_set_debug_flags": (None, [_i32]),
 }

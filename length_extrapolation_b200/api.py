@@ -291,6 +291,47 @@ def sparse_attend(q_block, v_cache, out=None, *, q_start, kv_len, chunk_size, lo
     return out
 
 
+def sparse_select(q_block, v_cache, *, q_start, kv_len, chunk_size, local_window,
+                  pretrain_window, rope_base=1e7, yarn_scale=1.0, n_vertical, n_slash,
+                  n_last=64, continuous=True, workspace: Workspace, sparse: SparseWorkspace,
+                  scratch=None, window_reading="query_offset"):
+    """Online key selection into `sparse` from the last n_last rows of the
+    block (continuous=True: true positions, the refinement; False: DCA)."""
+    _check_cuda(q_block, v_cache)
+    Lq, Hq, d = q_block.shape
+    if scratch is None:
+        n = N.lib().dca_sparse_select_scratch_size(int(kv_len), Hq, int(chunk_size))
+        if n == 0:
+            raise N.DCAError(N.DCA_ERR_ARG, "dca_sparse_select_scratch_size")
+        scratch = torch.empty(n, dtype=torch.uint8, device=q_block.device)
+    opts = _options(window_reading)
+    rc = N.lib().dca_sparse_select(
+        ctypes.byref(sparse.cfg), q_block.data_ptr(), v_cache.data_ptr(), int(q_start), Lq,
+        int(kv_len), Hq, v_cache.shape[1], d, int(chunk_size), int(local_window),
+        int(pretrain_window), float(rope_base), float(yarn_scale), _dtype_code(q_block),
+        ctypes.byref(opts), int(n_last), 1 if continuous else 0, int(n_vertical), int(n_slash),
+        workspace.ptr, workspace.nbytes, sparse.ptr, sparse.nbytes, scratch.data_ptr(),
+        scratch.numel(), _stream_ptr(q_block.device))
+    N.check(rc, "dca_sparse_select")
+
+
+def sparse_pattern_get(sparse: SparseWorkspace, Hq):
+    """(vertical, slash) lists per head currently held by `sparse` (syncs)."""
+    import numpy as np
+    mv, ms = int(sparse.cfg.max_vertical), int(sparse.cfg.max_slash)
+    vc = np.zeros(Hq, np.int32)
+    sc = np.zeros(Hq, np.int32)
+    vi = np.zeros(max(1, Hq * mv), np.int32)
+    so = np.zeros(max(1, Hq * ms), np.int32)
+    rc = N.lib().dca_sparse_pattern_get(ctypes.byref(sparse.cfg), Hq, sparse.ptr, sparse.nbytes,
+                                        vc.ctypes.data, vi.ctypes.data, sc.ctypes.data,
+                                        so.ctypes.data, _stream_ptr(sparse.device))
+    N.check(rc, "dca_sparse_pattern_get")
+    V = [vi[h * mv:h * mv + vc[h]].astype(np.int64) for h in range(Hq)]
+    S = [so[h * ms:h * ms + sc[h]].astype(np.int64) for h in range(Hq)]
+    return V, S
+
+
 def sparse_prefill(q, k, v, pattern: SparsePattern, *, chunk_size, local_window,
                    pretrain_window, rope_base=1e7, yarn_scale=1.0, out=None,
                    window_reading="query_offset"):

@@ -515,6 +515,7 @@ int dca_sparse_prepare(const dca_sparse_config* cfg, const int64_t* v_ptr, const
                        int dtype, const void* v_cache, const void* workspace, size_t ws_bytes,
                        void* sparse_ws, size_t sparse_bytes, void* cuda_stream) {
   if (!sparse_cfg_ok(cfg) || v_ptr == nullptr || s_ptr == nullptr) return DCA_ERR_ARG;
+  if (dtype == DCA_F32) return DCA_ERR_UNSUPPORTED;  // the sparse path is bf16
   // the dense workspace holds the rotated keys [0, Lk)
   Layout L;
   int rc = check_common(0, 0, Lk, Hq, Hkv, d, chunk_size, local_window, pretrain_window, 1.0,
@@ -584,6 +585,7 @@ int dca_sparse_attend(const dca_sparse_config* cfg, const void* q_block, const v
                       void* cuda_stream) {
   const int reading = reading_of(opts);
   if (reading < 0 || !sparse_cfg_ok(cfg)) return DCA_ERR_ARG;
+  if (dtype == DCA_F32) return DCA_ERR_UNSUPPORTED;  // the sparse path is bf16
   Layout L;
   int rc = check_common(q_start, Lq, Lk, Hq, Hkv, d, chunk_size, local_window, pretrain_window,
                         yarn_scale, dtype, workspace, ws_bytes, &L);
@@ -656,6 +658,116 @@ int dca_sparse_plan_items(const int32_t* v_idx, int64_t n_v, const int32_t* s_of
     ++n;
   }
   return n;
+}
+
+size_t dca_sparse_select_scratch_size(int64_t Lk, int Hq, int64_t chunk_size) {
+  if (Lk < 1 || Lk > (1LL << 31) - 1 || Hq <= 0 || chunk_size < 1) return 0;
+  return dca::select_scratch_bytes(Lk, Hq, (Lk + chunk_size - 1) / chunk_size);
+}
+
+int dca_sparse_select(const dca_sparse_config* cfg, const void* q_block, const void* v_cache,
+                      int64_t q_start, int64_t Lq, int64_t Lk, int Hq, int Hkv, int d,
+                      int64_t chunk_size, int64_t local_window, int64_t pretrain_window,
+                      double rope_base, double yarn_scale, int dtype, const dca_options* opts,
+                      int n_last, int continuous_positions, int64_t n_vertical, int64_t n_slash,
+                      void* workspace, size_t ws_bytes, void* sparse_ws, size_t sparse_bytes,
+                      void* scratch, size_t scratch_bytes, void* cuda_stream) {
+  const int reading = reading_of(opts);
+  if (reading < 0 || !sparse_cfg_ok(cfg)) return DCA_ERR_ARG;
+  if (dtype == DCA_F32) return DCA_ERR_UNSUPPORTED;  // the sparse path is bf16
+  Layout L;
+  int rc = check_common(q_start, Lq, Lk, Hq, Hkv, d, chunk_size, local_window, pretrain_window,
+                        yarn_scale, dtype, workspace, ws_bytes, &L);
+  if (rc != DCA_OK) return rc;
+  if (dtype != DCA_BF16) return DCA_ERR_UNSUPPORTED;
+  if (!(rope_base > 0.0) || !isfinite(rope_base)) return DCA_ERR_ARG;
+  if (Lq < 1 || n_last < 1 || n_last > 64 || n_last > Lq || Lk > cfg->kv_capacity)
+    return DCA_ERR_ARG;
+  if (continuous_positions != 0 && continuous_positions != 1) return DCA_ERR_ARG;
+  if (n_vertical < 0 || n_vertical > cfg->max_vertical || n_slash < 0 ||
+      n_slash > cfg->max_slash || n_slash > dca::SPARSE_MAX_RUNS)
+    return DCA_ERR_ARG;
+  if (!ptrs_ok(q_block) || !ptrs_ok(v_cache)) return DCA_ERR_ARG;
+  if (sparse_ws == nullptr || !aligned(sparse_ws, 1024)) return DCA_ERR_WORKSPACE;
+  const SparseLayout S = make_sparse_layout(cfg, Hq);
+  if (sparse_bytes < S.total) return DCA_ERR_WORKSPACE;
+  const int64_t n_chunks = (Lk + chunk_size - 1) / chunk_size;
+  if (scratch == nullptr || !aligned(scratch, 256) ||
+      scratch_bytes < dca::select_scratch_bytes(Lk, Hq, n_chunks))
+    return DCA_ERR_WORKSPACE;
+  cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
+  uint8_t* sb = static_cast<uint8_t*>(sparse_ws);
+  uint8_t* base = static_cast<uint8_t*>(workspace);
+  // the head's lists are rewritten; bitmaps start empty
+  if (cudaMemsetAsync(sb + S.vbit_off, 0, S.gk_off - S.vbit_off, st) != cudaSuccess)
+    return DCA_ERR_CUDA;
+  dca::SelectArgs a;
+  a.q = q_block;
+  a.kr = base + L.kr_off;
+  a.tab = reinterpret_cast<const float2*>(base + L.tab_off);
+  a.scratch = scratch;
+  a.q_start = q_start;
+  a.Lq = Lq;
+  a.Lk = Lk;
+  a.s = chunk_size;
+  a.w = local_window;
+  a.tab_c1 = L.T - 1;
+  a.n_chunks = n_chunks;
+  a.n_v = n_vertical;
+  a.n_s = n_slash;
+  a.n_last = n_last;
+  a.Hq = Hq;
+  a.Hkv = Hkv;
+  a.reading = reading;
+  a.continuous = continuous_positions;
+  a.rope_base = rope_base;
+  a.scale_log2 = logit_scale_log2(yarn_scale, d);
+  a.nv = reinterpret_cast<int32_t*>(sb + S.nv_off);
+  a.ns = reinterpret_cast<int32_t*>(sb + S.ns_off);
+  a.vidx = reinterpret_cast<int32_t*>(sb + S.vidx_off);
+  a.soff = reinterpret_cast<int32_t*>(sb + S.soff_off);
+  a.nruns = reinterpret_cast<int32_t*>(sb + S.nruns_off);
+  a.runs = reinterpret_cast<int2*>(sb + S.runs_off);
+  a.vbit = reinterpret_cast<uint32_t*>(sb + S.vbit_off);
+  a.sbit = reinterpret_cast<uint32_t*>(sb + S.sbit_off);
+  a.nv_cap = S.nv_cap;
+  a.s_cap = S.s_cap;
+  a.wpr = S.wpr;
+  cudaError_t e = dca::launch_select(a, st);
+  if (e == cudaSuccess) {
+    const dca::SparseArgs sa = sparse_args(S, sparse_ws);
+    e = dca::launch_sparse_gather(sa.vidx, sa.nv, S.nv_cap, base + L.kr_off, v_cache,
+                                  sb + S.gk_off, sb + S.gv_off, Hq, Hkv, st);
+  }
+  return e == cudaSuccess ? DCA_OK : DCA_ERR_CUDA;
+}
+
+int dca_sparse_pattern_get(const dca_sparse_config* cfg, int Hq, const void* sparse_ws,
+                           size_t sparse_bytes, int32_t* v_counts, int32_t* v_idx,
+                           int32_t* s_counts, int32_t* s_off, void* cuda_stream) {
+  if (!sparse_cfg_ok(cfg) || Hq <= 0 || !v_counts || !s_counts) return DCA_ERR_ARG;
+  if ((cfg->max_vertical > 0 && !v_idx) || (cfg->max_slash > 0 && !s_off)) return DCA_ERR_ARG;
+  if (sparse_ws == nullptr || !aligned(sparse_ws, 1024)) return DCA_ERR_WORKSPACE;
+  const SparseLayout S = make_sparse_layout(cfg, Hq);
+  if (sparse_bytes < S.total) return DCA_ERR_WORKSPACE;
+  cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
+  if (cudaStreamSynchronize(st) != cudaSuccess) return DCA_ERR_CUDA;
+  std::vector<uint8_t> blob(S.host_bytes);
+  if (cudaMemcpy(blob.data(), sparse_ws, S.host_bytes, cudaMemcpyDeviceToHost) != cudaSuccess)
+    return DCA_ERR_CUDA;
+  const int32_t* nv = reinterpret_cast<const int32_t*>(blob.data() + S.nv_off);
+  const int32_t* ns = reinterpret_cast<const int32_t*>(blob.data() + S.ns_off);
+  const int32_t* vi = reinterpret_cast<const int32_t*>(blob.data() + S.vidx_off);
+  const int32_t* so = reinterpret_cast<const int32_t*>(blob.data() + S.soff_off);
+  for (int h = 0; h < Hq; ++h) {
+    v_counts[h] = nv[h];
+    s_counts[h] = ns[h];
+    for (int64_t e = 0; e < nv[h] && e < cfg->max_vertical; ++e)
+      v_idx[h * cfg->max_vertical + e] = vi[h * S.nv_cap + e];
+    for (int64_t e = 0; e < ns[h] && e < cfg->max_slash; ++e)
+      s_off[h * cfg->max_slash + e] = so[h * S.s_cap + e];
+  }
+  return DCA_OK;
 }
 
 }  // extern "C"

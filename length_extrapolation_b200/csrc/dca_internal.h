@@ -68,6 +68,25 @@ struct SparseArgs {
   int64_t wpr, nv_cap;
 };
 
+// Key selection (scores of the last rows, top-k into the sparse workspace).
+struct SelectArgs {
+  const void* q;          // query block [Lq][Hq][128] bf16
+  const void* kr;         // rotated keys [cap][Hkv][128] bf16
+  const float2* tab;      // RoPE table
+  void* scratch;          // select_scratch_bytes(Lk, Hq, n_chunks)
+  int64_t q_start, Lq, Lk, s, w, tab_c1, n_chunks, n_v, n_s;
+  int n_last, Hq, Hkv, reading, continuous;
+  double rope_base;
+  float scale_log2;
+  // outputs in the sparse workspace (bitmaps zeroed before)
+  int32_t *nv, *ns, *vidx, *soff, *nruns;
+  int2* runs;
+  uint32_t *vbit, *sbit;
+  int64_t nv_cap, s_cap, wpr;
+};
+size_t select_scratch_bytes(int64_t Lk, int Hq, int64_t n_chunks);
+cudaError_t launch_select(const SelectArgs& sa, cudaStream_t st);
+
 // bf16 tcgen05/TMA kernel; returns a CUDA error or cudaSuccess, or
 // cudaErrorInvalidValue when a tensor map cannot be encoded.
 cudaError_t launch_attention_sm100(const AttnArgs& a, cudaStream_t st);

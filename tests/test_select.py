@@ -1,0 +1,136 @@
+"""Online key selection for the sparse attention (DCA or continuous positions).
+
+CPU: argument checks of dca_sparse_select.
+GPU: the selected keys and offsets are a top-k of the fp64 oracle's scores
+(vertical column sums and slash diagonal sums of the last rows' softmax);
+where several answers are correct (scores within the rounding of the bf16
+keys of each other) any of them passes, everything else must match.  Then
+the sparse attention over the selected pattern against the oracle.
+"""
+import ctypes
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import length_extrapolation_b200 as dca
+from length_extrapolation_b200 import _native as N
+from length_extrapolation_b200.workloads import Workload, generate
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from length_extrapolation_b200 import build as B
+    B.build()
+    return N.lib()
+
+
+def test_select_rejects(lib):
+    cfg = N.DCASparseConfig(1000, 64, 64)
+    n = lib.dca_sparse_workspace_size(ctypes.byref(cfg), 4)
+    ws = lib.dca_workspace_size(1000, 4, 2, 128, 64, 16, 128, 0)
+    sc = lib.dca_sparse_select_scratch_size(1000, 4, 64)
+    assert sc > 0 and lib.dca_sparse_select_scratch_size(0, 4, 64) == 0
+    p = 1 << 20
+
+    def call(n_last=16, cont=1, nv=8, ns=8, dtype=0, sbytes=sc, Lq=100):
+        return lib.dca_sparse_select(ctypes.byref(cfg), p, p, 900, Lq, 1000, 4, 2, 128, 64, 16,
+                                     128, 1e7, 1.0, dtype, None, n_last, cont, nv, ns, p, ws, p,
+                                     n, p, sbytes, None)
+
+    assert call(n_last=65) == N.DCA_ERR_ARG
+    assert call(n_last=0) == N.DCA_ERR_ARG
+    assert call(cont=2) == N.DCA_ERR_ARG
+    assert call(nv=65) == N.DCA_ERR_ARG                  # more than cfg.max_vertical
+    assert call(dtype=1) == N.DCA_ERR_UNSUPPORTED
+    assert call(sbytes=sc - 1) == N.DCA_ERR_WORKSPACE
+    big = N.DCASparseConfig(1000, 64, 2000)
+    nb = lib.dca_sparse_workspace_size(ctypes.byref(big), 4)
+    assert lib.dca_sparse_select(ctypes.byref(big), p, p, 900, 100, 1000, 4, 2, 128, 64, 16, 128,
+                                 1e7, 1.0, 0, None, 16, 1, 8, 1024, p, ws, p, nb, p, sc,
+                                 None) == N.DCA_ERR_ARG   # n_slash above DCA_SPARSE_MAX_RUNS
+
+
+DEV = "cuda:0"
+
+
+def wl(name, L, Hq, Hkv, s, w, c, yarn=1.0, sqrt_d=False):
+    return Workload(name, L=L, Hq=Hq, Hkv=Hkv, d=128, dtype="bf16", chunk_size=s,
+                    local_window=w, pretrain_window=c, yarn_scale=yarn, scale_by_sqrt_d=sqrt_d)
+
+
+def select_on_gpu(w, n_v, n_s, n_last, continuous, seed=0, q_start=None):
+    q, k, v = generate(w, device=DEV, seed=seed)
+    kw = dict(chunk_size=w.chunk_size, local_window=w.local_window,
+              pretrain_window=w.pretrain_window)
+    ws = dca.Workspace(w.L, w.Hq, w.Hkv, 128, w.chunk_size, w.local_window, w.pretrain_window,
+                       q.dtype, DEV)
+    dca.prepare(k, kv_len=w.L, k_rows_valid=0, rope_base=w.rope_base, workspace=ws, **kw)
+    sp = dca.SparseWorkspace(w.L, w.Hq, max(1, n_v), max(1, n_s), DEV)
+    q0 = 0 if q_start is None else q_start
+    dca.sparse_select(q[q0:], v, q_start=q0, kv_len=w.L, rope_base=w.rope_base,
+                      yarn_scale=w.yarn_scale, n_vertical=n_v, n_slash=n_s, n_last=n_last,
+                      continuous=continuous, workspace=ws, sparse=sp, **kw)
+    V, S = dca.sparse_pattern_get(sp, w.Hq)
+    return q, k, v, ws, sp, V, S
+
+
+def check_topk(sel, score, k, rel=3e-3):
+    """`sel` is a valid top-k of `score` up to ties within the tolerance."""
+    sel = np.asarray(sel)
+    assert len(sel) == k and np.all(np.diff(sel) > 0)
+    if k == 0:
+        return
+    thr = np.sort(score)[-k]
+    tol = rel * max(thr, 1e-12) + 1e-7
+    chosen = np.zeros(score.size, bool)
+    chosen[sel] = True
+    assert np.all(score[chosen] >= thr - tol), (score[chosen].min(), thr)
+    assert np.all(score[~chosen] <= thr + tol), (score[~chosen].max(), thr)
+
+
+CASES = [  # workload, n_vertical, n_slash, n_last
+    (wl("sel_mixed", 2000, 4, 2, 512, 64, 1024, yarn=2.0), 100, 60, 64),
+    (wl("sel_one_chunk", 900, 2, 1, 1024, 64, 2048), 50, 30, 32),
+    (wl("sel_small_chunks", 1500, 3, 1, 200, 50, 300), 300, 200, 64),
+    (wl("sel_g7", 3000, 7, 1, 1024, 128, 2048, sqrt_d=True), 128, 512, 64),
+]
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("continuous", [True, False], ids=["continuous", "dca"])
+@pytest.mark.parametrize("w,nv,ns,nl", CASES, ids=lambda x: getattr(x, "name", ""))
+def test_selection_is_a_topk_of_the_oracle_scores(w, nv, ns, nl, continuous):
+    q, k, v, ws, sp, V, S = select_on_gpu(w, nv, ns, nl, continuous)
+    vert, slash = oracle.vs_scores(q.cpu(), k.cpu(), n_last=nl, continuous=continuous,
+                                   **w.params())
+    for h in range(w.Hq):
+        check_topk(V[h], vert[h], min(nv, w.L))
+        check_topk(S[h], slash[h], min(ns, w.L))
+
+
+@pytest.mark.gpu
+def test_selected_pattern_attention_matches_oracle():
+    from tests.gpu_helpers import assert_close
+    w = wl("sel_e2e", 2500, 4, 2, 512, 64, 1024, yarn=2.0, sqrt_d=True)
+    q, k, v, ws, sp, V, S = select_on_gpu(w, 120, 400, 64, True, seed=4)
+    kw = dict(chunk_size=w.chunk_size, local_window=w.local_window,
+              pretrain_window=w.pretrain_window)
+    out = dca.sparse_attend(q, v, q_start=0, kv_len=w.L, yarn_scale=w.yarn_scale, workspace=ws,
+                            sparse=sp, **kw)
+    torch.cuda.synchronize()
+    assert ws.status() == N.DCA_OK
+    want = oracle.sparse_attention(q.cpu(), k.cpu(), v.cpu(), vertical=V, slash=S, **w.params())
+    assert_close(out.double().cpu().numpy(), want, torch.bfloat16, "selected pattern")
+
+
+@pytest.mark.gpu
+def test_continuous_and_dca_selections_differ_across_chunks():
+    """Several chunks: the true-position estimate selects other keys than the
+    DCA estimate (the motivation of the refinement)."""
+    w = wl("sel_modes", 2048, 2, 1, 256, 32, 512)
+    a = select_on_gpu(w, 64, 64, 64, True)
+    b = select_on_gpu(w, 64, 64, 64, False)
+    diff = sum(len(set(x.tolist()) ^ set(y.tolist())) for x, y in zip(a[5] + a[6], b[5] + b[6]))
+    assert diff > 0
