@@ -668,6 +668,36 @@ def run_sparse_bench(args, sw, world, rank, local, dist):
         "traffic": None, "launches_per_step": len(blocks),
         "avg_launch_ms": attn_ms / (args.steps * len(blocks)),
     }
+    # the online key selection (continuous positions) of the last block, timed alone
+    q0, lq, lk = blocks[-1]
+    n_s = min(sw.n_band + sw.n_far, N.DCA_SPARSE_MAX_RUNS)
+    sel_sp = dca.SparseWorkspace(w.L, w.Hq, sw.n_vertical, n_s, dev)
+    sel_scratch = torch.empty(N.lib().dca_sparse_select_scratch_size(lk, w.Hq, w.chunk_size),
+                              dtype=torch.uint8, device=dev)
+
+    def select():
+        dca.sparse_select(q[q0:q0 + lq], v, q_start=q0, kv_len=lk, rope_base=w.rope_base,
+                          yarn_scale=w.yarn_scale, n_vertical=sw.n_vertical, n_slash=n_s,
+                          n_last=64, continuous=True, workspace=ws, sparse=sel_sp,
+                          scratch=sel_scratch, **kw)
+
+    select()
+    torch.cuda.synchronize()
+    s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s0.record()
+    for _ in range(3):
+        select()
+    s1.record()
+    torch.cuda.synchronize()
+    sel_ms = s0.elapsed_time(s1) / 3
+    sel_flops = 2 * 2.0 * 64 * lk * w.Hq * w.d  # two score passes, 2 FLOP per multiply-add
+    alu_peak = 148 * 128 * 2 * (clk.get("sm_mhz") or 1965.0) * 1e6 / 1e12
+    select_info = {"kv_len": lk, "n_last": 64, "n_vertical": sw.n_vertical, "n_slash": n_s,
+                   "positions": "continuous", "ms": sel_ms,
+                   "score_tflops": sel_flops / (sel_ms / 1e3) / 1e12,
+                   "roofline": {"bound": "alu", "peak": alu_peak, "unit": "TFLOP/s",
+                                "frac": sel_flops / (sel_ms / 1e3) / 1e12 / alu_peak,
+                                "peak_kind": "FP32 FMA: 148 SMs x 128 lanes x 2 x median SM clock"}}
     line = {
         "metric": SPARSE_METRIC, "value": whole_job_rate(w.L, world, ms_per_step), "unit": UNIT,
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
@@ -676,6 +706,7 @@ def run_sparse_bench(args, sw, world, rank, local, dist):
         "config": {**sparse_config(sw), "parallelism": f"replicas x{world}" if world > 1 else "1 GPU"},
         "tflops_member_pairs": world * flops / (ms_per_step / 1e3) / 1e12,
         "roofline": roofline, "e2e": None, "cpu_baseline": cpu, "clocks": clk,
+        "select": select_info,
         "gpu_launches": args.steps * len(blocks) * 5,  # rotate, 2 prep kernels, attend (+ memset)
         "peaks_source": peaks["source"],
     }

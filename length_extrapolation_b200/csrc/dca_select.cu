@@ -24,6 +24,7 @@
 
 #include "dca_internal.h"
 #include "dca_plan.cuh"
+#include "sm100_ptx.cuh"
 
 namespace dca {
 namespace sel {
@@ -32,8 +33,6 @@ constexpr int ROWS = 64;     // rows of the estimate (max)
 constexpr int KT = 128;      // keys per tile
 constexpr int HD = 128;
 constexpr int THREADS = 256;
-constexpr int QPAD = HD + 4; // padded query row (floats)
-constexpr int KPAD = HD + 1; // padded key row (floats): conflict-free column reads
 constexpr int OBINS = ROWS + KT;  // distinct offsets i - j of one tile
 
 struct ScoreParams {
@@ -56,24 +55,30 @@ __device__ __forceinline__ int variant(const ScoreParams& p, int64_t i, int64_t 
   return pair_class(ni - nj, i - j, p.w, p.reading);
 }
 
+constexpr int KTP = KT + 4;    // padded key count of a dim-major key row
+constexpr int RP = ROWS + 4;   // padded row count of a dim-major query row
+
+// One CTA per (key tile, KV group): the tile's keys are loaded once (fp32,
+// dim-major; continuous positions: rotated from j mod s to j) and serve the
+// group's G query heads in turn.  Thread (ty, tx) owns rows 4ty..4ty+3 and
+// keys 8tx..8tx+7: per dim one 16-byte load of the rows, two of the keys, 16
+// packed FMAs.
 template <bool PASS2>
 __global__ void __launch_bounds__(THREADS)
     sel_score_kernel(const ScoreParams p) {
   extern __shared__ float sm[];
-  float* Ks = sm;                       // [KT][KPAD]
-  float* Qs = Ks + KT * KPAD;           // [nvar][ROWS][QPAD]
+  float* Kt = sm;                       // [HD][KTP]
+  float* Qt = Kt + HD * KTP;            // [nvar][HD][RP] (current head)
   __shared__ float colsum[16][KT];
   __shared__ float obin[OBINS];
   __shared__ float2 st[ROWS];
 
   const int tile = blockIdx.x;
-  const int h = blockIdx.y;
-  const int g = h / p.G;
+  const int g = blockIdx.y;
   const int64_t j0 = static_cast<int64_t>(tile) * KT;
   const int t = threadIdx.x;
-  const int ty = t >> 4, tx = t & 15;   // rows 4ty..4ty+3, keys tx + 16u
+  const int ty = t >> 4, tx = t & 15;
 
-  // keys (fp32; continuous: rotated from j mod s to j by the chunk's s*n*theta)
   for (int idx = t; idx < KT * (HD / 2); idx += THREADS) {
     const int r = idx / (HD / 2), k = idx % (HD / 2);
     const int64_t j = j0 + r;
@@ -89,132 +94,155 @@ __global__ void __launch_bounds__(THREADS)
         b = rb;
       }
     }
-    Ks[r * KPAD + k] = a;
-    Ks[r * KPAD + k + HD / 2] = b;
+    Kt[k * KTP + r] = a;
+    Kt[(k + HD / 2) * KTP + r] = b;
   }
-  for (int idx = t; idx < p.nvar * ROWS * HD; idx += THREADS) {
-    const int v = idx / (ROWS * HD), rem = idx % (ROWS * HD);
-    const int r = rem / HD, k = rem % HD;
-    Qs[(v * ROWS + r) * QPAD + k] =
-        p.qv[((static_cast<int64_t>(h) * p.nvar + v) * ROWS + r) * HD + k];
-  }
-  if (PASS2) {
-    for (int o = t; o < OBINS; o += THREADS) obin[o] = 0.f;
-    for (int r = t; r < ROWS; r += THREADS) st[r] = p.stats[h * ROWS + r];
-  }
-  __syncthreads();
 
-  // logits (log2 units) of rows 4ty..+3 x keys tx + 16u, variant by variant
-  int64_t nrow[4], nkey[8];
+  // the variant of each of this thread's pairs (-1: not a causal pair of the
+  // estimate) -- the same for every head of the group -- and the variants
+  // present in the tile
+  int8_t var[4][8];
+  {
+    int64_t nkey[8];
 #pragma unroll
-  for (int a = 0; a < 4; ++a) nrow[a] = (p.i_first + 4 * ty + a) / p.s;
-#pragma unroll
-  for (int u = 0; u < 8; ++u) nkey[u] = (j0 + tx + 16 * u) / p.s;
-  float x[4][8];
-#pragma unroll
-  for (int a = 0; a < 4; ++a)
-#pragma unroll
-    for (int u = 0; u < 8; ++u) x[a][u] = -INFINITY;
-  for (int v = 0; v < p.nvar; ++v) {
-    bool any = false;
+    for (int u = 0; u < 8; ++u) nkey[u] = (j0 + 8 * tx + u) / p.s;
 #pragma unroll
     for (int a = 0; a < 4; ++a) {
       const int r = 4 * ty + a;
       const int64_t i = p.i_first + r;
+      const int64_t ni = i / p.s;
 #pragma unroll
       for (int u = 0; u < 8; ++u) {
-        const int64_t j = j0 + tx + 16 * u;
-        any |= (r < p.n_last && j <= i && j < p.Lk && variant(p, i, nrow[a], j, nkey[u]) == v);
+        const int64_t j = j0 + 8 * tx + u;
+        var[a][u] = (r < p.n_last && j <= i && j < p.Lk)
+                        ? static_cast<int8_t>(variant(p, i, ni, j, nkey[u]))
+                        : static_cast<int8_t>(-1);
       }
     }
-    if (!__syncthreads_or(any)) continue;
-    float acc[4][8];
+  }
+  bool present[3];
+  for (int v = 0; v < 3; ++v) {
+    bool any = false;
 #pragma unroll
     for (int a = 0; a < 4; ++a)
 #pragma unroll
-      for (int u = 0; u < 8; ++u) acc[a][u] = 0.f;
-#pragma unroll 4
-    for (int k = 0; k < HD; ++k) {
-      float qa[4], kb[8];
+      for (int u = 0; u < 8; ++u) any |= var[a][u] == v;
+    present[v] = __syncthreads_or(any) != 0;
+  }
+
+  for (int hh = 0; hh < p.G; ++hh) {
+    const int h = g * p.G + hh;
+    __syncthreads();  // the previous head is done with Qt, obin, colsum
+    for (int v = 0; v < p.nvar; ++v) {
+      if (!present[v]) continue;
+      const float* src = p.qv + (static_cast<int64_t>(h) * p.nvar + v) * ROWS * HD;
+      for (int idx = t; idx < ROWS * HD; idx += THREADS) {
+        const int r = idx / HD, k = idx % HD;
+        Qt[(v * HD + k) * RP + r] = src[idx];
+      }
+    }
+    if (PASS2) {
+      for (int o = t; o < OBINS; o += THREADS) obin[o] = 0.f;
+      for (int r = t; r < ROWS; r += THREADS) st[r] = p.stats[h * ROWS + r];
+    }
+    __syncthreads();
+
+    float x[4][8];
 #pragma unroll
-      for (int a = 0; a < 4; ++a) qa[a] = Qs[(v * ROWS + 4 * ty + a) * QPAD + k];
+    for (int a = 0; a < 4; ++a)
 #pragma unroll
-      for (int u = 0; u < 8; ++u) kb[u] = Ks[(tx + 16 * u) * KPAD + k];
+      for (int u = 0; u < 8; ++u) x[a][u] = -INFINITY;
+    for (int v = 0; v < p.nvar; ++v) {
+      if (!present[v]) continue;
+      float2 acc[4][4];
 #pragma unroll
       for (int a = 0; a < 4; ++a)
 #pragma unroll
-        for (int u = 0; u < 8; ++u) acc[a][u] = fmaf(qa[a], kb[u], acc[a][u]);
+        for (int u = 0; u < 4; ++u) acc[a][u] = make_float2(0.f, 0.f);
+      const float* qb = Qt + v * HD * RP + 4 * ty;
+      const float* kb = Kt + 8 * tx;
+#pragma unroll 4
+      for (int k = 0; k < HD; ++k) {
+        const float4 q4 = *reinterpret_cast<const float4*>(qb + k * RP);
+        const float4 k0 = *reinterpret_cast<const float4*>(kb + k * KTP);
+        const float4 k1 = *reinterpret_cast<const float4*>(kb + k * KTP + 4);
+        const float2 kk[4] = {make_float2(k0.x, k0.y), make_float2(k0.z, k0.w),
+                              make_float2(k1.x, k1.y), make_float2(k1.z, k1.w)};
+        const float qq[4] = {q4.x, q4.y, q4.z, q4.w};
+#pragma unroll
+        for (int a = 0; a < 4; ++a)
+#pragma unroll
+          for (int u = 0; u < 4; ++u) acc[a][u] = fma2(make_float2(qq[a], qq[a]), kk[u], acc[a][u]);
+      }
+#pragma unroll
+      for (int a = 0; a < 4; ++a)
+#pragma unroll
+        for (int u = 0; u < 8; ++u)
+          if (var[a][u] == v) x[a][u] = (u & 1) ? acc[a][u >> 1].y : acc[a][u >> 1].x;
     }
+
+    if (!PASS2) {
+      // per row: tile max and sum of 2^(x - max) over the 16 threads of the row group
+#pragma unroll
+      for (int a = 0; a < 4; ++a) {
+        float m = x[a][0];
+#pragma unroll
+        for (int u = 1; u < 8; ++u) m = fmaxf(m, x[a][u]);
+#pragma unroll
+        for (int off = 8; off >= 1; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+        float l = 0.f;
+        if (m != -INFINITY) {
+#pragma unroll
+          for (int u = 0; u < 8; ++u) l += exp2f(x[a][u] - m);
+        }
+#pragma unroll
+        for (int off = 8; off >= 1; off >>= 1) l += __shfl_xor_sync(0xffffffffu, l, off);
+        if (tx == 0) {
+          const int r = 4 * ty + a;
+          p.part[(static_cast<int64_t>(h) * p.n_tiles + tile) * ROWS + r] = make_float2(m, l);
+        }
+      }
+      continue;
+    }
+
+    // pass 2: probabilities; column sums (vertical) and diagonal sums (slash)
+    float cs[8], dg[11];  // column sums; sums along this thread's 11 diagonals a - u
+#pragma unroll
+    for (int u = 0; u < 8; ++u) cs[u] = 0.f;
+#pragma unroll
+    for (int e = 0; e < 11; ++e) dg[e] = 0.f;
 #pragma unroll
     for (int a = 0; a < 4; ++a) {
       const int r = 4 * ty + a;
-      const int64_t i = p.i_first + r;
+      const float2 rs = st[r];
+      const float inv = rs.y > 0.f ? 1.f / rs.y : 0.f;
 #pragma unroll
       for (int u = 0; u < 8; ++u) {
-        const int64_t j = j0 + tx + 16 * u;
-        if (r < p.n_last && j <= i && j < p.Lk && variant(p, i, nrow[a], j, nkey[u]) == v)
-          x[a][u] = acc[a][u];
+        const float pr = x[a][u] == -INFINITY ? 0.f : exp2f(x[a][u] - rs.x) * inv;
+        cs[u] += pr;
+        dg[a - u + 7] += pr;
       }
     }
-  }
-
-  if (!PASS2) {
-    // per row: tile max and sum of 2^(x - max) over the 16 threads of the row group
+    // offset o = (i_first + 4ty + a) - (j0 + 8tx + u); bin = o - (i_first - j0 - KT + 1)
 #pragma unroll
-    for (int a = 0; a < 4; ++a) {
-      float m = x[a][0];
+    for (int e = 0; e < 11; ++e)
+      if (dg[e] != 0.f) atomicAdd(&obin[4 * ty - 8 * tx + (e - 7) + KT - 1], dg[e]);
 #pragma unroll
-      for (int u = 1; u < 8; ++u) m = fmaxf(m, x[a][u]);
+    for (int u = 0; u < 8; ++u) colsum[ty][8 * tx + u] = cs[u];
+    __syncthreads();
+    if (t < KT) {
+      float v = 0.f;
 #pragma unroll
-      for (int off = 8; off >= 1; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
-      float l = 0.f;
-      if (m != -INFINITY) {
-#pragma unroll
-        for (int u = 0; u < 8; ++u) l += exp2f(x[a][u] - m);
-      }
-#pragma unroll
-      for (int off = 8; off >= 1; off >>= 1) l += __shfl_xor_sync(0xffffffffu, l, off);
-      if (tx == 0) {
-        const int r = 4 * ty + a;
-        p.part[(static_cast<int64_t>(h) * p.n_tiles + tile) * ROWS + r] = make_float2(m, l);
-      }
+      for (int y = 0; y < 16; ++y) v += colsum[y][t];
+      const int64_t j = j0 + t;
+      if (j < p.Lk) p.vert[static_cast<int64_t>(h) * p.Lk + j] = v;
     }
-    return;
-  }
-
-  // pass 2: probabilities; column sums (vertical) and diagonal sums (slash)
-  float cs[8];
-#pragma unroll
-  for (int u = 0; u < 8; ++u) cs[u] = 0.f;
-#pragma unroll
-  for (int a = 0; a < 4; ++a) {
-    const int r = 4 * ty + a;
-    const float2 rs = st[r];
-    const float inv = rs.y > 0.f ? 1.f / rs.y : 0.f;
-#pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      if (x[a][u] == -INFINITY) continue;
-      const float pr = exp2f(x[a][u] - rs.x) * inv;
-      cs[u] += pr;
-      // offset o = i - j = (i_first + r) - (j0 + key); bin = o - (i_first - j0 - KT + 1)
-      const int bin = r - (tx + 16 * u) + KT - 1;
-      atomicAdd(&obin[bin], pr);
+    for (int b = t; b < OBINS; b += THREADS) {
+      const float v = obin[b];
+      const int64_t o = (p.i_first - j0 - KT + 1) + b;
+      if (v != 0.f && o >= 0 && o < p.Lk)
+        atomicAdd(&p.slash[static_cast<int64_t>(h) * p.Lk + o], v);
     }
-  }
-#pragma unroll
-  for (int u = 0; u < 8; ++u) colsum[ty][tx + 16 * u] = cs[u];
-  __syncthreads();
-  if (t < KT) {
-    float v = 0.f;
-#pragma unroll
-    for (int y = 0; y < 16; ++y) v += colsum[y][t];
-    const int64_t j = j0 + t;
-    if (j < p.Lk) p.vert[static_cast<int64_t>(h) * p.Lk + j] = v;
-  }
-  for (int b = t; b < OBINS; b += THREADS) {
-    const float v = obin[b];
-    const int64_t o = (p.i_first - j0 - KT + 1) + b;
-    if (v != 0.f && o >= 0 && o < p.Lk) atomicAdd(&p.slash[static_cast<int64_t>(h) * p.Lk + o], v);
   }
 }
 
@@ -355,10 +383,17 @@ __global__ void __launch_bounds__(1024)
     for (int b = tid; b < nb; b += 1024) hist[b] = 0;
     __syncthreads();
     const int top = pass == 0 ? 32 : shifts[pass - 1];
-    for (int64_t j = tid; j < Lk; j += 1024) {
-      const uint32_t bits = __float_as_uint(sc[j]);
-      if (pass > 0 && (bits >> top) != prefix) continue;
-      atomicAdd(&hist[(bits >> shifts[pass]) & (nb - 1)], 1);
+    const int lane = tid & 31;
+    for (int64_t base = 0; base < Lk; base += 1024) {
+      // lanes with the same bin add once (scores crowd into a few bins)
+      const int64_t j = base + tid;
+      int bin = -1;
+      if (j < Lk) {
+        const uint32_t bits = __float_as_uint(sc[j]);
+        if (pass == 0 || (bits >> top) == prefix) bin = static_cast<int>((bits >> shifts[pass]) & (nb - 1));
+      }
+      const unsigned peers = __match_any_sync(0xffffffffu, bin);
+      if (bin >= 0 && lane == __ffs(peers) - 1) atomicAdd(&hist[bin], __popc(peers));
     }
     __syncthreads();
     if (tid == 0) {
@@ -483,8 +518,8 @@ cudaError_t launch_select(const SelectArgs& sa, cudaStream_t st) {
   p.n_tiles = static_cast<int>(n_tiles);
   p.reading = sa.reading;
   p.continuous = sa.continuous;
-  const size_t smem = sizeof(float) * (KT * KPAD + nvar * ROWS * QPAD);
-  const dim3 grid(static_cast<unsigned>(n_tiles), static_cast<unsigned>(sa.Hq));
+  const size_t smem = sizeof(float) * (HD * KTP + nvar * HD * RP);
+  const dim3 grid(static_cast<unsigned>(n_tiles), static_cast<unsigned>(sa.Hkv));
   if ((e = cudaFuncSetAttribute(sel_score_kernel<false>,
                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 static_cast<int>(smem))) != cudaSuccess)
