@@ -187,12 +187,22 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   // ---- work unit
   // KV-group-major order: the CTAs running together stream the same group's
   // K'/V tiles (shared in L2); within a group, longest query tiles first.
+  // Within a group the CTAs with two heads come first and a lone head (odd
+  // G) after them: CTAs with equal work run side by side and stay in step
+  // along the key stream, so the tiles they read are still in L2.
   const int per_group = p.n_qtiles * p.n_pairs;
-  const int u = (static_cast<int>(blockIdx.x) / per_group) * p.n_pairs +
-                static_cast<int>(blockIdx.x % per_group) % p.n_pairs;
-  const int qt = p.n_qtiles - 1 - static_cast<int>((blockIdx.x % per_group) / p.n_pairs);
-  const int g = u / p.n_pairs;
-  const int pr = u % p.n_pairs;
+  const int g = static_cast<int>(blockIdx.x) / per_group;
+  const int c = static_cast<int>(blockIdx.x) % per_group;
+  const int n_two = p.G / 2;  // pairs with two heads
+  int qt_idx, pr;
+  if (c < p.n_qtiles * n_two) {
+    qt_idx = c / n_two;
+    pr = c % n_two;
+  } else {
+    qt_idx = c - p.n_qtiles * n_two;
+    pr = n_two;
+  }
+  const int qt = p.n_qtiles - 1 - qt_idx;
   const int h0 = g * p.G + 2 * pr;
   const bool two = (2 * pr + 1) < p.G;
   const int64_t i0 = p.q_start + static_cast<int64_t>(qt) * BM;
