@@ -84,6 +84,7 @@ def load_peaks():
 
 
 KERNEL_SOURCES = ["length_extrapolation_b200/csrc/dca_fwd_sm100.cu",
+                  "length_extrapolation_b200/csrc/dca_softmax.cuh",
                   "length_extrapolation_b200/csrc/sm100_ptx.cuh",
                   "length_extrapolation_b200/csrc/dca_plan.cuh"]
 TRAFFIC_RECORD = os.path.join(ROOT, "profiles", "dca_fwd_kernel_traffic.json")
