@@ -275,11 +275,12 @@ int dca_sparse_pattern_get(const dca_sparse_config* cfg, int Hq, const void* spa
  * Host-side introspection of the sparse kernel's work list (no GPU needed):
  * for the query tile whose rows are [i0, i0 + 128) (i0 a multiple of 128) with
  * real rows up to i_last, and one head's sorted vertical keys / slash offsets
- * (host arrays), writes up to max_items triples (src, tile, class): src 0 = a
- * 128-key tile of the head's gathered vertical keys (list positions
- * 128*tile ..), src 1 = cache k-tile `tile` crossed by a slash diagonal or by
- * the diagonal j = i; class as in dca_plan_items.  Returns the number of
- * items (which may exceed max_items) or DCA_ERR_ARG.
+ * (host arrays), writes up to max_items triples (src, start, class): src 0 =
+ * the 128 gathered vertical keys at list positions start .. start + 127
+ * (start a multiple of 128), src 1 = the 128 cache keys start .. start + 127,
+ * a window over what the slash diagonals and the diagonal j = i reach from
+ * the tile's rows; class as in dca_plan_items.  Returns the number of items
+ * (which may exceed max_items) or DCA_ERR_ARG.
  */
 int dca_sparse_plan_items(const int32_t* v_idx, int64_t n_v, const int32_t* s_off, int64_t n_s,
                           int64_t i0, int64_t i_last, int64_t chunk_size, int64_t local_window,

@@ -648,11 +648,11 @@ int dca_sparse_plan_items(const int32_t* v_idx, int64_t n_v, const int32_t* s_of
                          i_last, chunk_size, local_window, window_reading, 128);
   dca::SparseIter it;
   dca::sparse_iter_init(it);
-  int n = 0, src, tile, cls;
-  while (dca::sparse_iter_next(it, P[0], src, tile, cls)) {
+  int n = 0, src, start, cls;
+  while (dca::sparse_iter_next(it, P[0], src, start, cls)) {
     if (n < max_items) {
       items[3 * n] = src;
-      items[3 * n + 1] = tile;
+      items[3 * n + 1] = start;
       items[3 * n + 2] = cls;
     }
     ++n;

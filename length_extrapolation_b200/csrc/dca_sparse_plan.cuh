@@ -2,12 +2,18 @@
 // head) of the vertical-slash sparse attention, shared by the kernel (which
 // keeps the plan in shared memory) and the host introspection entry point.
 //
-// Items are 128-key tiles, visited class by class (INTER, SUCC, INTRA; see
-// dca_plan.cuh); within a class first the tiles of the head's gathered
-// vertical keys whose positions fall in the class's key range, then the
-// cache k-tiles that a slash diagonal (or the diagonal j = i) crosses for some
-// row of the tile, clipped to the class's k-tile range.  A tile shared by two
-// classes appears once per class; the kernel masks each item to its class.
+// Items are windows of 128 keys, visited class by class (INTER, SUCC, INTRA;
+// see dca_plan.cuh); within a class first the 128-position tiles of the
+// head's gathered vertical keys whose positions fall in the class's key
+// range, then windows of cache keys covering what the slash diagonals (and
+// the diagonal j = i) reach from the rows of the tile: each run of slash
+// offsets reaches one contiguous key range, the ranges are merged, and each
+// merged range, clipped to the class's key range, is covered by windows that
+// start at its first key (not at a tile boundary: a lone far diagonal reaches
+// 128 keys, one window).  Ranges closer than 128 keys are merged, so a
+// window that runs past the end of its range never reaches the next one.  A
+// key shared by two classes is visited once per class; the kernel masks each
+// item to its class and its member pairs.
 #pragma once
 #include <stdint.h>
 #include <vector_types.h>
@@ -23,10 +29,10 @@ struct SparsePlan {
   int n_iv;            // merged slash key-tile intervals
   int nv_eff;          // vertical keys <= the tile's last row
   int vt[3][2];        // vertical (gathered) tile range per class (indexed by CLS_*)
-  int ktr[3][2];       // cache k-tile range per class
+  int kr[3][2];        // cache key range [lo, hi) per class
   int qbuf_of[3];      // query operand tile of each class, -1 if absent
   int third_cls;       // class that reuses operand tile 0 (-1 if fewer than three)
-  int2 iv[SPARSE_IV_MAX];  // [x, y) k-tile intervals, ascending
+  int2 iv[SPARSE_IV_MAX];  // [x, y) key ranges reached by the slashes, ascending
 };
 
 DCA_HD int sparse_class_at(int ci) {  // visiting order INTER, SUCC, INTRA
@@ -35,8 +41,8 @@ DCA_HD int sparse_class_at(int ci) {  // visiting order INTER, SUCC, INTRA
 
 struct SparseIter {
   int ci, phase;  // class index in visiting order; -1 start, 0 vertical, 1 slash
-  int t, t_end;   // current tile and the end of the current range
-  int iv;         // slash interval index
+  int t, t_end;   // start of the next item and the end of the current range
+  int iv;         // slash range index
 };
 
 DCA_HD void sparse_iter_init(SparseIter& it) {
@@ -46,18 +52,21 @@ DCA_HD void sparse_iter_init(SparseIter& it) {
   it.iv = 0;
 }
 
-// Next item: src 0 = vertical (gathered tile index), 1 = slash (cache k-tile).
-DCA_HD bool sparse_iter_next(SparseIter& it, const SparsePlan& P, int& src, int& tile, int& cls) {
+// Next item: src 0 = vertical, `start` = first position in the gathered
+// keys (a multiple of 128); src 1 = slash, `start` = first cache key of the
+// 128-key window.
+DCA_HD bool sparse_iter_next(SparseIter& it, const SparsePlan& P, int& src, int& start, int& cls) {
   for (;;) {
     if (it.phase >= 0 && it.t < it.t_end) {
       src = it.phase;
-      tile = it.t++;
+      start = it.t;
+      it.t += 128;
       cls = sparse_class_at(it.ci);
       return true;
     }
     if (it.phase == 1) {
       const int c = sparse_class_at(it.ci);
-      const int clo = P.ktr[c][0], chi = P.ktr[c][1];
+      const int clo = P.kr[c][0], chi = P.kr[c][1];
       while (it.iv < P.n_iv) {
         const int2 r = P.iv[it.iv];
         if (r.x >= chi) break;
@@ -78,14 +87,14 @@ DCA_HD bool sparse_iter_next(SparseIter& it, const SparsePlan& P, int& src, int&
     const int c = sparse_class_at(it.ci);
     if (it.phase == -1) {
       it.phase = 0;
-      it.t = P.vt[c][0];
-      it.t_end = P.vt[c][1];
+      it.t = P.vt[c][0] * 128;
+      it.t_end = P.vt[c][1] * 128;
       continue;
     }
-    // vertical tiles done: slash intervals from the first that reaches the class
+    // vertical tiles done: slash ranges from the first that reaches the class
     it.phase = 1;
     it.iv = 0;
-    while (it.iv < P.n_iv && P.iv[it.iv].y <= P.ktr[c][0]) ++it.iv;
+    while (it.iv < P.n_iv && P.iv[it.iv].y <= P.kr[c][0]) ++it.iv;
     it.t = it.t_end = 0;
   }
 }
@@ -99,8 +108,8 @@ DCA_HD void sparse_plan_build(SparsePlan& P, const int32_t* vk, int nvh, const i
   int64_t klo[3], khi[3];
   class_key_ranges(i0, i_last, s, w, reading, klo, khi);
   for (int c = 0; c < 3; ++c) {
-    P.ktr[c][0] = static_cast<int>(klo[c] / bn);
-    P.ktr[c][1] = khi[c] > klo[c] ? static_cast<int>(cdiv64(khi[c], bn)) : P.ktr[c][0];
+    P.kr[c][0] = static_cast<int>(klo[c]);
+    P.kr[c][1] = static_cast<int>(khi[c] > klo[c] ? khi[c] : klo[c]);
   }
   // vertical tile ranges per class: positions of the class's key range
   auto lower = [&](int64_t key) {
@@ -122,8 +131,8 @@ DCA_HD void sparse_plan_build(SparsePlan& P, const int32_t* vk, int nvh, const i
     P.vt[c][0] = a / bn;
     P.vt[c][1] = b > a ? (b + bn - 1) / bn : a / bn;
   }
-  // slash intervals: runs from the largest offsets down (ascending keys),
-  // the diagonal j = i always included, merged
+  // slash key ranges: runs from the largest offsets down (ascending keys),
+  // the diagonal j = i always included; ranges closer than bn keys merged
   int n_iv = 0;
   for (int r = nr; r >= 0; --r) {
     int64_t oa, ob;
@@ -137,9 +146,8 @@ DCA_HD void sparse_plan_build(SparsePlan& P, const int32_t* vk, int nvh, const i
     if (oa > i_last) continue;
     int64_t ka = i0 - (ob - 1);
     if (ka < 0) ka = 0;
-    const int64_t kb = i_last - oa;
-    const int ta = static_cast<int>(ka / bn), tb = static_cast<int>(kb / bn) + 1;
-    if (n_iv > 0 && ta <= P.iv[n_iv - 1].y) {
+    const int ta = static_cast<int>(ka), tb = static_cast<int>(i_last - oa + 1);
+    if (n_iv > 0 && ta < P.iv[n_iv - 1].y + bn) {
       if (tb > P.iv[n_iv - 1].y) P.iv[n_iv - 1].y = tb;
       if (ta < P.iv[n_iv - 1].x) P.iv[n_iv - 1].x = ta;
     } else {
@@ -154,8 +162,8 @@ DCA_HD void sparse_plan_build(SparsePlan& P, const int32_t* vk, int nvh, const i
   P.third_cls = -1;
   SparseIter it;
   sparse_iter_init(it);
-  int n_items = 0, src, tile, cls, seen = 0;
-  while (sparse_iter_next(it, P, src, tile, cls)) {
+  int n_items = 0, src, start, cls, seen = 0;
+  while (sparse_iter_next(it, P, src, start, cls)) {
     if (P.qbuf_of[cls] < 0) {
       P.qbuf_of[cls] = seen & 1;
       if (seen == 2) P.third_cls = cls;

@@ -16,12 +16,12 @@
 //   vertical items  tiles of the head's gathered vertical keys (rotated keys
 //                   and values copied into a compact [n][Hq][128] array by
 //                   the preparation kernels), masked to j <= i and the class;
-//   slash items     K'/V tiles of the cache that a slash diagonal (or the
-//                   diagonal j = i) crosses for some row of the tile, masked
-//                   per element to the member pairs not already counted as
-//                   vertical, and to the class.
-// The slash tiles come from the head's runs of consecutive offsets, merged
-// into key-tile intervals once per CTA in shared memory.
+//   slash items     windows of 128 cache keys covering what the slash
+//                   diagonals (and the diagonal j = i) reach from the rows of
+//                   the tile, masked per element to the member pairs not
+//                   already counted as vertical, and to the class.
+// The slash windows come from the head's runs of consecutive offsets, merged
+// into key ranges once per CTA in shared memory (dca_sparse_plan.cuh).
 //
 // Warp roles as in the dense kernel (320 threads): warps 0-7 softmax (warp w
 // and w+4 split each row's 128 keys), warp 8 TMA producer (4-slot K/V ring,
@@ -126,7 +126,7 @@ __device__ __forceinline__ bool all_bits(const uint32_t* row, int64_t lo, int64_
 // first 64 columns of the S buffer), O rescaled when the reference moves
 // (after the previous item's P.V completed).
 __device__ __forceinline__ bool sparse_half_step(
-    uint32_t tS, uint32_t tO, int n, bool full, int src, int tile, int cls, int64_t i,
+    uint32_t tS, uint32_t tO, int n, bool full, int src, int start, int cls, int64_t i,
     const Params& p, int h, float sc, int64_t nb, int64_t pb, float& m_ref, float& l_sum,
     PairCtx& pc, SmemCtl* ctl, volatile int* abort, unsigned int* status) {
   const int half = pc.half;
@@ -135,7 +135,7 @@ __device__ __forceinline__ bool sparse_half_step(
   if (!full) {
     const uint32_t NEG_INF = 0xff800000u;
     if (src == 1) {
-      const int64_t j0 = static_cast<int64_t>(tile) * BN + 64 * half;
+      const int64_t j0 = start + 64 * half;  // first key of the window
       mask_cols<64>(sv, i, j0, cls, p.s, p.w, p.reading);
       const uint32_t* vrow = p.vbit + static_cast<int64_t>(h) * p.wpr;
       const uint32_t* srow = p.sbit + static_cast<int64_t>(h) * p.wpr;
@@ -148,7 +148,7 @@ __device__ __forceinline__ bool sparse_half_step(
       for (int e = 0; e < 64; ++e)
         if (!((mem >> e) & 1ull)) sv[e] = NEG_INF;
     } else {
-      const int64_t pos0 = static_cast<int64_t>(tile) * BN + 64 * half;
+      const int64_t pos0 = start + 64 * half;  // first gathered position
       const int nv = ctl->plan.nv_eff;
       const int32_t* vk = p.vidx + static_cast<int64_t>(h) * p.nv_cap + pos0;
 #pragma unroll
@@ -312,13 +312,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     sparse_iter_init(it);
     float m_ref = -INFINITY, l_sum = 0.f;
     bool ok = true;
-    int src, tile, cls;
+    int src, start, cls;
     for (int n = 0; n < N && ok; ++n) {
-      sparse_iter_next(it, plan, src, tile, cls);
+      sparse_iter_next(it, plan, src, start, cls);
       // full item: every pair causal, of this class and a member
       bool full;
       if (src == 1) {
-        const int64_t j0 = static_cast<int64_t>(tile) * BN, j1 = j0 + BN - 1;
+        const int64_t j0 = start, j1 = j0 + BN - 1;
         full = item_is_full(i0, i_hi, j0, j1, p.s, p.w, cls, p.reading);
         if (full) {
           const uint32_t* vrow = p.vbit + static_cast<int64_t>(h) * p.wpr;
@@ -327,7 +327,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         if (full) full = i0 - j1 >= 0 &&
                          all_bits(p.sbit + static_cast<int64_t>(h) * p.wpr, i0 - j1, i_hi - j0);
       } else {
-        const int64_t pos0 = static_cast<int64_t>(tile) * BN;
+        const int64_t pos0 = start;
         full = pos0 + BN <= plan.nv_eff;
         if (full) {
           const int32_t* vk = p.vidx + static_cast<int64_t>(h) * p.nv_cap;
@@ -343,7 +343,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       tc_fence_after();
       const uint32_t tS = tbase + lane_off + static_cast<uint32_t>(st * 128);
       const uint32_t tO = tbase + lane_off + 256u;
-      ok = sparse_half_step(tS, tO, n, full, src, tile, cls, i, p, h, sc, nb, pb, m_ref, l_sum,
+      ok = sparse_half_step(tS, tO, n, full, src, start, cls, i, p, h, sc, nb, pb, m_ref, l_sum,
                             pc, ctl, abort_flag, p.status);
       if (!ok) break;
       // the first class ends: its operand tile becomes the third class's
@@ -402,9 +402,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       SparseIter it;
       sparse_iter_init(it);
       bool ok = true;
-      int src, tile, cls;
+      int src, start, cls;
       for (int n = 0; n < N && ok; ++n) {
-        sparse_iter_next(it, plan, src, tile, cls);
+        sparse_iter_next(it, plan, src, start, cls);
         for (int which = 0; which < 2; ++which) {  // 0: keys, 1: values
           const int li = 2 * n + which;
           const int slot = li % NSLOT;
@@ -418,8 +418,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           const CUtensorMap* tm = src == 1 ? (which ? &tm_v : &tm_k) : (which ? &tm_gv : &tm_gk);
           const int head_coord = src == 1 ? g : h;
           mbar_arrive_expect_tx(&ctl->slot_full[slot], TILE_BYTES);
-          tma_load_3d(dst, tm, &ctl->slot_full[slot], 0, head_coord, tile * BN);
-          tma_load_3d(dst + HALF_BYTES, tm, &ctl->slot_full[slot], 64, head_coord, tile * BN);
+          // rows from the item's first key (slash) or first position (vertical)
+          tma_load_3d(dst, tm, &ctl->slot_full[slot], 0, head_coord, start);
+          tma_load_3d(dst + HALF_BYTES, tm, &ctl->slot_full[slot], 64, head_coord, start);
           last_li[slot] = li;
         }
       }
@@ -444,7 +445,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       };
       SparseIter it;
       sparse_iter_init(it);
-      int src, tile, cls;
+      int src, start, cls;
       // S(n) into buffer n & 1 with the class's query operand
       auto issue_s = [&](int n) {
         const int li = 2 * n;
@@ -462,7 +463,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       bool ok = wait_bounded(&ctl->q_ready, 0u, abort_flag, p.status, p.timeout_ns, ST_MMA);
       int issued = 0;  // S issued for items < issued
       for (int k = 0; k < 2 && k < N && ok; ++k) {
-        sparse_iter_next(it, plan, src, tile, cls);
+        sparse_iter_next(it, plan, src, start, cls);
         ok = full_wait(2 * k);
         if (!ok) break;
         tc_fence_after();
@@ -486,7 +487,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         mma_commit(&ctl->pv_done[n & 1]);
         mma_commit(&ctl->slot_empty[lv % NSLOT]);
         if (issued < N) {  // S(n + 2) reuses buffer n & 1 after P.V(n) (in issue order)
-          sparse_iter_next(it, plan, src, tile, cls);
+          sparse_iter_next(it, plan, src, start, cls);
           ok = full_wait(2 * issued);
           if (!ok) break;
           // the query operand of a class that reuses tile 0 is written by the

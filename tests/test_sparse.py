@@ -54,18 +54,18 @@ def check_cover(lib, V, S, i0, i_last, s, w, reading):
         return 2
 
     count = defaultdict(int)
-    for src, tile, cls in items:
+    for src, start, cls in items:
         if src == 0:
-            assert 0 <= 128 * tile < len(V), (tile, len(V))
-            keys = [int(x) for x in V[128 * tile:128 * tile + 128]]
+            assert start % 128 == 0 and 0 <= start < len(V), (start, len(V))
+            keys = [int(x) for x in V[start:start + 128]]
             for i in range(i0, i_last + 1):
                 for j in keys:
                     if j <= i and klass(i, j) == cls:
                         count[(i, j)] += 1
         else:
-            assert 0 <= tile <= i_last // 128
+            assert 0 <= start <= i_last
             for i in range(i0, i_last + 1):
-                for j in range(128 * tile, 128 * tile + 128):
+                for j in range(start, start + 128):
                     if j > i or j in Vset:
                         continue
                     if (i - j) not in Sset and j != i:
@@ -102,6 +102,16 @@ def test_plan_covers_every_member_once(lib, L, s, w, nv, nb, nf, reading):
         i0 = 128 * t
         i_last = min(i0 + 127, L - 1)
         check_cover(lib, V[0], S[0], i0, i_last, s, w, reading)
+
+
+@pytest.mark.parametrize("reading", [0, 1])
+def test_plan_windows_near_each_other(lib, reading):
+    """Far diagonals 100, 129 and 130 keys apart: windows that start at a
+    range's first key may run past its end but never into the next range."""
+    S = [0, 1, 2, 3, 300, 400, 529, 530, 659, 789, 1000]
+    V = [5, 77, 640, 641]
+    for i0 in (896, 1024, 1152):
+        check_cover(lib, V, S, i0, i0 + 127, 512, 64, reading)
 
 
 def test_plan_empty_pattern_is_the_diagonal(lib):
