@@ -691,14 +691,16 @@ def run_sparse_bench(args, sw, world, rank, local, dist):
     s1.record()
     torch.cuda.synchronize()
     sel_ms = s0.elapsed_time(s1) / 3
-    sel_flops = 2 * 2.0 * 64 * lk * w.Hq * w.d  # two score passes, 2 FLOP per multiply-add
-    alu_peak = 148 * 128 * 2 * (clk.get("sm_mhz") or 1965.0) * 1e6 / 1e12
+    # one 2^x per (row, key) pair and pass on the exponential unit (16 per SM
+    # per clock), the unit the score passes' softmax side is bound by
+    sel_ex2 = 2.0 * 64 * lk * w.Hq
+    ex2_peak = 148 * 16 * (clk.get("sm_mhz") or 1965.0) * 1e6 / 1e9
+    sel_rate = sel_ex2 / (sel_ms / 1e3) / 1e9
     select_info = {"kv_len": lk, "n_last": 64, "n_vertical": sw.n_vertical, "n_slash": n_s,
                    "positions": "continuous", "ms": sel_ms,
-                   "score_tflops": sel_flops / (sel_ms / 1e3) / 1e12,
-                   "roofline": {"bound": "alu", "peak": alu_peak, "unit": "TFLOP/s",
-                                "frac": sel_flops / (sel_ms / 1e3) / 1e12 / alu_peak,
-                                "peak_kind": "FP32 FMA: 148 SMs x 128 lanes x 2 x median SM clock"}}
+                   "roofline": {"bound": "alu", "achieved": sel_rate, "peak": ex2_peak,
+                                "unit": "G exp2/s", "frac": sel_rate / ex2_peak,
+                                "peak_kind": "MUFU exp2: 148 SMs x 16 per clock x median SM clock"}}
     line = {
         "metric": SPARSE_METRIC, "value": whole_job_rate(w.L, world, ms_per_step), "unit": UNIT,
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,

@@ -17,7 +17,8 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libdca_b200.so")
 SOURCES = ["dca_api.cu", "dca_prep.cu", "dca_fwd_sm100.cu", "dca_fwd_f32.cu", "dca_decode_sm100.cu",
-           "dca_sparse_sm100.cu", "dca_sparse_prep.cu", "dca_select.cu", "dca_noalloc.cu"]
+           "dca_sparse_sm100.cu", "dca_sparse_prep.cu", "dca_select.cu", "dca_select_mma.cu",
+           "dca_noalloc.cu"]
 HEADERS = ["dca_internal.h", "dca_plan.cuh", "dca_softmax.cuh", "dca_sparse_plan.cuh",
            "sm100_ptx.cuh"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]

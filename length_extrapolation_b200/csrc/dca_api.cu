@@ -733,6 +733,8 @@ int dca_sparse_select(const dca_sparse_config* cfg, const void* q_block, const v
   a.nv_cap = S.nv_cap;
   a.s_cap = S.s_cap;
   a.wpr = S.wpr;
+  a.status = reinterpret_cast<unsigned int*>(base);
+  a.timeout_ns = static_cast<unsigned long long>(g_timeout_ns.load());
   cudaError_t e = dca::launch_select(a, st);
   if (e == cudaSuccess) {
     const dca::SparseArgs sa = sparse_args(S, sparse_ws);

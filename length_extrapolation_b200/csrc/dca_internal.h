@@ -83,8 +83,19 @@ struct SelectArgs {
   int2* runs;
   uint32_t *vbit, *sbit;
   int64_t nv_cap, s_cap, wpr;
+  unsigned int* status;   // device status word (timeouts of the score passes)
+  unsigned long long timeout_ns;
 };
 size_t select_scratch_bytes(int64_t Lk, int Hq, int64_t n_chunks);
+// Score passes of the selection (tcgen05): pass 1 writes per-slice row
+// statistics `part` [Hq][select_slices(Lk)][64]; pass 2 reads the merged
+// `stats` [Hq][64] and writes vert (stored) and slash (accumulated).
+int select_slices(int64_t Lk);
+cudaError_t launch_select_scores(const void* kr, const float* qv, const float2* crot, float2* part,
+                                 const float2* stats, float* vert, float* slash, int64_t i_first,
+                                 int64_t Lk, int64_t s, int64_t w, int n_last, int Hq, int Hkv,
+                                 int reading, int continuous, int pass, unsigned int* status,
+                                 unsigned long long timeout_ns, cudaStream_t st);
 cudaError_t launch_select(const SelectArgs& sa, cudaStream_t st);
 
 // bf16 tcgen05/TMA kernel; returns a CUDA error or cudaSuccess, or

@@ -12,11 +12,9 @@
 // (lists, bitmaps, slash runs) for dca_sparse_attend.
 //
 // Kernels: query variants (fp64 angles where the table has none), two score
-// passes over the key tiles (row max/sum, then the sums of probabilities),
-// a merge of the row statistics, a radix select per (head, kind), and the
-// gather of the selected vertical rows.  The score passes are fp32 CUDA-core
-// dot products: 64 rows x 128 keys per tile is too thin for the tensor cores
-// to matter next to the attention that follows.
+// passes over the keys on the tensor cores (dca_select_mma.cu: row max/sum,
+// then the sums of probabilities), a merge of the row statistics, a radix
+// select per (head, kind), and the gather of the selected vertical rows.
 #include <cuda_bf16.h>
 #include <math.h>
 
@@ -32,221 +30,9 @@ namespace sel {
 constexpr int ROWS = 64;     // rows of the estimate (max)
 constexpr int KT = 128;      // keys per tile
 constexpr int HD = 128;
-constexpr int THREADS = 256;
-constexpr int OBINS = ROWS + KT;  // distinct offsets i - j of one tile
 
-struct ScoreParams {
-  const float* qv;          // [Hq][nvar][ROWS][HD] rotated, scaled (log2 units) query rows
-  const __nv_bfloat16* kr;  // rotated keys R(j mod s) k_j [cap][Hkv][HD]
-  const float2* crot;       // continuous: per key chunk n, (cos, sin) of s*n*theta_k [n_chunks][64]
-  float2* part;             // pass 1 out: [Hq][n_tiles][ROWS] (tile max, tile sum of 2^(x - max))
-  const float2* stats;      // pass 2 in: [Hq][ROWS] (row max, row sum)
-  float* vert;              // pass 2 out: [Hq][Lk]
-  float* slash;             // pass 2 out: [Hq][Lk]
-  int64_t i_first, Lk, s, w;
-  int n_last, Hq, Hkv, G, nvar, n_tiles, reading, continuous;
-};
-
-// Variant of the query row i (chunk ni) for key j (chunk nj): DCA class (0
-// intra, 1 successive, 2 inter), or 0 for continuous positions.
-__device__ __forceinline__ int variant(const ScoreParams& p, int64_t i, int64_t ni, int64_t j,
-                                       int64_t nj) {
-  if (p.continuous) return 0;
-  return pair_class(ni - nj, i - j, p.w, p.reading);
-}
-
-constexpr int KTP = KT + 4;    // padded key count of a dim-major key row
-constexpr int RP = ROWS + 4;   // padded row count of a dim-major query row
-
-// One CTA per (key tile, KV group): the tile's keys are loaded once (fp32,
-// dim-major; continuous positions: rotated from j mod s to j) and serve the
-// group's G query heads in turn.  Thread (ty, tx) owns rows 4ty..4ty+3 and
-// keys 8tx..8tx+7: per dim one 16-byte load of the rows, two of the keys, 16
-// packed FMAs.
-template <bool PASS2>
-__global__ void __launch_bounds__(THREADS)
-    sel_score_kernel(const ScoreParams p) {
-  extern __shared__ float sm[];
-  float* Kt = sm;                       // [HD][KTP]
-  float* Qt = Kt + HD * KTP;            // [nvar][HD][RP] (current head)
-  __shared__ float colsum[16][KT];
-  __shared__ float obin[OBINS];
-  __shared__ float2 st[ROWS];
-
-  const int tile = blockIdx.x;
-  const int g = blockIdx.y;
-  const int64_t j0 = static_cast<int64_t>(tile) * KT;
-  const int t = threadIdx.x;
-  const int ty = t >> 4, tx = t & 15;
-
-  for (int idx = t; idx < KT * (HD / 2); idx += THREADS) {
-    const int r = idx / (HD / 2), k = idx % (HD / 2);
-    const int64_t j = j0 + r;
-    float a = 0.f, b = 0.f;
-    if (j < p.Lk) {
-      const __nv_bfloat16* kr = p.kr + (j * p.Hkv + g) * static_cast<int64_t>(HD);
-      a = __bfloat162float(kr[k]);
-      b = __bfloat162float(kr[k + HD / 2]);
-      if (p.continuous) {
-        const float2 cs = p.crot[(j / p.s) * (HD / 2) + k];
-        const float ra = a * cs.x - b * cs.y, rb = a * cs.y + b * cs.x;
-        a = ra;
-        b = rb;
-      }
-    }
-    Kt[k * KTP + r] = a;
-    Kt[(k + HD / 2) * KTP + r] = b;
-  }
-
-  // the variant of each of this thread's pairs (-1: not a causal pair of the
-  // estimate) -- the same for every head of the group -- and the variants
-  // present in the tile
-  int8_t var[4][8];
-  {
-    int64_t nkey[8];
-#pragma unroll
-    for (int u = 0; u < 8; ++u) nkey[u] = (j0 + 8 * tx + u) / p.s;
-#pragma unroll
-    for (int a = 0; a < 4; ++a) {
-      const int r = 4 * ty + a;
-      const int64_t i = p.i_first + r;
-      const int64_t ni = i / p.s;
-#pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const int64_t j = j0 + 8 * tx + u;
-        var[a][u] = (r < p.n_last && j <= i && j < p.Lk)
-                        ? static_cast<int8_t>(variant(p, i, ni, j, nkey[u]))
-                        : static_cast<int8_t>(-1);
-      }
-    }
-  }
-  bool present[3];
-  for (int v = 0; v < 3; ++v) {
-    bool any = false;
-#pragma unroll
-    for (int a = 0; a < 4; ++a)
-#pragma unroll
-      for (int u = 0; u < 8; ++u) any |= var[a][u] == v;
-    present[v] = __syncthreads_or(any) != 0;
-  }
-
-  for (int hh = 0; hh < p.G; ++hh) {
-    const int h = g * p.G + hh;
-    __syncthreads();  // the previous head is done with Qt, obin, colsum
-    for (int v = 0; v < p.nvar; ++v) {
-      if (!present[v]) continue;
-      const float* src = p.qv + (static_cast<int64_t>(h) * p.nvar + v) * ROWS * HD;
-      for (int idx = t; idx < ROWS * HD; idx += THREADS) {
-        const int r = idx / HD, k = idx % HD;
-        Qt[(v * HD + k) * RP + r] = src[idx];
-      }
-    }
-    if (PASS2) {
-      for (int o = t; o < OBINS; o += THREADS) obin[o] = 0.f;
-      for (int r = t; r < ROWS; r += THREADS) st[r] = p.stats[h * ROWS + r];
-    }
-    __syncthreads();
-
-    float x[4][8];
-#pragma unroll
-    for (int a = 0; a < 4; ++a)
-#pragma unroll
-      for (int u = 0; u < 8; ++u) x[a][u] = -INFINITY;
-    for (int v = 0; v < p.nvar; ++v) {
-      if (!present[v]) continue;
-      float2 acc[4][4];
-#pragma unroll
-      for (int a = 0; a < 4; ++a)
-#pragma unroll
-        for (int u = 0; u < 4; ++u) acc[a][u] = make_float2(0.f, 0.f);
-      const float* qb = Qt + v * HD * RP + 4 * ty;
-      const float* kb = Kt + 8 * tx;
-#pragma unroll 4
-      for (int k = 0; k < HD; ++k) {
-        const float4 q4 = *reinterpret_cast<const float4*>(qb + k * RP);
-        const float4 k0 = *reinterpret_cast<const float4*>(kb + k * KTP);
-        const float4 k1 = *reinterpret_cast<const float4*>(kb + k * KTP + 4);
-        const float2 kk[4] = {make_float2(k0.x, k0.y), make_float2(k0.z, k0.w),
-                              make_float2(k1.x, k1.y), make_float2(k1.z, k1.w)};
-        const float qq[4] = {q4.x, q4.y, q4.z, q4.w};
-#pragma unroll
-        for (int a = 0; a < 4; ++a)
-#pragma unroll
-          for (int u = 0; u < 4; ++u) acc[a][u] = fma2(make_float2(qq[a], qq[a]), kk[u], acc[a][u]);
-      }
-#pragma unroll
-      for (int a = 0; a < 4; ++a)
-#pragma unroll
-        for (int u = 0; u < 8; ++u)
-          if (var[a][u] == v) x[a][u] = (u & 1) ? acc[a][u >> 1].y : acc[a][u >> 1].x;
-    }
-
-    if (!PASS2) {
-      // per row: tile max and sum of 2^(x - max) over the 16 threads of the row group
-#pragma unroll
-      for (int a = 0; a < 4; ++a) {
-        float m = x[a][0];
-#pragma unroll
-        for (int u = 1; u < 8; ++u) m = fmaxf(m, x[a][u]);
-#pragma unroll
-        for (int off = 8; off >= 1; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
-        float l = 0.f;
-        if (m != -INFINITY) {
-#pragma unroll
-          for (int u = 0; u < 8; ++u) l += exp2f(x[a][u] - m);
-        }
-#pragma unroll
-        for (int off = 8; off >= 1; off >>= 1) l += __shfl_xor_sync(0xffffffffu, l, off);
-        if (tx == 0) {
-          const int r = 4 * ty + a;
-          p.part[(static_cast<int64_t>(h) * p.n_tiles + tile) * ROWS + r] = make_float2(m, l);
-        }
-      }
-      continue;
-    }
-
-    // pass 2: probabilities; column sums (vertical) and diagonal sums (slash)
-    float cs[8], dg[11];  // column sums; sums along this thread's 11 diagonals a - u
-#pragma unroll
-    for (int u = 0; u < 8; ++u) cs[u] = 0.f;
-#pragma unroll
-    for (int e = 0; e < 11; ++e) dg[e] = 0.f;
-#pragma unroll
-    for (int a = 0; a < 4; ++a) {
-      const int r = 4 * ty + a;
-      const float2 rs = st[r];
-      const float inv = rs.y > 0.f ? 1.f / rs.y : 0.f;
-#pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const float pr = x[a][u] == -INFINITY ? 0.f : exp2f(x[a][u] - rs.x) * inv;
-        cs[u] += pr;
-        dg[a - u + 7] += pr;
-      }
-    }
-    // offset o = (i_first + 4ty + a) - (j0 + 8tx + u); bin = o - (i_first - j0 - KT + 1)
-#pragma unroll
-    for (int e = 0; e < 11; ++e)
-      if (dg[e] != 0.f) atomicAdd(&obin[4 * ty - 8 * tx + (e - 7) + KT - 1], dg[e]);
-#pragma unroll
-    for (int u = 0; u < 8; ++u) colsum[ty][8 * tx + u] = cs[u];
-    __syncthreads();
-    if (t < KT) {
-      float v = 0.f;
-#pragma unroll
-      for (int y = 0; y < 16; ++y) v += colsum[y][t];
-      const int64_t j = j0 + t;
-      if (j < p.Lk) p.vert[static_cast<int64_t>(h) * p.Lk + j] = v;
-    }
-    for (int b = t; b < OBINS; b += THREADS) {
-      const float v = obin[b];
-      const int64_t o = (p.i_first - j0 - KT + 1) + b;
-      if (v != 0.f && o >= 0 && o < p.Lk)
-        atomicAdd(&p.slash[static_cast<int64_t>(h) * p.Lk + o], v);
-    }
-  }
-}
-
-// Row statistics: max and sum over the tiles (one warp per (head, row)).
+// Row statistics: max and sum over the key slices' partial (max, sum) (one
+// warp per (head, row)).
 __global__ void sel_stats_kernel(const float2* __restrict__ part, float2* __restrict__ stats,
                                  int n_tiles, int Hq) {
   const int wid = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
@@ -462,7 +248,7 @@ size_t select_scratch_bytes(int64_t Lk, int Hq, int64_t n_chunks) {
   auto add = [&](size_t n) { b += (n + 255) / 256 * 256; };
   add(sizeof(float) * static_cast<size_t>(Hq) * 3 * sel::ROWS * sel::HD);   // query variants
   add(sizeof(float2) * static_cast<size_t>(n_chunks) * (sel::HD / 2));     // chunk rotations
-  add(sizeof(float2) * static_cast<size_t>(Hq) * n_tiles * sel::ROWS);     // tile statistics
+  add(sizeof(float2) * static_cast<size_t>(Hq) * n_tiles * sel::ROWS);     // slice statistics
   add(sizeof(float2) * static_cast<size_t>(Hq) * sel::ROWS);               // row statistics
   add(sizeof(float) * static_cast<size_t>(Hq) * Lk * 2);                   // scores
   return b;
@@ -487,7 +273,8 @@ cudaError_t launch_select(const SelectArgs& sa, cudaStream_t st) {
   float* vert = scores;
   float* slash = scores + static_cast<int64_t>(sa.Hq) * sa.Lk;
 
-  cudaError_t e = cudaMemsetAsync(scores, 0, sizeof(float) * sa.Hq * sa.Lk * 2, st);
+  // vert is stored whole by the second score pass; slash is accumulated
+  cudaError_t e = cudaMemsetAsync(slash, 0, sizeof(float) * sa.Hq * sa.Lk, st);
   if (e != cudaSuccess) return e;
   {
     const int64_t n = std::max<int64_t>(static_cast<int64_t>(sa.Hq) * nvar * ROWS * (HD / 2),
@@ -498,43 +285,19 @@ cudaError_t launch_select(const SelectArgs& sa, cudaStream_t st) {
         static_cast<int>(sa.n_chunks));
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
-  ScoreParams p;
-  p.qv = qv;
-  p.kr = static_cast<const __nv_bfloat16*>(sa.kr);
-  p.crot = crot;
-  p.part = part;
-  p.stats = stats;
-  p.vert = vert;
-  p.slash = slash;
-  p.i_first = sa.q_start + sa.Lq - sa.n_last;
-  p.Lk = sa.Lk;
-  p.s = sa.s;
-  p.w = sa.w;
-  p.n_last = sa.n_last;
-  p.Hq = sa.Hq;
-  p.Hkv = sa.Hkv;
-  p.G = sa.Hq / sa.Hkv;
-  p.nvar = nvar;
-  p.n_tiles = static_cast<int>(n_tiles);
-  p.reading = sa.reading;
-  p.continuous = sa.continuous;
-  const size_t smem = sizeof(float) * (HD * KTP + nvar * HD * RP);
-  const dim3 grid(static_cast<unsigned>(n_tiles), static_cast<unsigned>(sa.Hkv));
-  if ((e = cudaFuncSetAttribute(sel_score_kernel<false>,
-                                cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                static_cast<int>(smem))) != cudaSuccess)
-    return e;
-  if ((e = cudaFuncSetAttribute(sel_score_kernel<true>,
-                                cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                static_cast<int>(smem))) != cudaSuccess)
-    return e;
-  sel_score_kernel<false><<<grid, THREADS, smem, st>>>(p);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  const int64_t i_first = sa.q_start + sa.Lq - sa.n_last;
+  const int n_slices = select_slices(sa.Lk);
+  e = launch_select_scores(sa.kr, qv, crot, part, stats, vert, slash, i_first, sa.Lk, sa.s, sa.w,
+                           sa.n_last, sa.Hq, sa.Hkv, sa.reading, sa.continuous, 1, sa.status,
+                           sa.timeout_ns, st);
+  if (e != cudaSuccess) return e;
   sel_stats_kernel<<<static_cast<unsigned>((sa.Hq * ROWS * 32 + 255) / 256), 256, 0, st>>>(
-      part, stats, static_cast<int>(n_tiles), sa.Hq);
+      part, stats, n_slices, sa.Hq);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  sel_score_kernel<true><<<grid, THREADS, smem, st>>>(p);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  e = launch_select_scores(sa.kr, qv, crot, part, stats, vert, slash, i_first, sa.Lk, sa.s, sa.w,
+                           sa.n_last, sa.Hq, sa.Hkv, sa.reading, sa.continuous, 2, sa.status,
+                           sa.timeout_ns, st);
+  if (e != cudaSuccess) return e;
   SelectOut o;
   o.nv = sa.nv;
   o.ns = sa.ns;
