@@ -145,70 +145,172 @@ struct SelectOut {
   int64_t nv_cap, s_cap, wpr;
 };
 
-// Top-k by value (ties: smaller index) of scores[0 .. Lk) (all >= 0), for
-// (head, kind) = (blockIdx.x / 2, blockIdx.x % 2): radix select on the float
-// bits (order-preserving for non-negative floats) in three histogram passes,
-// then an ordered pass writes the selected indices ascending.
-__global__ void __launch_bounds__(1024)
-    sel_topk_kernel(const float* __restrict__ vert, const float* __restrict__ slash, int64_t Lk,
-                    int64_t n_v, int64_t n_s, SelectOut out) {
-  __shared__ int hist[4096];
-  __shared__ int warp_sums[32];
-  __shared__ int sh_bin, sh_above;
-  const int h = blockIdx.x >> 1, kind = blockIdx.x & 1;
-  const float* sc = (kind ? slash : vert) + static_cast<int64_t>(h) * Lk;
-  const int64_t kk = kind ? (n_s < Lk ? n_s : Lk) : (n_v < Lk ? n_v : Lk);
-  const int tid = threadIdx.x;
+// Top-k by value (ties: the smaller index) of each score row (vertical and
+// slash of every head, all scores >= 0): a radix select on the float bits
+// (order-preserving for non-negative floats), 12 + 12 + 8 bits.  Each pass
+// is a histogram over the row's spans (one CTA per span, warp-aggregated
+// shared-memory atomics, then the nonzero bins into a global histogram) and
+// a pick of the bin holding the k-th largest (a suffix scan over the bins).
+// Then per span the count above / equal to the k-th value, and an ordered
+// write: the spans' counts place each span's output, equal values are taken
+// in index order, so the list comes out ascending.
+constexpr int TK_THREADS = 1024;
+constexpr int TK_BINS = 4096;
 
-  uint32_t prefix = 0;   // selected high bits so far
-  int64_t above = 0;     // elements strictly above the current prefix bucket
-  const int shifts[3] = {20, 8, 0};
-  const int widths[3] = {12, 12, 8};
-  for (int pass = 0; pass < 3 && kk > 0; ++pass) {
-    const int nb = 1 << widths[pass];
-    for (int b = tid; b < nb; b += 1024) hist[b] = 0;
-    __syncthreads();
-    const int top = pass == 0 ? 32 : shifts[pass - 1];
-    const int lane = tid & 31;
-    for (int64_t base = 0; base < Lk; base += 1024) {
-      // lanes with the same bin add once (scores crowd into a few bins)
-      const int64_t j = base + tid;
-      int bin = -1;
-      if (j < Lk) {
-        const uint32_t bits = __float_as_uint(sc[j]);
-        if (pass == 0 || (bits >> top) == prefix) bin = static_cast<int>((bits >> shifts[pass]) & (nb - 1));
-      }
-      const unsigned peers = __match_any_sync(0xffffffffu, bin);
-      if (bin >= 0 && lane == __ffs(peers) - 1) atomicAdd(&hist[bin], __popc(peers));
+struct TopkState {
+  uint32_t prefix;  // the high bits of the k-th largest found so far
+  int32_t pad;
+  int64_t above;    // elements strictly above the prefix's bucket
+};
+
+struct TopkArgs {
+  const float* vert;   // [Hq][Lk]
+  const float* slash;  // [Hq][Lk]
+  int64_t Lk, n_v, n_s, span;
+  int nb;              // spans (CTAs) per row; rows = 2 Hq: (head, kind)
+  int* hist;           // [rows][TK_BINS]
+  TopkState* state;    // [rows]
+  int2* cnt;           // [rows][nb]: (above the k-th value, equal to it)
+};
+
+// span of one CTA: a multiple of the block, at least 16K, at most 1024 spans per row
+inline int64_t topk_span(int64_t Lk) {
+  int64_t sp = (Lk + 1023) / 1024;
+  if (sp < 16384) sp = 16384;
+  return (sp + TK_THREADS - 1) / TK_THREADS * TK_THREADS;
+}
+
+__device__ __forceinline__ int64_t topk_k(const TopkArgs& a, int row) {
+  const int64_t n = (row & 1) ? a.n_s : a.n_v;
+  return n < a.Lk ? n : a.Lk;
+}
+__device__ __forceinline__ const float* topk_row(const TopkArgs& a, int row) {
+  return ((row & 1) ? a.slash : a.vert) + static_cast<int64_t>(row >> 1) * a.Lk;
+}
+
+__global__ void __launch_bounds__(TK_THREADS)
+    sel_topk_hist_kernel(const TopkArgs a, int pass) {
+  __shared__ int hist[TK_BINS];
+  const int row = blockIdx.y;
+  if (topk_k(a, row) == 0) return;
+  const int shift = pass == 0 ? 20 : (pass == 1 ? 8 : 0);
+  const int nbin = pass == 2 ? 256 : TK_BINS;
+  const int top = pass == 0 ? 32 : (pass == 1 ? 20 : 8);  // bits above this pass
+  const uint32_t prefix = pass == 0 ? 0u : a.state[row].prefix;
+  const int tid = threadIdx.x, lane = tid & 31;
+  for (int b = tid; b < nbin; b += TK_THREADS) hist[b] = 0;
+  __syncthreads();
+  const float* sc = topk_row(a, row);
+  const int64_t j0 = static_cast<int64_t>(blockIdx.x) * a.span;
+  for (int64_t j = j0 + tid; j < j0 + a.span; j += TK_THREADS) {  // same trip count in every lane
+    int bin = -1;
+    if (j < a.Lk) {
+      const uint32_t bits = __float_as_uint(sc[j]);
+      if ((static_cast<uint64_t>(bits) >> top) == prefix) bin = static_cast<int>((bits >> shift) & (nbin - 1));
     }
-    __syncthreads();
-    if (tid == 0) {
-      int64_t cum = above;
-      int b = nb - 1;
-      for (; b >= 0; --b) {
-        if (cum + hist[b] >= kk) break;
-        cum += hist[b];
-      }
-      sh_bin = b < 0 ? 0 : b;
-      sh_above = static_cast<int>(cum);
-    }
-    __syncthreads();
-    prefix = (prefix << widths[pass]) | static_cast<uint32_t>(sh_bin);
-    above = sh_above;
-    __syncthreads();
+    const unsigned peers = __match_any_sync(0xffffffffu, bin);
+    if (bin >= 0 && lane == __ffs(peers) - 1) atomicAdd(&hist[bin], __popc(peers));
   }
-  const uint32_t T = prefix;                // the k-th largest value's bits
-  const int64_t need_eq = kk - above;       // how many equal to T are taken
+  __syncthreads();
+  int* g = a.hist + static_cast<int64_t>(row) * TK_BINS;
+  for (int b = tid; b < nbin; b += TK_THREADS)
+    if (hist[b] != 0) atomicAdd(&g[b], hist[b]);
+}
+
+// One CTA per row: the bin holding the k-th largest (bins scanned from the
+// top), appended to the prefix; clears the histogram for the next pass.
+__global__ void __launch_bounds__(TK_THREADS)
+    sel_topk_pick_kernel(const TopkArgs a, int pass) {
+  __shared__ int warp_sums[32];
+  const int row = blockIdx.x;
+  const int64_t kk = topk_k(a, row);
+  if (kk == 0) return;
+  const int nbin = pass == 2 ? 256 : TK_BINS;
+  const int width = pass == 2 ? 8 : 12;
+  const int per = nbin / TK_THREADS > 0 ? nbin / TK_THREADS : 1;  // bins per thread
+  const uint32_t prefix = pass == 0 ? 0u : a.state[row].prefix;
+  const int64_t above = pass == 0 ? 0 : a.state[row].above;
+  int* g = a.hist + static_cast<int64_t>(row) * TK_BINS;
+  const int tid = threadIdx.x;
+  int c[4] = {0, 0, 0, 0};
+  int sum = 0;
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    const int d = tid * per + e;  // rank of the bin from the top
+    if (e < per && d < nbin) c[e] = g[nbin - 1 - d];
+    sum += c[e];
+  }
+  int total;
+  int64_t cum = above + block_scan(sum, warp_sums, total);  // elements in higher bins
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    const int d = tid * per + e;
+    if (e < per && d < nbin && cum < kk && cum + c[e] >= kk) {
+      a.state[row].prefix = (prefix << width) | static_cast<uint32_t>(nbin - 1 - d);
+      a.state[row].above = cum;
+    }
+    cum += c[e];
+  }
+  for (int b = tid; b < TK_BINS; b += TK_THREADS) g[b] = 0;  // every read is behind the scan's barriers
+}
+
+// Per span: how many scores are above / equal to the k-th value T.
+__global__ void __launch_bounds__(TK_THREADS)
+    sel_topk_count_kernel(const TopkArgs a) {
+  __shared__ int warp_sums[32];
+  const int row = blockIdx.y;
+  if (topk_k(a, row) == 0) return;
+  const uint32_t T = a.state[row].prefix;
+  const float* sc = topk_row(a, row);
+  const int64_t j0 = static_cast<int64_t>(blockIdx.x) * a.span;
+  int gt = 0, eq = 0;
+  for (int64_t j = j0 + threadIdx.x; j < j0 + a.span && j < a.Lk; j += TK_THREADS) {
+    const uint32_t bits = __float_as_uint(sc[j]);
+    gt += bits > T;
+    eq += bits == T;
+  }
+  int tg, te;
+  block_scan(gt, warp_sums, tg);
+  block_scan(eq, warp_sums, te);
+  if (threadIdx.x == 0) a.cnt[static_cast<int64_t>(row) * a.nb + blockIdx.x] = make_int2(tg, te);
+}
+
+// Ordered write of the selected indices of each span (ascending), their
+// bitmap bits; equal values are taken while the row still needs them.
+__global__ void __launch_bounds__(TK_THREADS)
+    sel_topk_write_kernel(const TopkArgs a, SelectOut out) {
+  __shared__ int warp_sums[32];
+  __shared__ long long sh_start, sh_eq_before;
+  const int row = blockIdx.y, kind = row & 1, h = row >> 1;
+  const int64_t kk = topk_k(a, row);
+  if (kk == 0) return;
+  const uint32_t T = a.state[row].prefix;
+  const int64_t need_eq = kk - a.state[row].above;
+  if (threadIdx.x == 0) {
+    const int2* cr = a.cnt + static_cast<int64_t>(row) * a.nb;
+    int64_t start = 0, eqb = 0;
+    for (int b = 0; b < static_cast<int>(blockIdx.x); ++b) {
+      const int2 cb = cr[b];
+      int64_t take = need_eq - eqb;
+      take = take < 0 ? 0 : (take > cb.y ? cb.y : take);
+      start += cb.x + take;
+      eqb += cb.y;
+    }
+    sh_start = start;
+    sh_eq_before = eqb;
+  }
+  __syncthreads();
   int32_t* list = kind ? out.soff + h * out.s_cap : out.vidx + h * out.nv_cap;
   uint32_t* bitrow = (kind ? out.sbit : out.vbit) + h * out.wpr;
-  int64_t eq_seen = 0, written = 0;
-  for (int64_t base = 0; base < Lk && kk > 0; base += 1024) {
-    const int64_t j = base + tid;
-    const uint32_t bits = j < Lk ? __float_as_uint(sc[j]) : 0u;
-    const int is_eq = (j < Lk && bits == T) ? 1 : 0;
+  int64_t eq_seen = sh_eq_before, written = sh_start;
+  const int64_t j0 = static_cast<int64_t>(blockIdx.x) * a.span;
+  for (int64_t base = j0; base < j0 + a.span && base < a.Lk; base += TK_THREADS) {
+    const int64_t j = base + threadIdx.x;
+    const uint32_t bits = j < a.Lk ? __float_as_uint(topk_row(a, row)[j]) : 0u;
+    const int is_eq = (j < a.Lk && bits == T) ? 1 : 0;
     int eq_total;
     const int eq_before = block_scan(is_eq, warp_sums, eq_total);
-    const int sel = (j < Lk) && (bits > T || (is_eq && eq_seen + eq_before < need_eq)) ? 1 : 0;
+    const int sel = (j < a.Lk) && (bits > T || (is_eq && eq_seen + eq_before < need_eq)) ? 1 : 0;
     int sel_total;
     const int pos = block_scan(sel, warp_sums, sel_total);
     if (sel) {
@@ -218,26 +320,31 @@ __global__ void __launch_bounds__(1024)
     eq_seen += eq_total;
     written += sel_total;
   }
-  __syncthreads();  // the list is complete before one thread reads it
-  if (tid == 0) {
-    if (kind == 0) {
-      out.nv[h] = static_cast<int32_t>(written);
-    } else {
-      out.ns[h] = static_cast<int32_t>(written);
-      // runs of consecutive offsets (the caller keeps n_s <= SPARSE_MAX_RUNS)
-      int n = 0;
-      int2* rr = out.runs + static_cast<int64_t>(h) * SPARSE_MAX_RUNS;
-      for (int64_t e = 0; e < written; ++e) {
-        const int32_t o = list[e];
-        if (n > 0 && rr[n - 1].y == o) {
-          rr[n - 1].y = o + 1;
-        } else if (n < SPARSE_MAX_RUNS) {
-          rr[n++] = make_int2(o, o + 1);
-        }
-      }
-      out.nruns[h] = n;
-    }
+}
+
+// Counts, and the runs of consecutive slash offsets: one CTA per head, one
+// thread per list entry (the caller keeps n_s <= SPARSE_MAX_RUNS < 1024); an
+// entry starts a run unless it follows its predecessor, a scan of the starts
+// numbers the runs.
+__global__ void __launch_bounds__(TK_THREADS)
+    sel_topk_finish_kernel(const TopkArgs a, SelectOut out) {
+  __shared__ int warp_sums[32];
+  const int h = blockIdx.x, e = threadIdx.x;
+  const int64_t ks = topk_k(a, 2 * h + 1);
+  if (e == 0) {
+    out.nv[h] = static_cast<int32_t>(topk_k(a, 2 * h));
+    out.ns[h] = static_cast<int32_t>(ks);
   }
+  const int32_t* list = out.soff + h * out.s_cap;
+  const int32_t o = e < ks ? list[e] : 0;
+  const int start = (e < ks && (e == 0 || list[e - 1] + 1 != o)) ? 1 : 0;
+  const int last = (e < ks && (e + 1 == ks || list[e + 1] != o + 1)) ? 1 : 0;
+  int n_runs;
+  const int idx = block_scan(start, warp_sums, n_runs) - (start ? 0 : 1);  // this entry's run
+  int2* rr = out.runs + static_cast<int64_t>(h) * SPARSE_MAX_RUNS;
+  if (start) rr[idx].x = o;
+  if (last) rr[idx].y = o + 1;
+  if (e == 0) out.nruns[h] = n_runs;
 }
 
 }  // namespace sel
@@ -251,6 +358,10 @@ size_t select_scratch_bytes(int64_t Lk, int Hq, int64_t n_chunks) {
   add(sizeof(float2) * static_cast<size_t>(Hq) * n_tiles * sel::ROWS);     // slice statistics
   add(sizeof(float2) * static_cast<size_t>(Hq) * sel::ROWS);               // row statistics
   add(sizeof(float) * static_cast<size_t>(Hq) * Lk * 2);                   // scores
+  const int64_t nb = (Lk + sel::topk_span(Lk) - 1) / sel::topk_span(Lk);
+  add(sizeof(int) * static_cast<size_t>(2 * Hq) * sel::TK_BINS);            // top-k histograms
+  add(sizeof(sel::TopkState) * static_cast<size_t>(2 * Hq));                // top-k state
+  add(sizeof(int2) * static_cast<size_t>(2 * Hq) * nb);                     // top-k span counts
   return b;
 }
 
@@ -310,8 +421,31 @@ cudaError_t launch_select(const SelectArgs& sa, cudaStream_t st) {
   o.nv_cap = sa.nv_cap;
   o.s_cap = sa.s_cap;
   o.wpr = sa.wpr;
-  sel_topk_kernel<<<static_cast<unsigned>(2 * sa.Hq), 1024, 0, st>>>(vert, slash, sa.Lk, sa.n_v,
-                                                                      sa.n_s, o);
+  TopkArgs ta;
+  ta.vert = vert;
+  ta.slash = slash;
+  ta.Lk = sa.Lk;
+  ta.n_v = sa.n_v;
+  ta.n_s = sa.n_s;
+  ta.span = topk_span(sa.Lk);
+  ta.nb = static_cast<int>((sa.Lk + ta.span - 1) / ta.span);
+  ta.hist = reinterpret_cast<int*>(take(sizeof(int) * 2 * sa.Hq * TK_BINS));
+  ta.state = reinterpret_cast<TopkState*>(take(sizeof(TopkState) * 2 * sa.Hq));
+  ta.cnt = reinterpret_cast<int2*>(take(sizeof(int2) * 2 * sa.Hq * ta.nb));
+  if ((e = cudaMemsetAsync(ta.hist, 0, sizeof(int) * 2 * sa.Hq * TK_BINS, st)) != cudaSuccess)
+    return e;
+  const dim3 spans(static_cast<unsigned>(ta.nb), static_cast<unsigned>(2 * sa.Hq));
+  for (int pass = 0; pass < 3; ++pass) {
+    sel_topk_hist_kernel<<<spans, TK_THREADS, 0, st>>>(ta, pass);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    sel_topk_pick_kernel<<<static_cast<unsigned>(2 * sa.Hq), TK_THREADS, 0, st>>>(ta, pass);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
+  sel_topk_count_kernel<<<spans, TK_THREADS, 0, st>>>(ta);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  sel_topk_write_kernel<<<spans, TK_THREADS, 0, st>>>(ta, o);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  sel_topk_finish_kernel<<<static_cast<unsigned>(sa.Hq), TK_THREADS, 0, st>>>(ta, o);
   return cudaGetLastError();
 }
 

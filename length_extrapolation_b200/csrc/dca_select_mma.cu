@@ -2,7 +2,7 @@
 // cores (dca_select.cu holds the rest of the selection and states what it
 // computes: vertical and slash sums of the last rows' softmax).
 //
-// One CTA = one query head x one slice of 2048 keys.  The 64 estimate rows
+// One CTA = one query head x one slice of 4096 keys.  The 64 estimate rows
 // are the MMA N: S^T = K' Q_v^T (M = 128 keys, N = 64 rows, K = 128 dims,
 // tcgen05.mma kind::f16, fp32 accumulators in TMEM), so TMEM lane t holds
 // key t's logits for all rows and each softmax thread owns one key.
@@ -27,13 +27,15 @@
 //      added to the score arrays once per CTA.
 // The rows of an item's class (and of causality) are one contiguous range
 // per key (class_row_range), so masking is a range test.
-// Warps: 0-3 softmax, 4 TMA producer (3-slot ring of 32 KiB key tiles, no
-// multicast), 5 MMA issuer.  Every mbarrier wait is bounded; on timeout the
+// Warps: 0-3 softmax, 4 TMA producer (ring of 3 -- continuous positions: 4 --
+// 32 KiB key tiles, no multicast), 5 MMA issuer.  Every mbarrier wait is bounded; on timeout the
 // CTA raises its abort flag, ORs a code into the status word, drains its
 // copies and MMAs, frees TMEM and exits.  The softmax warps' own barriers
 // (bar.sync 1, 128) are reached by all four warps on every path.
 #include <cuda_bf16.h>
 #include <math.h>
+
+#include <type_traits>
 
 #include "dca_internal.h"
 #include "dca_plan.cuh"
@@ -43,8 +45,9 @@ namespace dca {
 namespace selm {
 
 constexpr int ROWS = 64, BN = 128, HD = 128;
-constexpr int SLICE = 1536;               // keys per CTA
-constexpr int NSLOT = 3;
+constexpr int SLICE = 4096;               // keys per CTA
+constexpr int NSLOT = 3;                  // key-tile ring (DCA)
+constexpr int NSLOT_MAX = 4;              // continuous: a 4th slot in the unused operand space
 constexpr int TILE_BYTES = 32768, HALF_BYTES = 16384;
 constexpr int QOP = ROWS * HD * 2;        // 16 KiB: one bf16 query operand
 constexpr int QOP_HALF = ROWS * 128;      // its 64-column block
@@ -56,17 +59,17 @@ constexpr int SBINS = SLICE + ROWS;       // offsets i - j met by a slice
 constexpr int MSTRIDE = 136;              // row stride of the merge buffers (conflict-free)
 constexpr int MROWS = 16;                 // rows per merge round
 // pass 2: vertical bins [SLICE] (key j is always updated by one thread) and
-// one copy of the slash bins per softmax warp [4][SBINS] (each lane of the
-// warp updates its own diagonals once per item; no other warp touches it)
+// the slash bins [SBINS] (each lane adds its three diagonal sums once per
+// item, atomically: the warps' diagonal ranges overlap)
 constexpr int BIN_FLOATS =
-    (SLICE + 4 * SBINS) > 2 * MROWS * MSTRIDE ? (SLICE + 4 * SBINS) : 2 * MROWS * MSTRIDE;
+    (SLICE + SBINS) > 2 * MROWS * MSTRIDE ? (SLICE + SBINS) : 2 * MROWS * MSTRIDE;
 constexpr float NEG_BIG = -1e30f;         // finite "no value yet" maximum
 
 constexpr unsigned ST_SOFTMAX = 0x10u, ST_LOAD = 0x100u, ST_MMA = 0x1000u, ST_DRAIN = 0x10000u;
 
 struct SmemCtl {
-  uint64_t slot_full[NSLOT];
-  uint64_t slot_empty[NSLOT];
+  uint64_t slot_full[NSLOT_MAX];
+  uint64_t slot_empty[NSLOT_MAX];
   uint64_t s_full[2];
   uint64_t s_free[2];
   uint64_t op_full[2];      // a query operand buffer is written (4 warp arrivals)
@@ -170,7 +173,8 @@ __device__ __forceinline__ void split_pack(float a, float b, uint32_t& hi, uint3
 // angles `cs` (continuous) or as they are (cs == nullptr).  128 threads.
 __device__ __forceinline__ void build_operand(uint8_t* op_hi, const float* __restrict__ src,
                                               const float2* __restrict__ cs, int tau) {
-  for (int task = tau; task < ROWS * 8; task += 128) {
+#pragma unroll
+  for (int task = tau; task < ROWS * 8; task += 128) {  // all loads issued together
     const int r = task >> 3, c = task & 7;
     const float* row = src + r * HD;
     const float4 a0 = *reinterpret_cast<const float4*>(row + 8 * c);
@@ -223,8 +227,13 @@ __global__ void __launch_bounds__(THREADS, 1)
   uint8_t* opnd = slots + NSLOT * TILE_BYTES;
   float* bins = reinterpret_cast<float*>(opnd + NOPND * QOP);
   float* vbin = bins;            // [SLICE]     pass 2
-  float* sbin = bins + SLICE;    // [4][SBINS]  pass 2
+  float* sbin = bins + SLICE;    // [SBINS]     pass 2
   SmemCtl* ctl = reinterpret_cast<SmemCtl*>(bins + BIN_FLOATS);
+
+  // key-tile ring: 3 slots, and in continuous mode (4 operands, not 6) a
+  // fourth slot in the operand space it leaves free
+  const int nslot = p.continuous ? NSLOT_MAX : NSLOT;
+  auto slot_at = [&](int k) { return k < NSLOT ? slots + k * TILE_BYTES : opnd + 4 * QOP; };
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   // the G heads of one KV group and slice are adjacent: they read the same keys
@@ -237,7 +246,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   const int64_t i_last = p.i_first + p.n_last - 1;
 
   if (threadIdx.x == 0) {
-    for (int k = 0; k < NSLOT; ++k) {
+    for (int k = 0; k < NSLOT_MAX; ++k) {
       mbar_init(&ctl->slot_full[k], 1);
       mbar_init(&ctl->slot_empty[k], 1);
     }
@@ -282,7 +291,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     fence_barrier_init();
   }
   if (PASS == 2)
-    for (int e = threadIdx.x; e < SLICE + 4 * SBINS; e += THREADS) bins[e] = 0.f;
+    for (int e = threadIdx.x; e < SLICE + SBINS; e += THREADS) bins[e] = 0.f;
   if (warp == WARP_MMA) {
     tmem_alloc(&ctl->tmem_base, TMEM_COLS);
     tmem_relinquish();
@@ -333,7 +342,6 @@ __global__ void __launch_bounds__(THREADS, 1)
         C[r] = st.y > 0.f ? st.x + __log2f(st.y) : 0.f;
       }
     }
-    float* sbw = sbin + warp * SBINS;  // this warp's copy of the slash bins
     Cursor it = first_item(ctl, p);
     for (int n = 0; n < N; ++n) {
       const int buf = n & 1;
@@ -353,35 +361,27 @@ __global__ void __launch_bounds__(THREADS, 1)
       // [-31, 63]: a0 (d = L - 32), a1 (d = L), a2 (d = L + 32).  At row r the
       // value p(r, (r - L) mod 32) is on one of lane L's diagonals.
       float a0 = 0.f, a1 = 0.f, a2 = 0.f;
+      // the rows of one half of S^T: online stats (pass 1) or probabilities,
+      // their vertical and diagonal sums (pass 2); MASKED applies [ra, rb)
+      auto rows_of_half = [&](const uint32_t* sv, const int half, auto masked) {
+        constexpr bool MASKED = decltype(masked)::value;
 #pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        uint32_t sv[32];
-        tmem_ld32(tbase + lane_off + static_cast<uint32_t>(buf * ROWS + half * 32), sv);
-        if (half == 1) {
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&ctl->s_free[buf]);
-        }
-        if (PASS == 1) {
-#pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            const int r = half * 32 + e;
+        for (int e = 0; e < 32; ++e) {
+          const int r = half * 32 + e;
+          if (PASS == 1) {
             float x = __uint_as_float(sv[e]);
-            if (!full) x = (r >= ra && r < rb) ? x : -INFINITY;
+            if (MASKED) x = (r >= ra && r < rb) ? x : -INFINITY;
             const float d = x - m[r];  // m is finite: a masked x gives -inf, t = 0
             const float t = ex2_approx(-fabsf(d));
             const bool up = d > 0.f;
             l[r] = up ? fmaf(l[r], t, 1.f) : l[r] + t;
             m[r] = up ? x : m[r];
-          }
-        } else {
-#pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            const int r = half * 32 + e;
+          } else {
             float pr = ex2_approx(__uint_as_float(sv[e]) - C[r]);
-            if (!full) pr = (r >= ra && r < rb) ? pr : 0.f;
+            if (MASKED) pr = (r >= ra && r < rb) ? pr : 0.f;
             vsum += pr;
-            const float v = __shfl_sync(0xffffffffu, pr, (r - lane) & 31);
+            // source lane (r - L) mod 32: the shuffle takes the index mod 32
+            const float v = __shfl_sync(0xffffffffu, pr, r - lane);
             if (r < 32) {
               if (lane <= r) a1 += v; else a0 += v;
             } else {
@@ -389,16 +389,33 @@ __global__ void __launch_bounds__(THREADS, 1)
             }
           }
         }
-      }
+      };
+      // one version per case, so no branch sits between the rows
+      auto item_rows = [&](auto masked) {
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+          uint32_t sv[32];
+          tmem_ld32(tbase + lane_off + static_cast<uint32_t>(buf * ROWS + half * 32), sv);
+          if (half == 1) {
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&ctl->s_free[buf]);
+          }
+          rows_of_half(sv, half, masked);
+        }
+      };
+      if (full)
+        item_rows(std::false_type{});
+      else
+        item_rows(std::true_type{});
       if (PASS == 2) {
         vbin[j - ka] += vsum;  // key j is always this thread's
         // bin of diagonal d: offset i - j minus the slice's smallest offset,
         // (ka + SLICE - 1 - j_t) + r = (ka + SLICE - 1 - j_0) + d
-        float* bw = sbw + (ka + SLICE - 1 - (static_cast<int64_t>(it.kt) * BN + warp * 32));
-        __syncwarp();  // the previous item's updates by other lanes are visible
-        if (lane > 0) bw[lane - 32] += a0;
-        bw[lane] += a1;
-        bw[lane + 32] += a2;
+        float* bw = sbin + (ka + SLICE - 1 - (static_cast<int64_t>(it.kt) * BN + warp * 32));
+        if (lane > 0) atomicAdd(&bw[lane - 32], a0);
+        atomicAdd(&bw[lane], a1);
+        atomicAdd(&bw[lane + 32], a2);
       }
 
       // continuous: the last item of chunk c frees its operand buffer for c + 2
@@ -452,7 +469,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       }
       const int64_t o0 = p.i_first - (ka + SLICE - 1);
       for (int e = tau; e < SBINS; e += 128) {
-        const float v = (sbin[e] + sbin[SBINS + e]) + (sbin[2 * SBINS + e] + sbin[3 * SBINS + e]);
+        const float v = sbin[e];
         const int64_t o = o0 + e;
         if (v != 0.f && o >= 0 && o < p.Lk) atomicAdd(&srow[o], v);
       }
@@ -460,26 +477,26 @@ __global__ void __launch_bounds__(THREADS, 1)
   } else if (warp == WARP_LOAD) {
     // =========================================================== TMA producer
     if (lane == 0) {
-      int last[NSLOT];
+      int last[NSLOT_MAX];
 #pragma unroll
-      for (int k = 0; k < NSLOT; ++k) last[k] = -1;
+      for (int k = 0; k < NSLOT_MAX; ++k) last[k] = -1;
       Cursor it = first_item(ctl, p);
       for (int n = 0; n < N; ++n) {
-        const int slot = n % NSLOT, use = n / NSLOT;
+        const int slot = n % nslot, use = n / nslot;
         if (use > 0 &&
             !wait_bounded(&ctl->slot_empty[slot], static_cast<uint32_t>((use - 1) & 1),
                           abort_flag, p.status, p.timeout_ns, ST_LOAD))
           break;
-        uint8_t* dst = slots + slot * TILE_BYTES;
+        uint8_t* dst = slot_at(slot);
         mbar_arrive_expect_tx(&ctl->slot_full[slot], TILE_BYTES);
         tma_load_3d(dst, &tm_k, &ctl->slot_full[slot], 0, g, it.kt * BN);
         tma_load_3d(dst + HALF_BYTES, &tm_k, &ctl->slot_full[slot], 64, g, it.kt * BN);
         last[slot] = n;
         next_item(ctl, p, it);
       }
-      for (int k = 0; k < NSLOT; ++k)
+      for (int k = 0; k < nslot; ++k)
         if (last[k] >= 0)
-          wait_drain(&ctl->slot_full[k], static_cast<uint32_t>((last[k] / NSLOT) & 1), p.status,
+          wait_drain(&ctl->slot_full[k], static_cast<uint32_t>((last[k] / nslot) & 1), p.status,
                      p.timeout_ns, ST_DRAIN);
     }
     __syncwarp();
@@ -493,7 +510,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       Cursor it = first_item(ctl, p);
       int64_t have = -1;  // the operand (class set or chunk) known to be written
       for (int n = 0; n < N && ok; ++n) {
-        const int slot = n % NSLOT;
+        const int slot = n % nslot;
         // operand readiness: DCA once; continuous once per chunk
         const int64_t need = p.continuous ? it.c : 0;
         if (need != have) {
@@ -503,7 +520,7 @@ __global__ void __launch_bounds__(THREADS, 1)
           if (!ok) break;
           have = need;
         }
-        ok = wait_spin(&ctl->slot_full[slot], static_cast<uint32_t>((n / NSLOT) & 1), abort_flag,
+        ok = wait_spin(&ctl->slot_full[slot], static_cast<uint32_t>((n / nslot) & 1), abort_flag,
                        p.status, p.timeout_ns, ST_MMA);
         if (!ok) break;
         if (n >= 2) {
@@ -513,7 +530,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         }
         tc_fence_after();
         const int op = p.continuous ? 2 * (it.v & 1) : 2 * it.v;
-        const uint64_t dk = dk0 + static_cast<uint64_t>((slot * TILE_BYTES) >> 4);
+        const uint64_t dk = dk0 + static_cast<uint64_t>((slot_at(slot) - slots) >> 4);
         const uint32_t d_tmem = tbase + static_cast<uint32_t>((n & 1) * ROWS);
 #pragma unroll
         for (int part = 0; part < 2; ++part) {  // hi, then lo

@@ -134,3 +134,33 @@ def test_continuous_and_dca_selections_differ_across_chunks():
     b = select_on_gpu(w, 64, 64, 64, False)
     diff = sum(len(set(x.tolist()) ^ set(y.tolist())) for x, y in zip(a[5] + a[6], b[5] + b[6]))
     assert diff > 0
+
+
+@pytest.mark.gpu
+def test_exact_ties_take_the_smaller_index():
+    """Equal cached keys of one class for every row score exactly alike (on
+    both sides); a top-k that cuts through them takes the smaller indices,
+    the oracle's rule.  Key 100 is made a sink and copied to 612, 1124, 1636
+    (same j mod s, all inter-chunk for rows in chunk 5)."""
+    w = wl("sel_ties", 3000, 2, 1, 512, 64, 1024)
+    q, k, v = generate(w, device=DEV, seed=5)
+    dup = [100, 612, 1124, 1636]
+    k[100] = (k[100].float() * 8).to(k.dtype)
+    for j in dup[1:]:
+        k[j] = k[100]
+    kw = dict(chunk_size=w.chunk_size, local_window=w.local_window,
+              pretrain_window=w.pretrain_window)
+    ws = dca.Workspace(w.L, w.Hq, w.Hkv, 128, w.chunk_size, w.local_window, w.pretrain_window,
+                       q.dtype, DEV)
+    dca.prepare(k, kv_len=w.L, k_rows_valid=0, rope_base=w.rope_base, workspace=ws, **kw)
+    sp = dca.SparseWorkspace(w.L, w.Hq, 8, 8, DEV)
+    vert, _ = oracle.vs_scores(q.cpu(), k.cpu(), n_last=64, continuous=False, **w.params())
+    for n_v in (1, 2, 3):
+        dca.sparse_select(q, v, q_start=0, kv_len=w.L, rope_base=w.rope_base,
+                          yarn_scale=w.yarn_scale, n_vertical=n_v, n_slash=4, n_last=64,
+                          continuous=False, workspace=ws, sparse=sp, **kw)
+        V, _ = dca.sparse_pattern_get(sp, w.Hq)
+        for h in range(w.Hq):
+            assert vert[h][dup[0]] == vert[h][dup[3]] and set(oracle.topk(vert[h], 4)) == set(dup)
+            assert V[h].tolist() == dup[:n_v], (n_v, h, V[h])
+            assert oracle.topk(vert[h], n_v).tolist() == dup[:n_v]
