@@ -18,20 +18,23 @@
 //
 // Two passes over the same items:
 //   1  per thread and row an online (max, sum of 2^(x - max)) over its keys,
-//      merged over the CTA's 128 threads and written per (head, slice, row);
+//      merged over the row's 128 key threads and written per (head, slice,
+//      row);
 //      sel_stats_kernel merges the slices;
 //   2  p = 2^(x - M) / L: the per-key sum over the rows (vertical) into a
 //      shared-memory bin per key of the slice; the sums along the diagonals
 //      i - j (slash) in registers, one lane per diagonal class mod 32 fed by a
-//      rotating shuffle, then into a bin per offset; the bins are stored /
-//      added to the score arrays once per CTA.
+//      rotating shuffle, then once per item into a bin per offset; the bins
+//      are stored / added to the score arrays once per CTA.
 // The rows of an item's class (and of causality) are one contiguous range
 // per key (class_row_range), so masking is a range test.
-// Warps: 0-3 softmax, 4 TMA producer (ring of 3 -- continuous positions: 4 --
-// 32 KiB key tiles, no multicast), 5 MMA issuer.  Every mbarrier wait is bounded; on timeout the
-// CTA raises its abort flag, ORs a code into the status word, drains its
-// copies and MMAs, frees TMEM and exits.  The softmax warps' own barriers
-// (bar.sync 1, 128) are reached by all four warps on every path.
+// Warps: 0-7 softmax (two per SMSP: warp w reads the TMEM lane quarter
+// w % 4, i.e. 32 keys, and rows 32 (w / 4) .. + 31), 8 TMA producer (ring of
+// 3 -- continuous positions: 4 -- 32 KiB key tiles, no multicast), 9 MMA
+// issuer.  Every mbarrier wait is bounded; on timeout the CTA raises its abort
+// flag, ORs a code into the status word, drains its copies and MMAs, frees
+// TMEM and exits.  The softmax warps' own barriers (bar.sync 1, 256) are
+// reached by all eight warps on every path.
 #include <cuda_bf16.h>
 #include <math.h>
 
@@ -52,11 +55,14 @@ constexpr int TILE_BYTES = 32768, HALF_BYTES = 16384;
 constexpr int QOP = ROWS * HD * 2;        // 16 KiB: one bf16 query operand
 constexpr int QOP_HALF = ROWS * 128;      // its 64-column block
 constexpr int NOPND = 6;                  // DCA: 3 classes x (hi, lo); continuous: 2 x (hi, lo)
-constexpr int THREADS = 192;
-constexpr int WARP_LOAD = 4, WARP_MMA = 5;
-constexpr uint32_t TMEM_COLS = 128;       // two S^T buffers of 64 columns
+constexpr int SM_WARPS = 8;               // softmax warps: 2 per SMSP
+constexpr int SM_THREADS = 32 * SM_WARPS;
+constexpr int THREADS = SM_THREADS + 64;
+constexpr int WARP_LOAD = SM_WARPS, WARP_MMA = SM_WARPS + 1;
+constexpr int NSBUF = 4;                  // S^T buffers in TMEM (the MMA runs up to 3 items ahead)
+constexpr uint32_t TMEM_COLS = NSBUF * ROWS;
 constexpr int SBINS = SLICE + ROWS;       // offsets i - j met by a slice
-constexpr int MSTRIDE = 136;              // row stride of the merge buffers (conflict-free)
+constexpr int MSTRIDE = 144;              // row stride of the merge buffers (conflict-free)
 constexpr int MROWS = 16;                 // rows per merge round
 // pass 2: vertical bins [SLICE] (key j is always updated by one thread) and
 // the slash bins [SBINS] (each lane adds its three diagonal sums once per
@@ -70,9 +76,9 @@ constexpr unsigned ST_SOFTMAX = 0x10u, ST_LOAD = 0x100u, ST_MMA = 0x1000u, ST_DR
 struct SmemCtl {
   uint64_t slot_full[NSLOT_MAX];
   uint64_t slot_empty[NSLOT_MAX];
-  uint64_t s_full[2];
-  uint64_t s_free[2];
-  uint64_t op_full[2];      // a query operand buffer is written (4 warp arrivals)
+  uint64_t s_full[NSBUF];
+  uint64_t s_free[NSBUF];
+  uint64_t op_full[2];      // a query operand buffer is written (one arrival per softmax warp)
   uint64_t drain;
   uint32_t tmem_base;
   int abort;
@@ -86,6 +92,7 @@ struct SmemCtl {
 constexpr size_t SMEM_BYTES =
     1024 + NSLOT * TILE_BYTES + NOPND * QOP + sizeof(float) * BIN_FLOATS + sizeof(SmemCtl);
 static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+static_assert(SLICE % BN == 0 && SLICE / BN <= 32, "one counting lane per k-tile of a slice");
 
 struct Params {
   const float* qv;          // [Hq][nvar][ROWS][HD] rotated query rows, log2 units
@@ -100,7 +107,7 @@ struct Params {
   unsigned long long timeout_ns;
 };
 
-__device__ __forceinline__ void softmax_bar() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+__device__ __forceinline__ void softmax_bar() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
 
 // The work item cursor: DCA walks the class ranges (INTER, SUCC, INTRA), the
 // continuous mode the (k-tile, chunk) pairs of the slice in key order.
@@ -170,11 +177,12 @@ __device__ __forceinline__ void split_pack(float a, float b, uint32_t& hi, uint3
 
 // Query operand pair (hi at op_hi, lo at op_hi + QOP): K-major, 128-byte
 // swizzle, from the fp32 rows `src` [ROWS][HD], rotated back by the chunk
-// angles `cs` (continuous) or as they are (cs == nullptr).  128 threads.
+// angles `cs` (continuous) or as they are (cs == nullptr).  The softmax warps'
+// 256 threads.
 __device__ __forceinline__ void build_operand(uint8_t* op_hi, const float* __restrict__ src,
                                               const float2* __restrict__ cs, int tau) {
 #pragma unroll
-  for (int task = tau; task < ROWS * 8; task += 128) {  // all loads issued together
+  for (int task = tau; task < ROWS * 8; task += 256) {  // all loads issued together
     const int r = task >> 3, c = task & 7;
     const float* row = src + r * HD;
     const float4 a0 = *reinterpret_cast<const float4*>(row + 8 * c);
@@ -245,37 +253,28 @@ __global__ void __launch_bounds__(THREADS, 1)
   const int64_t ka = static_cast<int64_t>(sl) * SLICE;
   const int64_t i_last = p.i_first + p.n_last - 1;
 
-  if (threadIdx.x == 0) {
-    for (int k = 0; k < NSLOT_MAX; ++k) {
-      mbar_init(&ctl->slot_full[k], 1);
-      mbar_init(&ctl->slot_empty[k], 1);
-    }
-    for (int k = 0; k < 2; ++k) {
-      mbar_init(&ctl->s_full[k], 1);
-      mbar_init(&ctl->s_free[k], 4);
-      mbar_init(&ctl->op_full[k], 4);
-    }
-    mbar_init(&ctl->drain, 1);
-    ctl->abort = 0;
+  if (warp == 0) {
+    // work list of the slice; continuous: per k-tile (one lane each) the
+    // chunks its causal keys meet, summed over the warp
     int n = 0;
     if (p.continuous) {
       int64_t kend = ka + SLICE;
       if (kend > i_last + 1) kend = i_last + 1;
       if (kend > p.Lk) kend = p.Lk;
-      ctl->kend = kend;
-      ctl->kt0 = static_cast<int>(ka / BN);
-      if (kend > ka) {
-        ctl->c_first = ka / p.s;
-        ctl->c_last = (kend - 1) / p.s;
-        // items: per k-tile, the chunks its causal keys meet
-        for (int64_t t0 = ka; t0 < kend; t0 += BN) {
-          const int64_t t1 = (t0 + BN < kend ? t0 + BN : kend) - 1;
-          n += static_cast<int>(t1 / p.s - t0 / p.s + 1);
-        }
-      } else {
-        ctl->c_first = ctl->c_last = 0;
+      const uint32_t s32 = static_cast<uint32_t>(p.s);
+      const int64_t t0 = ka + static_cast<int64_t>(lane) * BN;
+      if (lane < SLICE / BN && t0 < kend) {
+        const int64_t t1 = (t0 + BN < kend ? t0 + BN : kend) - 1;
+        n = static_cast<int>(static_cast<uint32_t>(t1) / s32 - static_cast<uint32_t>(t0) / s32 + 1);
       }
-    } else {
+      n = __reduce_add_sync(0xffffffffu, n);
+      if (lane == 0) {
+        ctl->kend = kend;
+        ctl->kt0 = static_cast<int>(ka / BN);
+        ctl->c_first = kend > ka ? ka / p.s : 0;
+        ctl->c_last = kend > ka ? (kend - 1) / p.s : 0;
+      }
+    } else if (lane == 0) {
       const TilePlan P = make_plan(p.i_first, i_last, p.s, p.w, BN, p.reading);
       const int t0 = static_cast<int>(ka / BN), t1 = static_cast<int>((ka + SLICE) / BN);
       for (int c = 0; c < 3; ++c) {
@@ -287,8 +286,21 @@ __global__ void __launch_bounds__(THREADS, 1)
         n += b - a;
       }
     }
-    ctl->n_items = n;
-    fence_barrier_init();
+    if (lane == 0) {
+      for (int k = 0; k < NSLOT_MAX; ++k) {
+        mbar_init(&ctl->slot_full[k], 1);
+        mbar_init(&ctl->slot_empty[k], 1);
+      }
+      for (int k = 0; k < NSBUF; ++k) {
+        mbar_init(&ctl->s_full[k], 1);
+        mbar_init(&ctl->s_free[k], SM_WARPS);
+      }
+      for (int k = 0; k < 2; ++k) mbar_init(&ctl->op_full[k], SM_WARPS);
+      mbar_init(&ctl->drain, 1);
+      ctl->abort = 0;
+      ctl->n_items = n;
+      fence_barrier_init();
+    }
   }
   if (PASS == 2)
     for (int e = threadIdx.x; e < SLICE + SBINS; e += THREADS) bins[e] = 0.f;
@@ -304,19 +316,23 @@ __global__ void __launch_bounds__(THREADS, 1)
   volatile int* abort_flag = &ctl->abort;
   const int N = ctl->n_items;
 
-  if (warp < 4) {
+  if (warp < SM_WARPS) {
     // =========================================================== softmax warps
-    const int tau = warp * 32 + lane;
-    const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+    // warp w: keys 32 (w % 4) + lane of each tile (its TMEM lane quarter) and
+    // rows r0 = 32 (w / 4) .. r0 + 31 of the estimate; two warps per SMSP
+    const int kq = warp & 3, r0 = (warp >> 2) * 32;
+    const int tau = kq * 32 + lane;  // key within the tile
+    const int stid = threadIdx.x;    // 0 .. 255
+    const uint32_t lane_off = static_cast<uint32_t>(kq * 32) << 16;
     const float* qh = p.qv + static_cast<int64_t>(h) * (p.continuous ? 1 : 3) * ROWS * HD;
     if (N > 0) {
       if (p.continuous) {
-        build_operand(opnd, qh, p.crot + ctl->c_first * (HD / 2), tau);
+        build_operand(opnd, qh, p.crot + ctl->c_first * (HD / 2), stid);
         if (ctl->c_first + 1 <= ctl->c_last)
-          build_operand(opnd + 2 * QOP, qh, p.crot + (ctl->c_first + 1) * (HD / 2), tau);
+          build_operand(opnd + 2 * QOP, qh, p.crot + (ctl->c_first + 1) * (HD / 2), stid);
       } else {
         for (int v = 0; v < 3; ++v)
-          build_operand(opnd + 2 * v * QOP, qh + v * ROWS * HD, nullptr, tau);
+          build_operand(opnd + 2 * v * QOP, qh + v * ROWS * HD, nullptr, stid);
       }
       fence_proxy_async_smem();
       __syncwarp();
@@ -328,94 +344,80 @@ __global__ void __launch_bounds__(THREADS, 1)
 
     // pass 1: running (max, sum) per row; pass 2: C_r = M_r + log2 L_r, so
     // p = 2^(x - C_r)
-    constexpr int NR1 = PASS == 1 ? ROWS : 1, NR2 = PASS == 2 ? ROWS : 1;
+    constexpr int NR1 = PASS == 1 ? 32 : 1, NR2 = PASS == 2 ? 32 : 1;
     float m[NR1], l[NR1], C[NR2];
 #pragma unroll
-    for (int r = 0; r < NR1; ++r) {
-      m[r] = NEG_BIG;
-      l[r] = 0.f;
+    for (int e = 0; e < NR1; ++e) {
+      m[e] = NEG_BIG;
+      l[e] = 0.f;
     }
     if (PASS == 2) {
 #pragma unroll
-      for (int r = 0; r < NR2; ++r) {
-        const float2 st = p.stats[h * ROWS + r];
-        C[r] = st.y > 0.f ? st.x + __log2f(st.y) : 0.f;
+      for (int e = 0; e < NR2; ++e) {
+        const float2 st = p.stats[h * ROWS + r0 + e];
+        C[e] = st.y > 0.f ? st.x + __log2f(st.y) : 0.f;
       }
     }
     Cursor it = first_item(ctl, p);
     for (int n = 0; n < N; ++n) {
-      const int buf = n & 1;
-      if (!wait_warp(&ctl->s_full[buf], static_cast<uint32_t>((n >> 1) & 1), abort_flag, p.status,
-                     p.timeout_ns, ST_SOFTMAX, lane))
+      const int buf = n % NSBUF;
+      if (!wait_warp(&ctl->s_full[buf], static_cast<uint32_t>((n / NSBUF) & 1), abort_flag,
+                     p.status, p.timeout_ns, ST_SOFTMAX, lane))
         break;
       tc_fence_after();
+      uint32_t sv[32];
+      tmem_ld32(tbase + lane_off + static_cast<uint32_t>(buf * ROWS + r0), sv);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&ctl->s_free[buf]);
+
       const int64_t j = static_cast<int64_t>(it.kt) * BN + tau;
       int ra, rb;
       class_row_range(j, p.i_first, p.n_last, p.Lk, p.s, p.w, p.reading,
                       p.continuous ? -1 : it.v, p.continuous ? it.c : -1, &ra, &rb);
-      // every row of every lane valid: no masks (the common case)
-      const bool full = __all_sync(0xffffffffu, ra == 0 && rb == ROWS);
+      // every row of the warp valid in every lane: no masks (the common case)
+      const bool full = __all_sync(0xffffffffu, ra <= r0 && rb >= r0 + 32);
       float vsum = 0.f;
-      // slash: the warp's 32 keys and 64 rows meet the diagonals d = r - t,
-      // t = lane of the key; lane L owns those with d = L (mod 32), d in
-      // [-31, 63]: a0 (d = L - 32), a1 (d = L), a2 (d = L + 32).  At row r the
-      // value p(r, (r - L) mod 32) is on one of lane L's diagonals.
-      float a0 = 0.f, a1 = 0.f, a2 = 0.f;
-      // the rows of one half of S^T: online stats (pass 1) or probabilities,
-      // their vertical and diagonal sums (pass 2); MASKED applies [ra, rb)
-      auto rows_of_half = [&](const uint32_t* sv, const int half, auto masked) {
+      // slash: the warp's 32 keys and 32 rows meet the diagonals d = r - t
+      // (t = lane of the key); lane L owns d = r0 + L - 32 (a0) and r0 + L
+      // (a1).  At local row e the value p(r0 + e, (e - L) mod 32) is on one of
+      // them: a1 when L <= e.
+      float a0 = 0.f, a1 = 0.f;
+      auto rows = [&](auto masked) {
         constexpr bool MASKED = decltype(masked)::value;
 #pragma unroll
         for (int e = 0; e < 32; ++e) {
-          const int r = half * 32 + e;
+          const int r = r0 + e;
           if (PASS == 1) {
             float x = __uint_as_float(sv[e]);
             if (MASKED) x = (r >= ra && r < rb) ? x : -INFINITY;
-            const float d = x - m[r];  // m is finite: a masked x gives -inf, t = 0
+            const float d = x - m[e];  // m is finite: a masked x gives -inf, t = 0
             const float t = ex2_approx(-fabsf(d));
             const bool up = d > 0.f;
-            l[r] = up ? fmaf(l[r], t, 1.f) : l[r] + t;
-            m[r] = up ? x : m[r];
+            l[e] = up ? fmaf(l[e], t, 1.f) : l[e] + t;
+            m[e] = up ? x : m[e];
           } else {
-            float pr = ex2_approx(__uint_as_float(sv[e]) - C[r]);
+            float pr = ex2_approx(__uint_as_float(sv[e]) - C[e]);
             if (MASKED) pr = (r >= ra && r < rb) ? pr : 0.f;
             vsum += pr;
-            // source lane (r - L) mod 32: the shuffle takes the index mod 32
-            const float v = __shfl_sync(0xffffffffu, pr, r - lane);
-            if (r < 32) {
-              if (lane <= r) a1 += v; else a0 += v;
-            } else {
-              if (lane <= r - 32) a2 += v; else a1 += v;
-            }
+            // source lane (e - L) mod 32: the shuffle takes the index mod 32
+            const float v = __shfl_sync(0xffffffffu, pr, e - lane);
+            if (lane <= e) a1 += v; else a0 += v;
           }
         }
       };
       // one version per case, so no branch sits between the rows
-      auto item_rows = [&](auto masked) {
-#pragma unroll
-        for (int half = 0; half < 2; ++half) {
-          uint32_t sv[32];
-          tmem_ld32(tbase + lane_off + static_cast<uint32_t>(buf * ROWS + half * 32), sv);
-          if (half == 1) {
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&ctl->s_free[buf]);
-          }
-          rows_of_half(sv, half, masked);
-        }
-      };
       if (full)
-        item_rows(std::false_type{});
+        rows(std::false_type{});
       else
-        item_rows(std::true_type{});
+        rows(std::true_type{});
       if (PASS == 2) {
-        vbin[j - ka] += vsum;  // key j is always this thread's
+        atomicAdd(&vbin[j - ka], vsum);  // the two row halves of key j
         // bin of diagonal d: offset i - j minus the slice's smallest offset,
         // (ka + SLICE - 1 - j_t) + r = (ka + SLICE - 1 - j_0) + d
-        float* bw = sbin + (ka + SLICE - 1 - (static_cast<int64_t>(it.kt) * BN + warp * 32));
+        float* bw = sbin + (ka + SLICE - 1 - (static_cast<int64_t>(it.kt) * BN + kq * 32)) + r0;
         if (lane > 0) atomicAdd(&bw[lane - 32], a0);
         atomicAdd(&bw[lane], a1);
-        atomicAdd(&bw[lane + 32], a2);
       }
 
       // continuous: the last item of chunk c frees its operand buffer for c + 2
@@ -424,7 +426,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         next_item(ctl, p, it);
         if ((n + 1 == N || it.c != c) && c + 2 <= ctl->c_last) {
           build_operand(opnd + 2 * static_cast<int>((c - ctl->c_first) & 1) * QOP, qh,
-                        p.crot + (c + 2) * (HD / 2), tau);
+                        p.crot + (c + 2) * (HD / 2), stid);
           fence_proxy_async_smem();
           __syncwarp();
           if (lane == 0) mbar_arrive(&ctl->op_full[(c - ctl->c_first) & 1]);
@@ -436,39 +438,43 @@ __global__ void __launch_bounds__(THREADS, 1)
 
     // ---- per-CTA results (every softmax warp runs this, whatever happened)
     if (PASS == 1) {
+      // per row over the 128 keys: 4 rounds of 8 rows of each half; 16
+      // threads per row each merge 8 entries, then a 16-lane shuffle merge
       float* mb = bins;
       float* lb = bins + MROWS * MSTRIDE;
-      const int rr = tau >> 3, q = tau & 7;
+      const int rr = stid >> 4, q = stid & 15;
 #pragma unroll
-      for (int round = 0; round < ROWS / MROWS; ++round) {
+      for (int round = 0; round < 4; ++round) {
         if (round > 0) softmax_bar();  // the previous round's reads are done
 #pragma unroll
-        for (int e = 0; e < MROWS; ++e) {
-          mb[e * MSTRIDE + tau] = m[round * MROWS + e];
-          lb[e * MSTRIDE + tau] = l[round * MROWS + e];
+        for (int e = 0; e < 8; ++e) {
+          mb[((r0 >> 2) + e) * MSTRIDE + tau] = m[round * 8 + e];
+          lb[((r0 >> 2) + e) * MSTRIDE + tau] = l[round * 8 + e];
         }
         softmax_bar();
         float2 acc = make_float2(NEG_BIG, 0.f);
 #pragma unroll
-        for (int e = 0; e < 128 / 8; ++e)
-          acc = merge_stat(acc, make_float2(mb[rr * MSTRIDE + q + 8 * e], lb[rr * MSTRIDE + q + 8 * e]));
+        for (int e = 0; e < 8; ++e)
+          acc = merge_stat(acc, make_float2(mb[rr * MSTRIDE + q + 16 * e], lb[rr * MSTRIDE + q + 16 * e]));
 #pragma unroll
-        for (int off = 1; off < 8; off <<= 1)
+        for (int off = 1; off < 16; off <<= 1)
           acc = merge_stat(acc, make_float2(__shfl_xor_sync(0xffffffffu, acc.x, off),
                                             __shfl_xor_sync(0xffffffffu, acc.y, off)));
-        if (q == 0)
-          p.part[(static_cast<int64_t>(h) * p.n_slices + sl) * ROWS + round * MROWS + rr] = acc;
+        if (q == 0) {
+          const int row = (rr >> 3) * 32 + round * 8 + (rr & 7);
+          p.part[(static_cast<int64_t>(h) * p.n_slices + sl) * ROWS + row] = acc;
+        }
       }
     } else {
       softmax_bar();  // every bin update is done
       float* vrow = p.vert + static_cast<int64_t>(h) * p.Lk;
       float* srow = p.slash + static_cast<int64_t>(h) * p.Lk;
-      for (int e = tau; e < SLICE; e += 128) {
+      for (int e = stid; e < SLICE; e += SM_THREADS) {
         const int64_t jj = ka + e;
         if (jj < p.Lk) vrow[jj] = vbin[e];
       }
       const int64_t o0 = p.i_first - (ka + SLICE - 1);
-      for (int e = tau; e < SBINS; e += 128) {
+      for (int e = stid; e < SBINS; e += SM_THREADS) {
         const float v = sbin[e];
         const int64_t o = o0 + e;
         if (v != 0.f && o >= 0 && o < p.Lk) atomicAdd(&srow[o], v);
@@ -523,15 +529,15 @@ __global__ void __launch_bounds__(THREADS, 1)
         ok = wait_spin(&ctl->slot_full[slot], static_cast<uint32_t>((n / nslot) & 1), abort_flag,
                        p.status, p.timeout_ns, ST_MMA);
         if (!ok) break;
-        if (n >= 2) {
-          ok = wait_spin(&ctl->s_free[n & 1], static_cast<uint32_t>(((n - 2) >> 1) & 1),
+        if (n >= NSBUF) {
+          ok = wait_spin(&ctl->s_free[n % NSBUF], static_cast<uint32_t>(((n - NSBUF) / NSBUF) & 1),
                          abort_flag, p.status, p.timeout_ns, ST_MMA);
           if (!ok) break;
         }
         tc_fence_after();
         const int op = p.continuous ? 2 * (it.v & 1) : 2 * it.v;
         const uint64_t dk = dk0 + static_cast<uint64_t>((slot_at(slot) - slots) >> 4);
-        const uint32_t d_tmem = tbase + static_cast<uint32_t>((n & 1) * ROWS);
+        const uint32_t d_tmem = tbase + static_cast<uint32_t>((n % NSBUF) * ROWS);
 #pragma unroll
         for (int part = 0; part < 2; ++part) {  // hi, then lo
           const uint64_t dq = dq0 + static_cast<uint64_t>(((op + part) * QOP) >> 4);
@@ -542,7 +548,7 @@ __global__ void __launch_bounds__(THREADS, 1)
             mma_ss(d_tmem, dk + a_off, dq + b_off, id, (part > 0 || kk > 0) ? 1u : 0u);
           }
         }
-        mma_commit(&ctl->s_full[n & 1]);
+        mma_commit(&ctl->s_full[n % NSBUF]);
         mma_commit(&ctl->slot_empty[slot]);
         next_item(ctl, p, it);
       }
