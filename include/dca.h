@@ -331,6 +331,22 @@ int dca_plan_items(int64_t i0, int64_t i_last, int64_t tile_rows, int64_t chunk_
                    int max_items);
 
 /*
+ * Host-side introspection of the key selection's masking (no GPU needed):
+ * for key j and the block of estimate rows at positions i_first + r,
+ * 0 <= r < n_rows (n_rows <= 64), writes to range[0..1] the rows [ra, rb) that
+ * pair with j -- causal (j <= i), j < kv_len, and either of work-list class
+ * `cls` (0, 1, 2 as in dca_plan_items; cls >= 0) or, with cls = -1, with
+ * j in key chunk `chunk` (j / chunk_size == chunk; continuous positions).
+ * These rows are one contiguous range because a key's class does not
+ * decrease as i grows.  Returns DCA_OK, or DCA_ERR_ARG (0 <= j < 2^31,
+ * i_first >= 0, 1 <= n_rows <= 64, chunk_size >= 1, 0 <= local_window <=
+ * chunk_size, cls in -1..2, range not NULL).
+ */
+int dca_class_rows(int64_t j, int64_t i_first, int n_rows, int64_t kv_len, int64_t chunk_size,
+                   int64_t local_window, int window_reading, int cls, int64_t chunk,
+                   int32_t* range);
+
+/*
  * No-allocation one-shot prefill (an addition for integrators; the pages on
  * DCA have no counterpart).  For callers that cannot call cudaMalloc: e.g. a
  * serving process that hands all free HBM to its own pool at start-up, where a

@@ -38,6 +38,7 @@ SIGNATURES = {
     "dca_prefill_host": (_i32, [_vp, _vp, _vp, _vp, _i64, _i64, _i32, _i32, _i32, _i64, _i64,
                                 _i64, _dbl, _dbl, _i32, _vp, _sz, _vp]),
     "dca_plan_items": (_i32, [_i64, _i64, _i64, _i64, _i64, _i32, _i32, _vp, _i32]),
+    "dca_class_rows": (_i32, [_i64, _i64, _i32, _i64, _i64, _i64, _i32, _i32, _i64, _vp]),
     "dca_prefill_chunked_ex": (_i32, [_vp, _vp, _vp, _vp, _i64, _i64, _i64, _i32, _i32, _i32, _i64,
                                       _i64, _i64, _dbl, _dbl, _i32, _vp, _vp, _sz, _vp]),
     "dca_attend_ex": (_i32, [_vp, _vp, _vp, _i64, _i64, _i64, _i32, _i32, _i32, _i64, _i64, _i64,

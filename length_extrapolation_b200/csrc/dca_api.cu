@@ -622,6 +622,22 @@ int dca_sparse_attend(const dca_sparse_config* cfg, const void* q_block, const v
   return e == cudaSuccess ? DCA_OK : DCA_ERR_CUDA;
 }
 
+int dca_class_rows(int64_t j, int64_t i_first, int n_rows, int64_t kv_len, int64_t chunk_size,
+                   int64_t local_window, int window_reading, int cls, int64_t chunk,
+                   int32_t* range) {
+  if (j < 0 || j > (1LL << 31) - 1 || i_first < 0 || n_rows < 1 || n_rows > 64 ||
+      chunk_size < 1 || local_window < 0 || local_window > chunk_size || cls < -1 || cls > 2 ||
+      range == nullptr ||
+      (window_reading != DCA_WINDOW_QUERY_OFFSET && window_reading != DCA_WINDOW_TRUE_DISTANCE))
+    return DCA_ERR_ARG;
+  int ra, rb;
+  dca::class_row_range(j, i_first, n_rows, kv_len, chunk_size, local_window, window_reading, cls,
+                       chunk, &ra, &rb);
+  range[0] = ra;
+  range[1] = rb;
+  return DCA_OK;
+}
+
 int dca_sparse_plan_items(const int32_t* v_idx, int64_t n_v, const int32_t* s_off, int64_t n_s,
                           int64_t i0, int64_t i_last, int64_t chunk_size, int64_t local_window,
                           int window_reading, int32_t* items, int max_items) {

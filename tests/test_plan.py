@@ -117,3 +117,45 @@ def test_big_config_phase_counts(lib):
     assert n_succ == s // 128
     assert n_intra == (L - 5 * s) // 128
     assert items[:, 2].sum() == len(items) - 1
+
+
+def test_selection_row_ranges_brute_force(lib):
+    """The key selection masks each key's rows to one contiguous range per
+    work-list class (or key chunk, continuous positions); against the
+    per-pair class over random small configurations."""
+    rng = np.random.default_rng(7)
+    rg = (ctypes.c_int32 * 2)()
+    for _ in range(3000):
+        s = int(rng.integers(1, 300))
+        w = int(rng.integers(0, s + 1))
+        reading = int(rng.integers(0, 2))
+        n_rows = int(rng.integers(1, 65))
+        i_first = int(rng.integers(0, 2000))
+        kv_len = i_first + n_rows - int(rng.integers(0, n_rows)) if rng.random() < 0.3 \
+            else i_first + n_rows + int(rng.integers(0, 50))
+        j = int(rng.integers(0, i_first + 200))
+        cls = int(rng.integers(-1, 3))
+        chunk = j // s if rng.random() < 0.5 else int(rng.integers(0, 20))
+        assert lib.dca_class_rows(j, i_first, n_rows, kv_len, s, w, reading, cls, chunk, rg) == 0
+        ra, rb = rg[0], rg[1]
+        assert 0 <= ra <= rb <= n_rows
+        for r in range(n_rows):
+            i = i_first + r
+            want = j <= i and j < kv_len
+            want = want and (chunk_class(i, j, s, w, reading) == cls if cls >= 0 else j // s == chunk)
+            assert want == (ra <= r < rb), (s, w, reading, i_first, j, cls, r, ra, rb)
+
+
+def test_selection_row_ranges_reject(lib):
+    rg = (ctypes.c_int32 * 2)()
+    ok = dict(j=5, i_first=0, n_rows=8, kv_len=100, s=16, w=4, reading=0, cls=0, chunk=0)
+
+    def call(**kw):
+        a = dict(ok, **kw)
+        return lib.dca_class_rows(a["j"], a["i_first"], a["n_rows"], a["kv_len"], a["s"], a["w"],
+                                  a["reading"], a["cls"], a["chunk"], rg)
+    assert call() == 0
+    for bad in (dict(j=-1), dict(j=1 << 31), dict(n_rows=0), dict(n_rows=65), dict(s=0),
+                dict(w=17), dict(cls=3), dict(cls=-2), dict(reading=2), dict(i_first=-1)):
+        assert call(**bad) == N.DCA_ERR_ARG, bad
+    assert lib.dca_class_rows(5, 0, 8, 100, 16, 4, 0, 0, 0, None) == N.DCA_ERR_ARG
