@@ -19,7 +19,8 @@ LIB = os.path.join(HERE, "libdca_b200.so")
 SOURCES = ["dca_api.cu", "dca_prep.cu", "dca_fwd_sm100.cu", "dca_fwd_f32.cu", "dca_decode_sm100.cu",
            "dca_sparse_sm100.cu", "dca_sparse_prep.cu", "dca_select.cu", "dca_select_mma.cu",
            "dca_noalloc.cu"]
-HEADERS = ["dca_internal.h", "dca_plan.cuh", "dca_softmax.cuh", "dca_sparse_plan.cuh",
+HEADERS = ["dca_internal.h", "dca_plan.cuh", "dca_select_rows.cuh", "dca_softmax.cuh",
+           "dca_sparse_plan.cuh",
            "sm100_ptx.cuh"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 

@@ -11,6 +11,7 @@
 #include "../../include/dca.h"
 #include "dca_internal.h"
 #include "dca_plan.cuh"
+#include "dca_select_rows.cuh"
 #include "dca_sparse_plan.cuh"
 
 namespace {

@@ -42,6 +42,7 @@
 
 #include "dca_internal.h"
 #include "dca_plan.cuh"
+#include "dca_select_rows.cuh"
 #include "sm100_ptx.cuh"
 
 namespace dca {
