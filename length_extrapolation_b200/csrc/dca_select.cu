@@ -208,8 +208,11 @@ __global__ void __launch_bounds__(TK_THREADS)
       const uint32_t bits = __float_as_uint(sc[j]);
       if ((static_cast<uint64_t>(bits) >> top) == prefix) bin = static_cast<int>((bits >> shift) & (nbin - 1));
     }
-    const unsigned peers = __match_any_sync(0xffffffffu, bin);
-    if (bin >= 0 && lane == __ffs(peers) - 1) atomicAdd(&hist[bin], __popc(peers));
+    // after the first pass few scores match the prefix: most warps skip
+    if (__any_sync(0xffffffffu, bin >= 0)) {
+      const unsigned peers = __match_any_sync(0xffffffffu, bin);
+      if (bin >= 0 && lane == __ffs(peers) - 1) atomicAdd(&hist[bin], __popc(peers));
+    }
   }
   __syncthreads();
   int* g = a.hist + static_cast<int64_t>(row) * TK_BINS;
@@ -276,7 +279,12 @@ __global__ void __launch_bounds__(TK_THREADS)
 }
 
 // Ordered write of the selected indices of each span (ascending), their
-// bitmap bits; equal values are taken while the row still needs them.
+// bitmap bits; equal values are taken while the row still needs them.  The
+// span is walked in blocks of TK_THREADS x TK_PER scores, each thread owning
+// TK_PER consecutive ones, so two block scans per block (equal values before
+// the thread, selected before the thread) place everything.
+constexpr int TK_PER = 16;
+
 __global__ void __launch_bounds__(TK_THREADS)
     sel_topk_write_kernel(const TopkArgs a, SelectOut out) {
   __shared__ int warp_sums[32];
@@ -302,23 +310,50 @@ __global__ void __launch_bounds__(TK_THREADS)
   __syncthreads();
   int32_t* list = kind ? out.soff + h * out.s_cap : out.vidx + h * out.nv_cap;
   uint32_t* bitrow = (kind ? out.sbit : out.vbit) + h * out.wpr;
-  int64_t eq_seen = sh_eq_before, written = sh_start;
-  const int64_t j0 = static_cast<int64_t>(blockIdx.x) * a.span;
-  for (int64_t base = j0; base < j0 + a.span && base < a.Lk; base += TK_THREADS) {
-    const int64_t j = base + threadIdx.x;
-    const uint32_t bits = j < a.Lk ? __float_as_uint(topk_row(a, row)[j]) : 0u;
-    const int is_eq = (j < a.Lk && bits == T) ? 1 : 0;
-    int eq_total;
-    const int eq_before = block_scan(is_eq, warp_sums, eq_total);
-    const int sel = (j < a.Lk) && (bits > T || (is_eq && eq_seen + eq_before < need_eq)) ? 1 : 0;
-    int sel_total;
-    const int pos = block_scan(sel, warp_sums, sel_total);
-    if (sel) {
-      list[written + pos] = static_cast<int32_t>(j);
-      atomicOr(&bitrow[j >> 5], 1u << (j & 31));
+  const float* sc = topk_row(a, row);
+  const int64_t span0 = static_cast<int64_t>(blockIdx.x) * a.span;
+  const int64_t span1 = span0 + a.span < a.Lk ? span0 + a.span : a.Lk;
+  // blocks of TK_THREADS x TK_PER scores in order; thread t owns TK_PER
+  // consecutive scores of each, so (block, thread, element) is index order
+  for (int64_t c0 = span0; c0 < span1; c0 += TK_THREADS * TK_PER) {
+    const int64_t jt = c0 + static_cast<int64_t>(threadIdx.x) * TK_PER;
+    // this block's starting counts, read before thread 0 advances them
+    const int64_t eq_before = sh_eq_before, start = sh_start;
+    uint32_t bits[TK_PER];
+    int eq = 0;
+#pragma unroll
+    for (int e = 0; e < TK_PER; ++e) {
+      const int64_t j = jt + e;
+      bits[e] = j < span1 ? __float_as_uint(sc[j]) : 0u;
+      eq += (j < span1 && bits[e] == T) ? 1 : 0;
     }
-    eq_seen += eq_total;
-    written += sel_total;
+    int eq_total;
+    int64_t eq_seen = eq_before + block_scan(eq, warp_sums, eq_total);
+    uint32_t take = 0;  // bit e: element e selected
+#pragma unroll
+    for (int e = 0; e < TK_PER; ++e) {
+      const int64_t j = jt + e;
+      if (j < span1 && bits[e] > T) take |= 1u << e;
+      if (j < span1 && bits[e] == T) {
+        if (eq_seen < need_eq) take |= 1u << e;
+        ++eq_seen;
+      }
+    }
+    int sel_total;
+    int64_t pos = start + block_scan(__popc(take), warp_sums, sel_total);
+#pragma unroll
+    for (int e = 0; e < TK_PER; ++e) {
+      if (take & (1u << e)) {
+        const int64_t j = jt + e;
+        list[pos++] = static_cast<int32_t>(j);
+        atomicOr(&bitrow[j >> 5], 1u << (j & 31));
+      }
+    }
+    if (threadIdx.x == 0) {  // every thread read the counts before the scans' barriers
+      sh_eq_before = eq_before + eq_total;
+      sh_start = start + sel_total;
+    }
+    __syncthreads();
   }
 }
 
