@@ -84,6 +84,7 @@ struct SmemCtl {
   uint32_t tmem_base;
   int abort;
   int n_items;
+  int rot;                  // item order rotation (see Cursor)
   int lo[3], hi[3];         // DCA: k-tile range per class, clipped to the slice
   int kt0;                  // continuous: first k-tile of the slice
   int64_t kend;             // continuous: end of the slice's causal keys
@@ -119,18 +120,29 @@ struct Cursor {
   int64_t c;   // continuous: key chunk
 };
 
+// The G CTAs of a KV group walk the slice's items from different starting
+// points (item n is the list's item (n + rot) mod N, rot = hh N / G), so
+// they do not all ask L2 for the same key tile at once.  Continuous
+// positions rotate only a single-chunk slice (the operand buffers need the
+// chunks in order).
+__device__ __forceinline__ int phys_item(const SmemCtl* ctl, int n) {
+  const int q = n + ctl->rot;
+  return q >= ctl->n_items ? q - ctl->n_items : q;
+}
+
 __device__ __forceinline__ void dca_item(const SmemCtl* ctl, Cursor& it) {
   const int c2 = ctl->hi[CLS_INTER] - ctl->lo[CLS_INTER];
   const int c1 = ctl->hi[CLS_SUCC] - ctl->lo[CLS_SUCC];
-  if (it.n < c2) {
+  const int q = phys_item(ctl, it.n);
+  if (q < c2) {
     it.v = CLS_INTER;
-    it.kt = ctl->lo[CLS_INTER] + it.n;
-  } else if (it.n < c2 + c1) {
+    it.kt = ctl->lo[CLS_INTER] + q;
+  } else if (q < c2 + c1) {
     it.v = CLS_SUCC;
-    it.kt = ctl->lo[CLS_SUCC] + (it.n - c2);
+    it.kt = ctl->lo[CLS_SUCC] + (q - c2);
   } else {
     it.v = CLS_INTRA;
-    it.kt = ctl->lo[CLS_INTRA] + (it.n - c2 - c1);
+    it.kt = ctl->lo[CLS_INTRA] + (q - c2 - c1);
   }
 }
 
@@ -138,7 +150,7 @@ __device__ __forceinline__ Cursor first_item(const SmemCtl* ctl, const Params& p
   Cursor it;
   it.n = 0;
   if (p.continuous) {
-    it.kt = ctl->kt0;
+    it.kt = ctl->kt0 + (ctl->c_first == ctl->c_last ? phys_item(ctl, 0) : 0);
     it.c = ctl->c_first;
     it.v = 0;
   } else {
@@ -150,7 +162,9 @@ __device__ __forceinline__ Cursor first_item(const SmemCtl* ctl, const Params& p
 
 __device__ __forceinline__ void next_item(const SmemCtl* ctl, const Params& p, Cursor& it) {
   ++it.n;
-  if (p.continuous) {
+  if (p.continuous && ctl->c_first == ctl->c_last) {
+    it.kt = ctl->kt0 + phys_item(ctl, it.n);  // one item per k-tile
+  } else if (p.continuous) {
     const int64_t tile_end = static_cast<int64_t>(it.kt) * BN + BN;
     const int64_t last = (tile_end < ctl->kend ? tile_end : ctl->kend) - 1;
     const uint32_t s32 = static_cast<uint32_t>(p.s);
@@ -300,6 +314,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       mbar_init(&ctl->drain, 1);
       ctl->abort = 0;
       ctl->n_items = n;
+      ctl->rot = (n == 0 || (p.continuous && ctl->c_first != ctl->c_last)) ? 0 : (hh * n) / p.G;
       fence_barrier_init();
     }
   }
