@@ -65,9 +65,9 @@ constexpr uint32_t TMEM_COLS = NSBUF * ROWS;
 constexpr int SBINS = SLICE + ROWS;       // offsets i - j met by a slice
 constexpr int MSTRIDE = 144;              // row stride of the merge buffers (conflict-free)
 constexpr int MROWS = 16;                 // rows per merge round
-// pass 2: vertical bins [SLICE] (key j is always updated by one thread) and
-// the slash bins [SBINS] (each lane adds its three diagonal sums once per
-// item, atomically: the warps' diagonal ranges overlap)
+// pass 2: vertical bins [SLICE] (key j: one atomic add per row half) and the
+// slash bins [SBINS] (each lane adds its two diagonal sums once per item,
+// atomically: the warps' diagonal ranges overlap)
 constexpr int BIN_FLOATS =
     (SLICE + SBINS) > 2 * MROWS * MSTRIDE ? (SLICE + SBINS) : 2 * MROWS * MSTRIDE;
 constexpr float NEG_BIG = -1e30f;         // finite "no value yet" maximum
@@ -84,7 +84,7 @@ struct SmemCtl {
   uint32_t tmem_base;
   int abort;
   int n_items;
-  int rot;                  // item order rotation (see Cursor)
+  int rot;                  // item order rotation (see phys_item)
   int lo[3], hi[3];         // DCA: k-tile range per class, clipped to the slice
   int kt0;                  // continuous: first k-tile of the slice
   int64_t kend;             // continuous: end of the slice's causal keys
@@ -195,9 +195,9 @@ __device__ __forceinline__ void split_pack(float a, float b, uint32_t& hi, uint3
 // angles `cs` (continuous) or as they are (cs == nullptr).  The softmax warps'
 // 256 threads.
 __device__ __forceinline__ void build_operand(uint8_t* op_hi, const float* __restrict__ src,
-                                              const float2* __restrict__ cs, int tau) {
+                                              const float2* __restrict__ cs, int t) {
 #pragma unroll
-  for (int task = tau; task < ROWS * 8; task += 256) {  // all loads issued together
+  for (int task = t; task < ROWS * 8; task += SM_THREADS) {  // all loads issued together
     const int r = task >> 3, c = task & 7;
     const float* row = src + r * HD;
     const float4 a0 = *reinterpret_cast<const float4*>(row + 8 * c);
