@@ -158,9 +158,11 @@ def decode_scratch_size(Lq, Hq, Hkv) -> int:
 def decode(q_block, v_cache, out=None, *, q_start, kv_len, chunk_size, local_window,
            pretrain_window, yarn_scale=1.0, workspace: Workspace, scratch=None, lse=None,
            window_reading="query_offset"):
-    """Decode-stage attention of a few query tokens (absolute rows q_start ..)
-    against the rotated keys [0, kv_len) in `workspace` and v_cache.  `lse`
-    (optional fp32 [Lq, Hq]) receives the natural-log LSE of each row."""
+    """Decode-stage attention of a few query tokens (absolute rows q_start ..,
+    Lq <= DCA_DECODE_MAX_TOKENS = 256) against the rotated keys [0, kv_len)
+    in `workspace` and v_cache, split over the key range and merged.  `lse`
+    (optional fp32 [Lq, Hq]) receives the natural-log LSE of each row.
+    Returns out [Lq, Hq, 128]."""
     _check_cuda(q_block, v_cache)
     Lq, Hq, d = q_block.shape
     if out is None:
@@ -260,7 +262,10 @@ class SparseWorkspace:
 def sparse_prepare(pattern: SparsePattern, v_cache, *, kv_len, chunk_size, local_window,
                    pretrain_window, workspace: Workspace, sparse: SparseWorkspace):
     """Copy the pattern (restricted to keys < kv_len), build the bitmaps and
-    gather the vertical rows from the rotated keys in `workspace`."""
+    gather the vertical rows from the rotated keys in `workspace` (which
+    must hold rows [0, kv_len): call prepare first).  The lists are checked
+    on the host: sorted, no repeats, at most 1023 runs of consecutive slash
+    offsets per head; per-head sizes within sparse's configuration."""
     _check_cuda(v_cache)
     pat = pattern.restricted(kv_len)
     rc = N.lib().dca_sparse_prepare(
@@ -275,7 +280,14 @@ def sparse_prepare(pattern: SparsePattern, v_cache, *, kv_len, chunk_size, local
 def sparse_attend(q_block, v_cache, out=None, *, q_start, kv_len, chunk_size, local_window,
                   pretrain_window, yarn_scale=1.0, workspace: Workspace, sparse: SparseWorkspace,
                   window_reading="query_offset"):
-    """Sparse DCA attention of a query block over the prepared structures."""
+    """Sparse DCA attention of a query block over the prepared structures.
+
+    q_block [Lq, Hq, 128] bf16 holds the rows q_start .. q_start + Lq - 1;
+    row i attends, per head, only its pattern's members among keys j <= i:
+    the vertical keys, the keys i - o for the slash offsets o, and j = i,
+    each counted once, with the DCA positions of the pair.  `sparse` must
+    hold a pattern prepared (sparse_prepare) or selected (sparse_select)
+    for kv_len >= q_start + Lq keys.  Returns out [Lq, Hq, 128]."""
     _check_cuda(q_block, v_cache)
     Lq, Hq, d = q_block.shape
     if out is None:
@@ -296,7 +308,14 @@ def sparse_select(q_block, v_cache, *, q_start, kv_len, chunk_size, local_window
                   n_last=64, continuous=True, workspace: Workspace, sparse: SparseWorkspace,
                   scratch=None, window_reading="query_offset"):
     """Online key selection into `sparse` from the last n_last rows of the
-    block (continuous=True: true positions, the refinement; False: DCA)."""
+    block (continuous=True: true positions, the refinement; False: DCA).
+
+    For each query head, the softmax of the last n_last (<= 64) rows over
+    keys j < kv_len gives per-key column sums (vertical) and per-offset
+    diagonal sums (slash); the n_vertical keys and n_slash offsets of
+    largest sum (ties: the smaller index) become the head's pattern, ready
+    for sparse_attend.  n_vertical <= sparse's max_vertical, n_slash <=
+    max_slash and <= 1023.  bf16 only.  sparse_pattern_get reads it back."""
     _check_cuda(q_block, v_cache)
     Lq, Hq, d = q_block.shape
     if scratch is None:
