@@ -302,7 +302,7 @@ def run_reference(args, w, rank, world):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": t_full * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic",
-        "config": workload_config(w),
+        "config": {**workload_config(w), "parallelism": f"replicas x{world}" if world > 1 else "1 GPU"},
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
                          "sample": desc},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -374,7 +374,8 @@ def run_decode_bench(args, dw, world, rank, local, dist):
             "impl": "reference", "metric": DECODE_METRIC, "value": value, "unit": UNIT,
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": t_step * 1e3, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "f64", "data": "synthetic", "config": decode_config(dw),
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {**decode_config(dw), "parallelism": f"replicas x{world}" if world > 1 else "1 GPU"},
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
                              "sample": desc},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
@@ -595,7 +596,7 @@ def run_sparse_bench(args, sw, world, rank, local, dist):
                     "unit": UNIT, "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
                     "ms_per_step": t_full * 1e3, "higher_is_better": True, "scaling": "weak",
                     "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-                    "config": sparse_config(sw), "cpu_baseline": cpu,
+                    "config": {**sparse_config(sw), "parallelism": f"replicas x{world}" if world > 1 else "1 GPU"}, "cpu_baseline": cpu,
                     "e2e": {"value": cpu["value"], "unit": UNIT, "h2d_bytes_per_step": 0,
                             "d2h_bytes_per_step": 0}}), flush=True)
             return 0

@@ -353,24 +353,47 @@ int dca_class_rows(int64_t j, int64_t i_first, int n_rows, int64_t kv_len, int64
  * later allocation fails or stalls the device, or a plugin whose host
  * framework owns every device allocation.  Same arguments and result as
  * dca_prefill, minus the workspace: the library uses a fixed scratch area of
- * DCA_NOALLOC_SCRATCH_BYTES that is part of its image (present on every GPU
- * that loads the library until the process exits), and calls no cudaMalloc,
- * cudaFree or allocating library routine.
- *   - Returns DCA_ERR_WORKSPACE, before any launch, when
+ * DCA_NOALLOC_SCRATCH_BYTES that is part of its image, and calls no
+ * cudaMalloc, cudaFree or allocating library routine.
+ *   - The scratch exists on a device once the library's device code is loaded
+ *     there, and stays until the process exits.  Under lazy module loading
+ *     (CUDA_MODULE_LOADING=LAZY, the default of recent CUDA) that happens at
+ *     the first use on the device, not when the library is opened: call
+ *     dca_noalloc_prepare() once per device, with that device current, before
+ *     reserving the rest of the device's memory and before any stream capture.
+ *     Otherwise the first dca_prefill_noalloc call does it.
+ *   - The scratch address is looked up once per device and kept; do not use
+ *     these entry points across cudaDeviceReset (the kept address is stale).
+ *   - Returns DCA_ERR_WORKSPACE, before any device work, when
  *     dca_workspace_size(L, ...) exceeds DCA_NOALLOC_SCRATCH_BYTES (about
- *     L <= 16384 for 4 KV heads in bf16).
- *   - The first call on a device looks up the scratch address on that device
- *     (with it current); make that first call before any stream capture.
+ *     L <= 16384 for 4 KV heads in bf16).  Every other argument is checked
+ *     as dca_prefill checks it, also before any device work.
  *   - All calls share the one scratch area: calls that overlap on the GPU
  *     (other streams, other threads) race and must be serialised by the caller.
- *   - The status word in the scratch is cleared at the start of each call and
- *     cannot be read back with dca_device_status.
+ *   - The status word in the scratch is cleared at the start of each call;
+ *     dca_noalloc_device_status reads it back after the call.
  */
 #define DCA_NOALLOC_SCRATCH_BYTES (32u * 1024u * 1024u)
 int dca_prefill_noalloc(const void* q, const void* k, const void* v, void* out, int64_t L,
                         int Hq, int Hkv, int d, int64_t chunk_size, int64_t local_window,
                         int64_t pretrain_window, double rope_base, double yarn_scale, int dtype,
                         void* cuda_stream);
+
+/*
+ * Loads the library's device code on the current device and looks up the
+ * no-allocation scratch there (no device memory is allocated beyond the
+ * library image).  Returns DCA_OK or DCA_ERR_CUDA.
+ */
+int dca_noalloc_prepare(void);
+
+/*
+ * dca_device_status for the no-allocation scratch of the current device:
+ * synchronises `cuda_stream`, returns DCA_ERR_TIMEOUT (and clears the word)
+ * when a bounded device wait of the last dca_prefill_noalloc call ran out
+ * (its output is then incomplete), DCA_OK otherwise, DCA_ERR_CUDA on a CUDA
+ * error.
+ */
+int dca_noalloc_device_status(void* cuda_stream);
 
 /*
  * Test hooks.  dca_set_wait_timeout_ns sets the limit of every bounded device

@@ -133,6 +133,19 @@ int attend_impl(const void* q, const void* v, void* out, int64_t q_start, int64_
 
 bool ptrs_ok(const void* p) { return p != nullptr && aligned(p, 16); }
 
+// Host-side checks of a one-shot or chunked prefill call (no device work).
+int prefill_checks(const void* q, const void* k, const void* v, const void* out, int64_t q_start,
+                   int64_t Lq, int64_t Lk, int Hq, int Hkv, int d, int64_t s, int64_t w,
+                   int64_t c, double rope_base, double yarn_scale, int dtype, const void* ws,
+                   size_t ws_bytes, Layout* L) {
+  int rc = check_common(q_start, Lq, Lk, Hq, Hkv, d, s, w, c, yarn_scale, dtype, ws, ws_bytes, L);
+  if (rc != DCA_OK) return rc;
+  if (!(rope_base > 0.0) || !isfinite(rope_base)) return DCA_ERR_ARG;
+  if (Lq == 0) return DCA_OK;
+  if (!ptrs_ok(q) || !ptrs_ok(k) || !ptrs_ok(v) || !ptrs_ok(out)) return DCA_ERR_ARG;
+  return DCA_OK;
+}
+
 // Scratch bytes of a decode call (0 for invalid sizes).
 size_t decode_scratch_bytes(int64_t Lq, int Hq, int Hkv) {
   if (Lq < 1 || Lq > DCA_DECODE_MAX_TOKENS || Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0) return 0;
@@ -230,6 +243,16 @@ int64_t list_runs(const int32_t* a, int64_t n, int64_t Lk) {
 }
 
 }  // namespace
+
+namespace dca {
+int check_prefill_args(const void* q, const void* k, const void* v, const void* out, int64_t L,
+                       int Hq, int Hkv, int d, int64_t s, int64_t w, int64_t c, double rope_base,
+                       double yarn_scale, int dtype, const void* ws, size_t ws_bytes) {
+  Layout lay;
+  return prefill_checks(q, k, v, out, 0, L, L, Hq, Hkv, d, s, w, c, rope_base, yarn_scale, dtype,
+                        ws, ws_bytes, &lay);
+}
+}  // namespace dca
 
 extern "C" {
 
@@ -371,13 +394,10 @@ int dca_prefill_chunked_ex(const void* q_block, const void* k_cache, const void*
   const int reading = reading_of(opts);
   if (reading < 0) return DCA_ERR_ARG;
   Layout L;
-  int rc = check_common(q_start, Lq, Lk, Hq, Hkv, d, chunk_size, local_window, pretrain_window,
-                        yarn_scale, dtype, workspace, ws_bytes, &L);
-  if (rc != DCA_OK) return rc;
-  if (!(rope_base > 0.0) || !isfinite(rope_base)) return DCA_ERR_ARG;
-  if (Lq == 0) return DCA_OK;
-  if (!ptrs_ok(q_block) || !ptrs_ok(k_cache) || !ptrs_ok(v_cache) || !ptrs_ok(out_block))
-    return DCA_ERR_ARG;
+  int rc = prefill_checks(q_block, k_cache, v_cache, out_block, q_start, Lq, Lk, Hq, Hkv, d,
+                          chunk_size, local_window, pretrain_window, rope_base, yarn_scale, dtype,
+                          workspace, ws_bytes, &L);
+  if (rc != DCA_OK || Lq == 0) return rc;
   cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
   rc = prepare_impl(k_cache, Lk, 0, Hkv, d, chunk_size, local_window, pretrain_window, rope_base,
                     dtype, workspace, L, st);

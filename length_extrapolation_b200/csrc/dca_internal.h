@@ -98,6 +98,12 @@ cudaError_t launch_select_scores(const void* kr, const float* qv, const float2* 
                                  unsigned long long timeout_ns, cudaStream_t st);
 cudaError_t launch_select(const SelectArgs& sa, cudaStream_t st);
 
+// Host-side argument checks of dca_prefill (no device work): the dca_status
+// that dca_prefill would return before launching anything, or DCA_OK.
+int check_prefill_args(const void* q, const void* k, const void* v, const void* out, int64_t L,
+                       int Hq, int Hkv, int d, int64_t s, int64_t w, int64_t c, double rope_base,
+                       double yarn_scale, int dtype, const void* ws, size_t ws_bytes);
+
 // bf16 tcgen05/TMA kernel; returns a CUDA error or cudaSuccess, or
 // cudaErrorInvalidValue when a tensor map cannot be encoded.
 cudaError_t launch_attention_sm100(const AttnArgs& a, cudaStream_t st);

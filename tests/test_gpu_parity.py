@@ -235,6 +235,17 @@ def test_empty_block_is_a_no_op():
 
 
 # ------------------------------------------------------------------ full size
+def _rows_to_check(w, q0, lq, n_random, max_rows):
+    """Block-relative rows: every chunk-structure row of sample_rows (chunk
+    offsets 0, 1, w-1, w, w+1, s-1 and the block's edges) first, then its
+    seeded random rows up to max_rows in total."""
+    structural = sample_rows(w, q0, lq, n_random=0).numpy()
+    extra = np.setdiff1d(sample_rows(w, q0, lq, n_random=n_random).numpy(), structural)
+    if max_rows is not None:
+        extra = extra[:max(0, max_rows - len(structural))]
+    return np.union1d(structural, extra)
+
+
 def _full_size_check(name, max_rows=None, n_random=48, blocks_to_check=None):
     w = WORKLOADS[name]
     q, k, v = generate(w, device=DEV)
@@ -249,10 +260,7 @@ def _full_size_check(name, max_rows=None, n_random=48, blocks_to_check=None):
         blocks = [blocks[b] for b in blocks_to_check]
     worst = (0.0, 0.0)
     for q0, lq, lk in blocks:
-        rows = sample_rows(w, q0, lq, n_random=n_random).numpy()
-        if max_rows is not None and len(rows) > max_rows:
-            sel = np.linspace(0, len(rows) - 1, max_rows).round().astype(int)
-            rows = rows[np.unique(sel)]
+        rows = _rows_to_check(w, q0, lq, n_random, max_rows)
         want = oracle.attention(q[q0:q0 + lq].cpu(), kc[:lk], vc[:lk], q_start=q0, rows=rows,
                                 heads=heads, **w.params())
         got = gather(out[q0:q0 + lq], rows, heads)
@@ -274,5 +282,19 @@ def test_full_size_qwen7b_256k():
 
 
 def test_full_size_qwen7b_1m_chunked():
-    # first, a middle and the last query block (all 32 blocks run on the GPU)
-    _full_size_check("qwen7b_1m_chunked", max_rows=12, n_random=4, blocks_to_check=[0, 13, 31])
+    """All 32 query blocks run on the GPU; five are checked on sampled rows.
+    Block 0 lies in chunk 0 (intra pairs only).  Blocks 6 and 30 start at the
+    starts of chunks 1 and 5, so every row has r_i < w: their pairs with the
+    previous chunk keep the true distance, with queries rotated by s + r_i up
+    to s + w - 1 = 229,375 (the largest table position below c - 1); block 30
+    also has inter-chunk pairs against chunks 0-3.  Blocks 13 and 31 start at
+    offset 32,768 = w of chunks 2 and 5: their previous-chunk pairs take the
+    inter rule."""
+    w = WORKLOADS["qwen7b_1m_chunked"]
+    s, lw, blk = w.chunk_size, w.local_window, w.block
+    for b, want_succ_true in ((6, True), (30, True), (13, False), (31, False)):
+        q0 = b * blk
+        r0, r1 = q0 % s, (q0 + blk - 1) % s
+        assert (r1 < lw) == want_succ_true and (r0 >= lw) == (not want_succ_true)
+    _full_size_check("qwen7b_1m_chunked", max_rows=12, n_random=4,
+                     blocks_to_check=[0, 6, 13, 30, 31])

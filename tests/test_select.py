@@ -110,6 +110,81 @@ def test_selection_is_a_topk_of_the_oracle_scores(w, nv, ns, nl, continuous):
         check_topk(S[h], slash[h], min(ns, w.L))
 
 
+# Key ranges beyond one score slice (4096 keys per CTA of the score passes) and
+# beyond one top-k span (16,384 keys per CTA of the radix select): the slices'
+# row statistics are merged across CTAs and the spans' counts place each
+# span's part of the ordered output.
+#   sel_50k_g7:  13 slices, 4 spans (the last ragged), G = 7, n_last = 64
+#   sel_70k_gqa: 18 slices, 5 spans (the last ragged), G = 2, YaRN 2, n_last = 48
+MULTI = [
+    (wl("sel_50k_g7", 50000, 7, 1, 4096, 512, 8192, sqrt_d=True), 1000, 1000, 64),
+    (wl("sel_70k_gqa", 70000, 4, 2, 16384, 2048, 32768, yarn=2.0), 700, 900, 48),
+]
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("continuous", [True, False], ids=["continuous", "dca"])
+@pytest.mark.parametrize("w,nv,ns,nl", MULTI, ids=lambda x: getattr(x, "name", ""))
+def test_selection_spanning_slices_and_spans(w, nv, ns, nl, continuous):
+    assert w.L > 2 * 16384 and w.L % 16384 != 0 and w.L > 4 * 4096
+    q, k, v, ws, sp, V, S = select_on_gpu(w, nv, ns, nl, continuous)
+    vert, slash = oracle.vs_scores(q.cpu(), k.cpu(), n_last=nl, continuous=continuous,
+                                   **w.params())
+    for h in range(w.Hq):
+        check_topk(V[h], vert[h], nv)
+        check_topk(S[h], slash[h], ns)
+        # the selections reach into every span, not only the first
+        assert V[h].max() >= 2 * 16384 and S[h].max() >= 16384
+
+
+def _rope(x, pos, base=1e7):
+    """Rotate the last axis of x (d = 128, pairs (k, k + 64)) by position pos (fp64)."""
+    d = x.shape[-1]
+    th = base ** (-2.0 * np.arange(d // 2) / d)
+    c, sn = np.cos(pos * th), np.sin(pos * th)
+    a, b = x[..., : d // 2], x[..., d // 2:]
+    return np.concatenate([a * c - b * sn, a * sn + b * c], axis=-1)
+
+
+@pytest.mark.gpu
+def test_exact_ties_across_topk_spans():
+    """Seven bit-identical keys with the same j mod s (12000 + 4096 n,
+    n = 0..6), all inter-chunk for the estimate rows, straddle the first three
+    16,384-key spans (two in span 0, four in span 1, one in span 2).  The last
+    rows' queries point along the keys' rotated direction, so these keys
+    score highest, exactly alike on both sides; a top-k that cuts through
+    them takes the smaller indices (the oracle's rule), across spans."""
+    w = wl("sel_span_ties", 50000, 2, 1, 4096, 512, 8192)
+    q, k, v = generate(w, device=DEV, seed=9)
+    dup = [12000 + 4096 * n for n in range(7)]
+    assert [j // 16384 for j in dup] == [0, 0, 1, 1, 1, 1, 2]
+    rng = np.random.default_rng(9)
+    u = rng.standard_normal(128)
+    key = _rope(0.5 * u, w.pretrain_window - 1 - dup[0] % w.chunk_size)   # R(j mod s) key = R(c-1) u / 2
+    q[-64:] = torch.as_tensor(u, dtype=torch.float32).to(q.dtype).to(DEV)
+    kb = torch.as_tensor(key, dtype=torch.float32).to(k.dtype).to(DEV)
+    for j in dup:
+        k[j, 0] = kb
+    kw = dict(chunk_size=w.chunk_size, local_window=w.local_window,
+              pretrain_window=w.pretrain_window)
+    ws = dca.Workspace(w.L, w.Hq, w.Hkv, 128, w.chunk_size, w.local_window, w.pretrain_window,
+                       q.dtype, DEV)
+    dca.prepare(k, kv_len=w.L, k_rows_valid=0, rope_base=w.rope_base, workspace=ws, **kw)
+    sp = dca.SparseWorkspace(w.L, w.Hq, 8, 8, DEV)
+    vert, _ = oracle.vs_scores(q.cpu(), k.cpu(), n_last=64, continuous=False, **w.params())
+    for h in range(w.Hq):
+        assert len({vert[h][j] for j in dup}) == 1
+        assert set(oracle.topk(vert[h], 7).tolist()) == set(dup)
+    for n_v in (1, 2, 3, 6):
+        dca.sparse_select(q, v, q_start=0, kv_len=w.L, rope_base=w.rope_base,
+                          yarn_scale=w.yarn_scale, n_vertical=n_v, n_slash=4, n_last=64,
+                          continuous=False, workspace=ws, sparse=sp, **kw)
+        V, _ = dca.sparse_pattern_get(sp, w.Hq)
+        for h in range(w.Hq):
+            assert oracle.topk(vert[h], n_v).tolist() == dup[:n_v]
+            assert V[h].tolist() == dup[:n_v], (n_v, h, V[h])
+
+
 @pytest.mark.gpu
 def test_selected_pattern_attention_matches_oracle():
     from tests.gpu_helpers import assert_close
