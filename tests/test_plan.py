@@ -159,3 +159,28 @@ def test_selection_row_ranges_reject(lib):
                 dict(w=17), dict(cls=3), dict(cls=-2), dict(reading=2), dict(i_first=-1)):
         assert call(**bad) == N.DCA_ERR_ARG, bad
     assert lib.dca_class_rows(5, 0, 8, 100, 16, 4, 0, 0, 0, None) == N.DCA_ERR_ARG
+
+
+@pytest.mark.parametrize("s,w,q_start,L", [
+    (128, 0, 0, 1000), (256, 128, 128, 1500), (384, 200, 256, 2600), (1024, 1024, 0, 4200),
+    (512, 77, 1024, 3000), (128, 128, 384, 900)])
+def test_consecutive_tiles_share_an_ascending_key_order(lib, s, w, q_start, L):
+    """Under reading A with s a multiple of 128 and a 128-aligned q_start (the
+    condition under which the attention kernel runs a group's last head on two
+    consecutive query tiles in one CTA), every tile's work list is its key
+    tiles 0, 1, 2, ... in order, each once, and tile t's list is a prefix of
+    tile t + 1's, with its own class per key tile."""
+    rows = 128
+    prev = None
+    for q0 in range(q_start, L, rows):
+        i_last = min(q0 + rows - 1, L - 1)
+        a = plan(lib, q0, i_last, rows, s, 128, w=w, reading=0)
+        assert a[:, 0].tolist() == list(range(len(a)))
+        for kt, cls, _ in a:
+            js = range(kt * 128, min(kt * 128 + 128, i_last + 1))
+            want = {chunk_class(i, j, s, w) for i in range(q0, i_last + 1) for j in js if j <= i}
+            assert want == {cls}
+        if prev is not None:
+            assert len(a) == len(prev) + 1
+            assert a[:len(prev), 0].tolist() == prev[:, 0].tolist()
+        prev = a
