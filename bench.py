@@ -58,11 +58,15 @@ def parse_args(argv=None):
                     choices=sorted(WORKLOADS) + sorted(DECODE_WORKLOADS) + sorted(SPARSE_WORKLOADS),
                     help="a prefill workload, or a decode step (*_decode*: the new tokens "
                          "against a full cache)")
-    ap.add_argument("--e2e-steps", type=int, default=2)
+    ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--cpu-seconds", type=float, default=20.0,
                     help="approximate CPU seconds for the oracle baseline sample")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--block", type=int, default=None, metavar="B",
+                    help="profiling mode for a chunked workload: allocate only query block B "
+                         "and the KV cache it attends (a few GB), time its attention launch "
+                         "alone; prints a profiling line, not the workload's metric")
     ap.add_argument("--record-traffic", metavar="NCU_CSV",
                     help="store the attention kernel's DRAM bytes per launch from an ncu CSV "
                          "capture of --workload, then exit")
@@ -722,6 +726,64 @@ def run_sparse_bench(args, sw, world, rank, local, dist):
     return 0
 
 
+# ----------------------------------------------------------------------------- one block
+def run_block_bench(args, w, local=0):
+    """One query block of a chunked workload, alone on the device: q/out of
+    that block and the keys/values it attends (seeded like the workload's
+    inputs, but drawn for these rows only).  The keys are rotated once before
+    timing; each step is one attention launch.  For ncu captures of a long
+    block (the last block of the 1M workload holds about 3.6 GB on the device)."""
+    import length_extrapolation_b200 as dca
+    from length_extrapolation_b200 import _native as N
+    from length_extrapolation_b200.workloads import _draw
+
+    q0, lq, lk = w.blocks()[args.block]
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    peaks = load_peaks()
+    g = torch.Generator(device=dev)
+    g.manual_seed(0)
+    k = _draw(w, g, lk, w.Hkv, dev)
+    v = _draw(w, g, lk, w.Hkv, dev)
+    q = _draw(w, g, lq, w.Hq, dev)
+    out = torch.empty_like(q)
+    p = w.params()
+    ws = dca.Workspace(lk, w.Hq, w.Hkv, w.d, w.chunk_size, w.local_window, w.pretrain_window,
+                       w.torch_dtype, dev)
+    dca.prepare(k, kv_len=lk, k_rows_valid=0, chunk_size=p["chunk_size"],
+                local_window=p["local_window"], pretrain_window=p["pretrain_window"],
+                rope_base=p["rope_base"], workspace=ws)
+
+    def step():
+        dca.attend(q, v, out, q_start=q0, kv_len=lk, chunk_size=p["chunk_size"],
+                   local_window=p["local_window"], pretrain_window=p["pretrain_window"],
+                   yarn_scale=p["yarn_scale"], workspace=ws)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if ws.status() != N.DCA_OK:
+        raise RuntimeError("device status after warm-up")
+    clocks = ClockSampler(dev.index).start()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps):
+        step()
+    e1.record()
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    ms = e0.elapsed_time(e1) / args.steps
+    flops = 4.0 * w.d * w.Hq * causal_pairs(q0, lq)
+    print(json.dumps({
+        "profiling": f"attention of query block {args.block} of {w.name} alone",
+        "q_start": q0, "Lq": lq, "Lk": lk, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_launch": ms, "tflops": flops / (ms / 1e3) / 1e12,
+        "frac_of_measured_sustained": flops / (ms / 1e3) / 1e12 / peaks["bf16_tflops_sustained"],
+        "algorithmic_bytes": (2 * lq * w.Hq + 2 * lk * w.Hkv) * w.d * q.element_size(),
+        "clocks": clk}), flush=True)
+    return 0
+
+
 # ----------------------------------------------------------------------------- our arm
 def main(argv=None):
     args = parse_args(argv)
@@ -738,6 +800,8 @@ def main(argv=None):
         dist = init_dist(world, local)
         return run_decode_bench(args, DECODE_WORKLOADS[args.workload], world, rank, local, dist)
     w = WORKLOADS[args.workload]
+    if args.block is not None:
+        return run_block_bench(args, w)
     if args.record_traffic:
         write_traffic_record(w.name, args.record_traffic)
         return 0
@@ -842,12 +906,30 @@ def main(argv=None):
         barrier()
         ems_step = max_over_ranks([e0.elapsed_time(e1)], dist, dev)[0] / args.e2e_steps
         esz = q.element_size()
+        h2d_bytes = (q.numel() + k.numel() + v.numel()) * esz
+        d2h_bytes = q.numel() * esz
+        # copy rates of the same bytes alone (one pinned copy each way, device timed)
+        del arena
+        torch.cuda.empty_cache()
+        buf = torch.empty(q.numel() * esz, dtype=torch.uint8, device=dev)
+        c0 = torch.cuda.Event(enable_timing=True)
+        c1 = torch.cuda.Event(enable_timing=True)
+        c2 = torch.cuda.Event(enable_timing=True)
+        c0.record()
+        for t in (qh, kh, vh):
+            buf[:t.numel() * esz].copy_(t.view(-1).view(torch.uint8), non_blocking=True)
+        c1.record()
+        oh.view(-1).view(torch.uint8).copy_(buf[:d2h_bytes], non_blocking=True)
+        c2.record()
+        torch.cuda.synchronize()
+        del buf
         e2e = {"value": whole_job_rate(w.L, world, ems_step), "unit": UNIT,
                "ms_per_step": ems_step,
-               "h2d_bytes_per_step": (q.numel() + k.numel() + v.numel()) * esz,
-               "d2h_bytes_per_step": q.numel() * esz,
-               "path": "dca_prefill_host (pinned host buffers, copies and kernels on one stream)"}
-        del arena
+               "h2d_bytes_per_step": h2d_bytes, "d2h_bytes_per_step": d2h_bytes,
+               "h2d_gbs_alone": h2d_bytes / (c0.elapsed_time(c1) / 1e3) / 1e9,
+               "d2h_gbs_alone": d2h_bytes / (c1.elapsed_time(c2) / 1e3) / 1e9,
+               "path": "dca_prefill_host (pinned host buffers; copies on the library's copy "
+                       "stream overlap the kernels on the caller's stream)"}
 
     # ---------------------------------------------------------------- CPU baseline
     cpu = None

@@ -296,13 +296,18 @@ int dca_device_status(void* workspace, void* cuda_stream);
 /*
  * Host-buffer entry point: whole prefill of L tokens from HOST memory.
  * q_h, out_h [L][Hq][d]; k_h, v_h [L][Hkv][d] in host memory (pinned memory
- * gives full copy bandwidth).  The input is processed in query blocks of
- * `block` rows (block <= 0: one block): per block the library copies the
- * block's q, k and v rows host->device, appends the keys to the rotated-key
- * cache, runs the attention kernel and copies the block's output rows back.
- * All device memory comes from the caller's `arena` (dca_host_arena_size bytes,
- * 256-byte aligned).  Returns after enqueuing; call dca_device_status or
- * synchronise the stream before reading out_h.
+ * gives full copy bandwidth and lets the copies overlap the kernels).  The
+ * input is processed in query blocks of `block` rows (block <= 0: one block):
+ * per block the library copies the block's q, k and v rows host->device,
+ * appends the keys to the rotated-key cache, runs the attention kernel and
+ * copies the block's output rows back.  The copies run on a copy stream of
+ * the library's own (one non-blocking stream per device, created on first
+ * use), ordered against `cuda_stream` by events: block b + 1's inputs and
+ * block b - 1's outputs move while block b is attended (two query and two
+ * output block buffers in the arena).  All device memory comes from the
+ * caller's `arena` (dca_host_arena_size bytes, 256-byte aligned).  Returns
+ * after enqueuing; `cuda_stream` waits for every copy, so synchronising it
+ * (or dca_device_status) makes out_h readable.
  */
 size_t dca_host_arena_size(int64_t L, int64_t block, int Hq, int Hkv, int d,
                            int64_t chunk_size, int64_t local_window, int64_t pretrain_window,
@@ -345,6 +350,19 @@ int dca_plan_items(int64_t i0, int64_t i_last, int64_t tile_rows, int64_t chunk_
 int dca_class_rows(int64_t j, int64_t i_first, int n_rows, int64_t kv_len, int64_t chunk_size,
                    int64_t local_window, int window_reading, int cls, int64_t chunk,
                    int32_t* range);
+
+/*
+ * Host-side introspection of the attention kernel's per-row masking (no GPU
+ * needed): the keys [range[0], range[1]) that form pairs of work-list class
+ * `cls` (0, 1, 2 as in dca_plan_items) with query row i, causal (j <= i)
+ * included -- one contiguous range per row and class (empty: range[0] ==
+ * range[1]).  A masked tile keeps exactly its columns inside this range.
+ * Computed in 32-bit arithmetic as on the device.  Returns DCA_OK, or
+ * DCA_ERR_ARG (0 <= i < 2^31 - 1, cls in 0..2, chunk_size >= 1,
+ * 0 <= local_window <= chunk_size, range not NULL).
+ */
+int dca_row_keys(int64_t i, int cls, int64_t chunk_size, int64_t local_window, int window_reading,
+                 int64_t* range);
 
 /*
  * No-allocation one-shot prefill (an addition for integrators; the pages on

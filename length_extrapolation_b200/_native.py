@@ -45,6 +45,7 @@ SIGNATURES = {
                              _dbl, _i32, _vp, _vp, _sz, _vp]),
     "dca_prefill_noalloc": (_i32, [_vp, _vp, _vp, _vp, _i64, _i32, _i32, _i32, _i64, _i64, _i64,
                                    _dbl, _dbl, _i32, _vp]),
+    "dca_row_keys": (_i32, [_i64, _i32, _i64, _i64, _i32, _vp]),
     "dca_noalloc_prepare": (_i32, []),
     "dca_noalloc_device_status": (_i32, [_vp]),
     "dca_decode_scratch_size": (_sz, [_i64, _i32, _i32]),

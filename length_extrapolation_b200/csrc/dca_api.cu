@@ -6,6 +6,7 @@
 #include <stdint.h>
 
 #include <atomic>
+#include <mutex>
 #include <vector>
 
 #include "../../include/dca.h"
@@ -132,6 +133,24 @@ int attend_impl(const void* q, const void* v, void* out, int64_t q_start, int64_
 }
 
 bool ptrs_ok(const void* p) { return p != nullptr && aligned(p, 16); }
+
+// One non-blocking copy stream per device for the host-buffer entry point,
+// created on first use with that device current and kept until exit.
+std::mutex g_copy_mu;
+cudaStream_t g_copy_stream[64] = {};
+
+int copy_stream_on_current_device(cudaStream_t* out) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return DCA_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_copy_mu);
+  if (g_copy_stream[dev] == nullptr &&
+      cudaStreamCreateWithFlags(&g_copy_stream[dev], cudaStreamNonBlocking) != cudaSuccess) {
+    g_copy_stream[dev] = nullptr;
+    return DCA_ERR_CUDA;
+  }
+  *out = g_copy_stream[dev];
+  return DCA_OK;
+}
 
 // Host-side checks of a one-shot or chunked prefill call (no device work).
 int prefill_checks(const void* q, const void* k, const void* v, const void* out, int64_t q_start,
@@ -438,7 +457,7 @@ size_t dca_host_arena_size(int64_t L, int64_t block, int Hq, int Hkv, int d, int
   const size_t esize = dtype == DCA_BF16 ? 2 : 4;
   const size_t kv = align_up(static_cast<size_t>(L) * Hkv * d * esize, 1024);
   const size_t qo = align_up(static_cast<size_t>(blk) * Hq * d * esize, 1024);
-  return align_up(ws, 1024) + 2 * kv + 2 * qo;
+  return align_up(ws, 1024) + 2 * kv + 4 * qo;  // two query and two output block buffers
 }
 
 int dca_prefill_host(const void* q_h, const void* k_h, const void* v_h, void* out_h, int64_t L,
@@ -462,34 +481,73 @@ int dca_prefill_host(const void* q_h, const void* k_h, const void* v_h, void* ou
   uint8_t* ws = base;
   uint8_t* kc = base + align_up(ws_bytes, 1024);
   uint8_t* vc = kc + kv;
-  uint8_t* qb = vc + kv;
-  uint8_t* ob = qb + qo;
+  uint8_t* qb[2] = {vc + kv, vc + kv + qo};
+  uint8_t* ob[2] = {vc + kv + 2 * qo, vc + kv + 3 * qo};
   cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
-  if (dca_workspace_init(ws, ws_bytes, cuda_stream) != DCA_OK) return DCA_ERR_CUDA;
+  cudaStream_t cs = nullptr;
+  if (copy_stream_on_current_device(&cs) != DCA_OK) return DCA_ERR_CUDA;
+  // events: start (caller's stream), inputs of a block landed (copy stream),
+  // a block's attention done (caller's stream), last copy done (copy stream)
+  cudaEvent_t ev_start = nullptr, ev_done = nullptr, ev_in[2] = {}, ev_out[2] = {};
+  auto destroy_events = [&]() {
+    for (cudaEvent_t e : {ev_start, ev_done, ev_in[0], ev_in[1], ev_out[0], ev_out[1]})
+      if (e != nullptr) cudaEventDestroy(e);
+  };
+  for (cudaEvent_t* e : {&ev_start, &ev_done, &ev_in[0], &ev_in[1], &ev_out[0], &ev_out[1]})
+    if (cudaEventCreateWithFlags(e, cudaEventDisableTiming) != cudaSuccess) {
+      destroy_events();
+      return DCA_ERR_CUDA;
+    }
   const size_t krow = static_cast<size_t>(Hkv) * d * esize;
   const size_t qrow = static_cast<size_t>(Hq) * d * esize;
-  for (int64_t q0 = 0; q0 < L; q0 += blk) {
-    const int64_t lq = (L - q0 < blk) ? L - q0 : blk;
-    const int64_t lk = q0 + lq;
-    if (cudaMemcpyAsync(kc + q0 * krow, static_cast<const uint8_t*>(k_h) + q0 * krow, lq * krow,
-                        cudaMemcpyHostToDevice, st) != cudaSuccess ||
-        cudaMemcpyAsync(vc + q0 * krow, static_cast<const uint8_t*>(v_h) + q0 * krow, lq * krow,
-                        cudaMemcpyHostToDevice, st) != cudaSuccess ||
-        cudaMemcpyAsync(qb, static_cast<const uint8_t*>(q_h) + q0 * qrow, lq * qrow,
-                        cudaMemcpyHostToDevice, st) != cudaSuccess)
-      return DCA_ERR_CUDA;
+  const int64_t nb = (L + blk - 1) / blk;
+  // host -> device copies of block b's key/value rows and query rows (copy stream)
+  auto copy_in = [&](int64_t b) {
+    const int64_t q0 = b * blk, lq = (L - q0 < blk) ? L - q0 : blk;
+    return cudaMemcpyAsync(kc + q0 * krow, static_cast<const uint8_t*>(k_h) + q0 * krow,
+                           lq * krow, cudaMemcpyHostToDevice, cs) == cudaSuccess &&
+           cudaMemcpyAsync(vc + q0 * krow, static_cast<const uint8_t*>(v_h) + q0 * krow,
+                           lq * krow, cudaMemcpyHostToDevice, cs) == cudaSuccess &&
+           cudaMemcpyAsync(qb[b & 1], static_cast<const uint8_t*>(q_h) + q0 * qrow, lq * qrow,
+                           cudaMemcpyHostToDevice, cs) == cudaSuccess &&
+           cudaEventRecord(ev_in[b & 1], cs) == cudaSuccess;
+  };
+  int rc = dca_workspace_init(ws, ws_bytes, cuda_stream);
+  bool ok = rc == DCA_OK && cudaEventRecord(ev_start, st) == cudaSuccess &&
+            cudaStreamWaitEvent(cs, ev_start, 0) == cudaSuccess && copy_in(0);
+  if (rc == DCA_OK && !ok) rc = DCA_ERR_CUDA;
+  // Copy-stream order: in(0) | in(1), out(0) | in(2), out(1) | ...  The inputs
+  // of block b + 1 land while block b is attended; in(b + 2) follows out(b),
+  // which waits for block b's attention, so query buffer b & 1 is free again,
+  // and block b + 2's attention waits for in(b + 2), so output buffer b & 1
+  // has been copied out.  Key/value rows of later blocks are not read by
+  // earlier blocks.
+  for (int64_t b = 0; b < nb && rc == DCA_OK; ++b) {
+    const int64_t q0 = b * blk, lq = (L - q0 < blk) ? L - q0 : blk, lk = q0 + lq;
+    if (cudaStreamWaitEvent(st, ev_in[b & 1], 0) != cudaSuccess) {
+      rc = DCA_ERR_CUDA;
+      break;
+    }
     // the rotated-key cache keeps rows [0, q0) from earlier blocks
-    int rc = dca_prepare(kc, lk, q0, Hkv, d, chunk_size, local_window, pretrain_window, rope_base,
-                         dtype, ws, ws_bytes, cuda_stream);
-    if (rc != DCA_OK) return rc;
-    rc = dca_attend(qb, vc, ob, q0, lq, lk, Hq, Hkv, d, chunk_size, local_window,
+    rc = dca_prepare(kc, lk, q0, Hkv, d, chunk_size, local_window, pretrain_window, rope_base,
+                     dtype, ws, ws_bytes, cuda_stream);
+    if (rc != DCA_OK) break;
+    rc = dca_attend(qb[b & 1], vc, ob[b & 1], q0, lq, lk, Hq, Hkv, d, chunk_size, local_window,
                     pretrain_window, yarn_scale, dtype, ws, ws_bytes, cuda_stream);
-    if (rc != DCA_OK) return rc;
-    if (cudaMemcpyAsync(static_cast<uint8_t*>(out_h) + q0 * qrow, ob, lq * qrow,
-                        cudaMemcpyDeviceToHost, st) != cudaSuccess)
-      return DCA_ERR_CUDA;
+    if (rc != DCA_OK) break;
+    if (cudaEventRecord(ev_out[b & 1], st) != cudaSuccess || (b + 1 < nb && !copy_in(b + 1)) ||
+        cudaStreamWaitEvent(cs, ev_out[b & 1], 0) != cudaSuccess ||
+        cudaMemcpyAsync(static_cast<uint8_t*>(out_h) + q0 * qrow, ob[b & 1], lq * qrow,
+                        cudaMemcpyDeviceToHost, cs) != cudaSuccess)
+      rc = DCA_ERR_CUDA;
   }
-  return DCA_OK;
+  // the caller's stream covers every copy: synchronising it (or
+  // dca_device_status) makes out_h readable
+  if (cudaEventRecord(ev_done, cs) != cudaSuccess ||
+      cudaStreamWaitEvent(st, ev_done, 0) != cudaSuccess)
+    rc = DCA_ERR_CUDA;
+  destroy_events();
+  return rc;
 }
 
 int dca_plan_items(int64_t i0, int64_t i_last, int64_t tile_rows, int64_t chunk_size,
@@ -656,6 +714,22 @@ int dca_class_rows(int64_t j, int64_t i_first, int n_rows, int64_t kv_len, int64
                        chunk, &ra, &rb);
   range[0] = ra;
   range[1] = rb;
+  return DCA_OK;
+}
+
+int dca_row_keys(int64_t i, int cls, int64_t chunk_size, int64_t local_window, int window_reading,
+                 int64_t* range) {
+  if (i < 0 || i > (1LL << 31) - 2 || cls < 0 || cls > 2 || chunk_size < 1 || local_window < 0 ||
+      local_window > chunk_size || range == nullptr ||
+      (window_reading != DCA_WINDOW_QUERY_OFFSET && window_reading != DCA_WINDOW_TRUE_DISTANCE))
+    return DCA_ERR_ARG;
+  // the kernel's 32-bit form: chunk size and window clamped to 2^31 - 1
+  const int s32 = chunk_size < 0x7fffffff ? static_cast<int>(chunk_size) : 0x7fffffff;
+  const int w32 = local_window < 0x7fffffff ? static_cast<int>(local_window) : 0x7fffffff;
+  int lo, hi;
+  dca::row_key_range<int>(static_cast<int>(i), cls, s32, w32, window_reading, lo, hi);
+  range[0] = lo;
+  range[1] = hi;
   return DCA_OK;
 }
 

@@ -118,6 +118,39 @@ DCA_HD void class_key_ranges(int64_t i0, int64_t i_last, int64_t s, int64_t w, i
   hi[CLS_INTRA] = i_last + 1;
 }
 
+// Keys [lo, hi) that pair with query row i in work-list class `cls` (causal
+// j <= i included): one contiguous range per row and class.  INTRA: the
+// row's own chunk up to i; SUCC: chunk n_i - 1 (reading B: only i - j < w);
+// INTER: chunks up to n_i - 2 (reading B: also chunk n_i - 1 where
+// i - j >= w).  Works in any signed integer type holding i, s and w.
+template <class I>
+DCA_HD void row_key_range(I i, int cls, I s, I w, int reading, I& lo, I& hi) {
+  const I ni = i / s;
+  if (cls == CLS_INTRA) {
+    lo = s * ni;
+    hi = i + 1;
+    return;
+  }
+  if (ni == 0) {
+    lo = hi = 0;
+    return;
+  }
+  const I a = s * (ni - 1), b = s * ni;
+  if (cls == CLS_SUCC) {
+    lo = a;
+    hi = b;
+    if (reading == READING_B && i - w + 1 > lo) lo = i - w + 1;
+    if (hi < lo) hi = lo;
+    return;
+  }
+  lo = 0;
+  hi = a;
+  if (reading == READING_B) {
+    const I f = (i - w + 1 < b) ? i - w + 1 : b;
+    if (f > hi) hi = f;
+  }
+}
+
 // Item n of the work list -> (k-tile, class).  Order: INTER, SUCC, INTRA.
 DCA_HD void plan_item(const TilePlan& P, int n, int& kt, int& cls) {
   const int c2 = P.hi[CLS_INTER] - P.lo[CLS_INTER];

@@ -56,6 +56,19 @@ __device__ __forceinline__ float2 exp2_poly2(float2 x) {
                      __uint_as_float(__float_as_uint(q.y) + (__float_as_uint(t.y) << 23)));
 }
 
+// The same software 2^x for one argument with the constants as instruction
+// immediates (no registers held for them; the packed form above keeps six
+// constant pairs in registers).
+__device__ __forceinline__ float exp2_poly1(float x) {
+  x = fmaxf(x, -126.0f);
+  const float t = x + 12582912.0f;  // 1.5 * 2^23: rounds x to an integer n in t's low bits
+  const float f = x - (t - 12582912.0f);
+  float q = fmaf(EXP2_C3, f, EXP2_C2);
+  q = fmaf(q, f, EXP2_C1);
+  q = fmaf(q, f, EXP2_C0);
+  return __uint_as_float(__float_as_uint(q) + (__float_as_uint(t) << 23));
+}
+
 // Of every 8 score pairs of a row, this many take the software exp2.
 #ifndef DCA_EXP2_POLY_PAIRS
 #define DCA_EXP2_POLY_PAIRS 2

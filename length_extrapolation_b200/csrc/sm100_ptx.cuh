@@ -153,6 +153,11 @@ static __device__ __noinline__ bool wait_drain(uint64_t* bar, uint32_t parity, u
   }
 }
 
+// Named barrier `id` (1..15; 0 is __syncthreads) over `n` threads (a multiple of 32).
+__device__ __forceinline__ void named_bar_sync(int id, int n) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
+}
+
 // ---------------------------------------------------------------- TMA
 // 3-D tiled load of one box into shared memory, completing on `bar`
 // (transaction bytes).  Plain CTA-local load: no cluster multicast.
@@ -261,6 +266,13 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t* r) {
         "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
         "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
       : "r"(taddr)
+      : "memory");
+}
+// r[0..7] -> 8 TMEM columns of this thread's lane (call tmem_st_wait before use).
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t* r) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
       : "memory");
 }
 // r[0..15] -> 16 TMEM columns of this thread's lane (call tmem_st_wait before use).

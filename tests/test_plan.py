@@ -184,3 +184,22 @@ def test_consecutive_tiles_share_an_ascending_key_order(lib, s, w, q_start, L):
             assert len(a) == len(prev) + 1
             assert a[:len(prev), 0].tolist() == prev[:, 0].tolist()
         prev = a
+
+
+@pytest.mark.parametrize("s,w,reading", [(1, 0, 0), (3, 2, 0), (3, 2, 1), (7, 0, 1), (7, 7, 1),
+                                         (10, 4, 0), (10, 4, 1), (16, 1, 1), (64, 63, 1)])
+def test_row_key_ranges_match_pair_classes(lib, s, w, reading):
+    """The attention kernel masks a tile to one contiguous key range per row
+    and class; brute force over rows and keys: key j is inside row i's range
+    for class c exactly when j <= i and the pair's class is c."""
+    rng = ctypes.c_int64 * 2
+    for i in range(0, 6 * s + 5):
+        for c in range(3):
+            r = rng()
+            assert lib.dca_row_keys(i, c, s, w, reading, r) == N.DCA_OK
+            want = [j for j in range(i + 1) if chunk_class(i, j, s, w, reading) == c]
+            got = list(range(r[0], r[1]))
+            assert got == want, (i, c, r[0], r[1], want[:3], want[-3:])
+    r = rng()
+    assert lib.dca_row_keys(5, 3, 4, 1, 0, r) == N.DCA_ERR_ARG
+    assert lib.dca_row_keys(5, 0, 4, 5, 0, r) == N.DCA_ERR_ARG
