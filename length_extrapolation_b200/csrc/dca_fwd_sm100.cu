@@ -75,8 +75,10 @@ constexpr float RESCALE_LOG2 = 8.0f;
 #ifndef DCA_S_WAIT
 #define DCA_S_WAIT wait_poll
 #endif
-// How the MMA issuer waits: polling with a short back-off (wait_spin) or a
-// suspending try_wait (wait_bounded).
+// How the MMA issuer waits: polling (wait_poll) or polling with a short
+// back-off (wait_spin).  Its waits sit outside the MMA bursts where they can:
+// a poll between two groups of MMAs leaves the tensor pipe idle for ~160
+// cycles (measured on B200), so a unit's P.V and next S go out back to back.
 #ifndef DCA_MMA_WAIT
 #define DCA_MMA_WAIT wait_poll
 #endif
@@ -516,8 +518,8 @@ __global__ void DCA_FWD_BOUNDS
       // Descriptors are built once; a k-step only adds its byte offset / 16 to
       // the start-address field (no carry out of the 14-bit field: shared
       // memory addresses stay below 256 KiB).
-      const uint64_t dq[2] = {sdesc_sw128(smem_u32(q_bufs), 16, 1024),
-                              sdesc_sw128(smem_u32(q_bufs + TILE_BYTES), 16, 1024)};
+      const uint64_t dq0 = sdesc_sw128(smem_u32(q_bufs), 16, 1024);
+      const uint64_t dq1 = sdesc_sw128(smem_u32(q_bufs + TILE_BYTES), 16, 1024);
       const uint64_t dk0 = sdesc_sw128(slot_addr0, 16, 1024);
       const uint64_t dv0 = sdesc_sw128(slot_addr0, HALF_BYTES, 1024);
       auto issue_s = [&](int st, int li) {
@@ -525,7 +527,7 @@ __global__ void DCA_FWD_BOUNDS
 #pragma unroll
         for (int kk = 0; kk < HD / 16; ++kk) {
           const uint64_t off = static_cast<uint64_t>(((kk >> 2) * HALF_BYTES + (kk & 3) * 32) >> 4);
-          mma_ss(tbase + static_cast<uint32_t>(st * 128), dq[st] + off, dk + off, id_s,
+          mma_ss(tbase + static_cast<uint32_t>(st * 128), (st ? dq1 : dq0) + off, dk + off, id_s,
                  kk > 0 ? 1u : 0u);
         }
       };
@@ -578,14 +580,18 @@ __global__ void DCA_FWD_BOUNDS
         const bool more = n + 1 < N;
         ok = full_wait(lv);
         if (!ok) break;
+        // the next key tile is normally resident long before it is needed;
+        // waiting for it here keeps the waits out of the unit's MMA burst
+        if (more) {
+          ok = full_wait(lk);
+          if (!ok) break;
+        }
         if (n < NA) {
           ok = pv_unit(0, n, lv);
           if (!ok) break;
           if (n + 1 == NA) mma_commit(&ctl->o_final[0]);
         }
         if (more) {
-          ok = full_wait(lk);
-          if (!ok) break;
           tc_fence_after();
           if (n + 1 < NA) {
             issue_s(0, lk);
