@@ -1,7 +1,7 @@
 // dca_softmax.cuh -- device helpers shared by the tcgen05 attention kernels:
 // bf16 packing, the software exp2 of part of the scores, query-row rotation
-// into the 128-byte-swizzled operand tile, the DCA class/causal mask of a
-// run of scores, and the exchange between the two threads of a row.
+// into the 128-byte-swizzled operand tile, and the exchange between the two
+// threads of a row.
 #pragma once
 #include <cuda_bf16.h>
 #include <math.h>
@@ -104,37 +104,6 @@ __device__ __forceinline__ void write_q_row(uint8_t* qb, int r, const __nv_bfloa
     const uint32_t phys = static_cast<uint32_t>((c ^ (r & 7)) * 16);
     *reinterpret_cast<uint4*>(qb + row_off + phys) = oa;
     *reinterpret_cast<uint4*>(qb + HALF_BYTES + row_off + phys) = ob;
-  }
-}
-
-// Mask NC consecutive scores of row i (keys j0 .. j0+NC-1) to the pairs that
-// are causal and belong to work-list class `cls` under window reading `reading`.
-template <int NC>
-__device__ __forceinline__ void mask_cols(uint32_t* sv, int64_t i, int64_t j0, int cls, int64_t s,
-                                          int64_t w, int reading) {
-  const int64_t ni = i / s;
-  const int64_t nj0 = j0 / s;
-  const int64_t dn64 = ni - nj0;
-  int dn = static_cast<int>(dn64 > (1 << 20) ? (1 << 20) : dn64);
-  const int64_t b64 = (nj0 + 1) * s - j0;  // first column of the next chunk
-  int bnd = static_cast<int>(b64 > (1 << 30) ? (1 << 30) : b64);
-  const int s32 = static_cast<int>(s > (1 << 30) ? (1 << 30) : s);
-  const int64_t lim64 = i - j0;  // last causal column; also i - j of column 0
-  const int lim = static_cast<int>(lim64 > 1024 ? 1024 : (lim64 < -1 ? -1 : lim64));
-  // i - j = (i - j0) - e, compared with w only under reading B
-  const int64_t far64 = lim64 - w;  // columns e <= far64 have i - j >= w
-  const int far = static_cast<int>(far64 > 1024 ? 1024 : (far64 < -1 ? -1 : far64));
-  const uint32_t NEG_INF = 0xff800000u;
-#pragma unroll
-  for (int e = 0; e < NC; ++e) {
-    if (e >= bnd) {
-      dn -= 1;
-      bnd += s32;
-    }
-    const int ce = dn <= 0 ? CLS_INTRA
-                           : ((dn == 1 && (reading == READING_A || e > far)) ? CLS_SUCC
-                                                                              : CLS_INTER);
-    if (e > lim || ce != cls) sv[e] = NEG_INF;
   }
 }
 

@@ -110,69 +110,72 @@ __device__ __forceinline__ uint64_t bits64(const uint32_t* row, int64_t lo) {
   return v;
 }
 
-// True when every bit of [lo, hi] (0 <= lo <= hi) is set.
-__device__ __forceinline__ bool all_bits(const uint32_t* row, int64_t lo, int64_t hi) {
-  for (int64_t b = lo; b <= hi; b += 64) {
-    const int64_t n = hi - b + 1 < 64 ? hi - b + 1 : 64;
-    const uint64_t want = n == 64 ? ~0ull : ((1ull << n) - 1);
-    if ((bits64(row, b) & want) != want) return false;
+// Columns of this thread's half-row of an item (64 keys) that are attended:
+// causal and of the item's class (the row's key range for the class), and
+// members -- for a slash window the keys on a slash diagonal of the head (or
+// j = i) that are not vertical keys, for a vertical tile the gathered keys
+// inside the list.  Bit e keeps column e.  Its global loads are issued one
+// item ahead, so they overlap the softmax of the current item.
+__device__ __forceinline__ uint64_t item_keep(int src, int64_t start, int cls, int64_t i, int half,
+                                              const Params& p, int h, int nv_eff, int64_t nb,
+                                              int64_t pb) {
+  if (src == 1) {
+    const int64_t j0 = start + 64 * half;  // first key of the half window
+    int64_t lo, hi;
+    row_key_range<int64_t>(i, cls, p.s, p.w, p.reading, lo, hi);
+    const int64_t a = lo - j0 < 0 ? 0 : (lo - j0 > 64 ? 64 : lo - j0);
+    const int64_t b = hi - j0 < a ? a : (hi - j0 > 64 ? 64 : hi - j0);
+    const uint64_t rng = (b >= 64 ? ~0ull : ((1ull << b) - 1)) & ~(a >= 64 ? ~0ull : ((1ull << a) - 1));
+    const uint32_t* vrow = p.vbit + static_cast<int64_t>(h) * p.wpr;
+    const uint32_t* srow = p.sbit + static_cast<int64_t>(h) * p.wpr;
+    const uint64_t vm = bits64(vrow, j0);
+    const int64_t base = i - j0;  // offset of key e is base - e
+    uint64_t sm = __brevll(bits64(srow, base - 63));
+    if (base >= 0 && base < 64) sm |= 1ull << base;
+    return rng & sm & ~vm;
   }
-  return true;
+  const int64_t pos0 = start + 64 * half;  // first gathered position
+  const int32_t* vk = p.vidx + static_cast<int64_t>(h) * p.nv_cap + pos0;
+  uint64_t keep = 0;
+#pragma unroll
+  for (int e4 = 0; e4 < 16; ++e4) {
+    int4 jj = make_int4(0x7fffffff, 0x7fffffff, 0x7fffffff, 0x7fffffff);
+    if (pos0 + 4 * e4 + 3 < nv_eff) {
+      jj = *reinterpret_cast<const int4*>(vk + 4 * e4);
+    } else {
+      if (pos0 + 4 * e4 + 0 < nv_eff) jj.x = vk[4 * e4 + 0];
+      if (pos0 + 4 * e4 + 1 < nv_eff) jj.y = vk[4 * e4 + 1];
+      if (pos0 + 4 * e4 + 2 < nv_eff) jj.z = vk[4 * e4 + 2];
+    }
+    const int js[4] = {jj.x, jj.y, jj.z, jj.w};
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int64_t j = js[u];
+      int c;
+      if (j >= nb) c = CLS_INTRA;
+      else if (j >= pb && (p.reading == READING_A || i - j < p.w)) c = CLS_SUCC;
+      else c = CLS_INTER;
+      if (j <= i && c == cls) keep |= 1ull << (4 * e4 + u);
+    }
+  }
+  return keep;
 }
 
 // One online-softmax step for half of a query row (see the dense kernel):
-// mask (when the item is not full) by causality, class and membership,
-// half-row max exchanged with the partner thread, exponentials into P (bf16,
-// first 64 columns of the S buffer), O rescaled when the reference moves
-// (after the previous item's P.V completed).
+// columns outside `keep` masked, half-row max exchanged with the partner
+// thread, exponentials into P (bf16, first 64 columns of the S buffer), O
+// rescaled when the reference moves (after the previous item's P.V
+// completed).
 __device__ __forceinline__ bool sparse_half_step(
-    uint32_t tS, uint32_t tO, int n, bool full, int src, int start, int cls, int64_t i,
-    const Params& p, int h, float sc, int64_t nb, int64_t pb, float& m_ref, float& l_sum,
-    PairCtx& pc, SmemCtl* ctl, volatile int* abort, unsigned int* status) {
+    uint32_t tS, uint32_t tO, int n, uint64_t keep, const Params& p, float sc, float& m_ref,
+    float& l_sum, PairCtx& pc, SmemCtl* ctl, volatile int* abort, unsigned int* status) {
   const int half = pc.half;
   uint32_t sv[64];
   tmem_ld64(tS + 64u * half, sv);
-  if (!full) {
-    const uint32_t NEG_INF = 0xff800000u;
-    if (src == 1) {
-      const int64_t j0 = start + 64 * half;  // first key of the window
-      mask_cols<64>(sv, i, j0, cls, p.s, p.w, p.reading);
-      const uint32_t* vrow = p.vbit + static_cast<int64_t>(h) * p.wpr;
-      const uint32_t* srow = p.sbit + static_cast<int64_t>(h) * p.wpr;
-      const uint64_t vm = bits64(vrow, j0);
-      const int64_t base = i - j0;  // offset of key e is base - e
-      uint64_t sm = __brevll(bits64(srow, base - 63));
-      if (base >= 0 && base < 64) sm |= 1ull << base;
-      const uint64_t mem = sm & ~vm;
+  if (keep != ~0ull) {
 #pragma unroll
-      for (int e = 0; e < 64; ++e)
-        if (!((mem >> e) & 1ull)) sv[e] = NEG_INF;
-    } else {
-      const int64_t pos0 = start + 64 * half;  // first gathered position
-      const int nv = ctl->plan.nv_eff;
-      const int32_t* vk = p.vidx + static_cast<int64_t>(h) * p.nv_cap + pos0;
-#pragma unroll
-      for (int e4 = 0; e4 < 16; ++e4) {
-        int4 jj = make_int4(0x7fffffff, 0x7fffffff, 0x7fffffff, 0x7fffffff);
-        if (pos0 + 4 * e4 + 3 < nv) {
-          jj = *reinterpret_cast<const int4*>(vk + 4 * e4);
-        } else {
-          if (pos0 + 4 * e4 + 0 < nv) jj.x = vk[4 * e4 + 0];
-          if (pos0 + 4 * e4 + 1 < nv) jj.y = vk[4 * e4 + 1];
-          if (pos0 + 4 * e4 + 2 < nv) jj.z = vk[4 * e4 + 2];
-        }
-        const int js[4] = {jj.x, jj.y, jj.z, jj.w};
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const int64_t j = js[u];
-          int c;
-          if (j >= nb) c = CLS_INTRA;
-          else if (j >= pb && (p.reading == READING_A || i - j < p.w)) c = CLS_SUCC;
-          else c = CLS_INTER;
-          if (j > i || c != cls) sv[4 * e4 + u] = NEG_INF;
-        }
-      }
-    }
+    for (int e = 0; e < 64; ++e)
+      if (!((keep >> e) & 1ull)) sv[e] = 0xff800000u;  // -inf
   }
   float mx = max64(sv);
   float mx_other = -INFINITY;
@@ -234,7 +237,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const int64_t i0 = p.q_start + static_cast<int64_t>(qt) * BM;
   const int64_t q_end = p.q_start + p.Lq;
   const int64_t i_last = (i0 + BM - 1 < q_end - 1) ? i0 + BM - 1 : q_end - 1;
-  const int64_t i_hi = i0 + BM - 1;
 
   if (threadIdx.x == 0) {
     for (int k = 0; k < NSLOT; ++k) {
@@ -312,54 +314,45 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     sparse_iter_init(it);
     float m_ref = -INFINITY, l_sum = 0.f;
     bool ok = true;
-    int src, start, cls;
-    for (int n = 0; n < N && ok; ++n) {
+    int src = 0, start = 0, cls = CLS_INTRA;
+    uint64_t keep = 0;
+    if (N > 0) {
       sparse_iter_next(it, plan, src, start, cls);
-      // full item: every pair causal, of this class and a member
-      bool full;
-      if (src == 1) {
-        const int64_t j0 = start, j1 = j0 + BN - 1;
-        full = item_is_full(i0, i_hi, j0, j1, p.s, p.w, cls, p.reading);
-        if (full) {
-          const uint32_t* vrow = p.vbit + static_cast<int64_t>(h) * p.wpr;
-          full = (bits64(vrow, j0) | bits64(vrow, j0 + 64)) == 0ull;
-        }
-        if (full) full = i0 - j1 >= 0 &&
-                         all_bits(p.sbit + static_cast<int64_t>(h) * p.wpr, i0 - j1, i_hi - j0);
-      } else {
-        const int64_t pos0 = start;
-        full = pos0 + BN <= plan.nv_eff;
-        if (full) {
-          const int32_t* vk = p.vidx + static_cast<int64_t>(h) * p.nv_cap;
-          const int64_t ja = vk[pos0], jb = vk[pos0 + BN - 1];
-          full = jb <= i0 && item_is_full(i0, i_hi, ja, jb, p.s, p.w, cls, p.reading);
-        }
-      }
+      keep = item_keep(src, start, cls, i, half, p, h, plan.nv_eff, nb, pb);
+    }
+    for (int n = 0; n < N && ok; ++n) {
       const int st = n & 1;
       ok = wait_poll(&ctl->s_full[st], static_cast<uint32_t>((n >> 1) & 1), abort_flag, p.status,
                      p.timeout_ns, ST_SOFTMAX);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
       tc_fence_after();
+      // the next item and its mask: their loads overlap this item's softmax
+      int src1 = src, start1 = start, cls1 = cls;
+      uint64_t keep1 = 0;
+      if (n + 1 < N) {
+        sparse_iter_next(it, plan, src1, start1, cls1);
+        keep1 = item_keep(src1, start1, cls1, i, half, p, h, plan.nv_eff, nb, pb);
+      }
       const uint32_t tS = tbase + lane_off + static_cast<uint32_t>(st * 128);
       const uint32_t tO = tbase + lane_off + 256u;
-      ok = sparse_half_step(tS, tO, n, full, src, start, cls, i, p, h, sc, nb, pb, m_ref, l_sum,
-                            pc, ctl, abort_flag, p.status);
+      ok = sparse_half_step(tS, tO, n, keep, p, sc, m_ref, l_sum, pc, ctl, abort_flag, p.status);
       if (!ok) break;
       // the first class ends: its operand tile becomes the third class's
-      if (plan.third_cls >= 0 && plan.qbuf_of[cls] == 0 && cls != plan.third_cls) {
-        SparseIter peek = it;
-        int s2, t2, c2;
-        if (n + 1 < N && sparse_iter_next(peek, plan, s2, t2, c2) && c2 != cls) {
-          const float2* trow =
-              real ? p.tab + query_table_row(i, plan.third_cls, p.s, p.w, p.tab_c1) * 64 : nullptr;
-          write_q_row(q_buf[0], r, qrow, trow, c0, c1);
-          fence_proxy_async_smem();
-        }
+      if (plan.third_cls >= 0 && plan.qbuf_of[cls] == 0 && cls != plan.third_cls &&
+          n + 1 < N && cls1 != cls) {
+        const float2* trow =
+            real ? p.tab + query_table_row(i, plan.third_cls, p.s, p.w, p.tab_c1) * 64 : nullptr;
+        write_q_row(q_buf[0], r, qrow, trow, c0, c1);
+        fence_proxy_async_smem();
       }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&ctl->p_full[st]);
+      src = src1;
+      start = start1;
+      cls = cls1;
+      keep = keep1;
     }
     // epilogue: O / (l_half0 + l_half1) -> bf16 -> out
     if (ok && N > 0) {
@@ -473,6 +466,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       for (int n = 0; n < N && ok; ++n) {
         const int lv = 2 * n + 1;
         ok = full_wait(lv);
+        // the next S's key tile too: a wait between the P.V and the S MMAs
+        // would leave the tensor pipe idle
+        if (ok && issued < N) ok = full_wait(2 * issued);
         if (!ok) break;
         ok = wait_spin(&ctl->p_full[n & 1], static_cast<uint32_t>((n >> 1) & 1), abort_flag,
                        p.status, p.timeout_ns, ST_MMA);
@@ -488,8 +484,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         mma_commit(&ctl->slot_empty[lv % NSLOT]);
         if (issued < N) {  // S(n + 2) reuses buffer n & 1 after P.V(n) (in issue order)
           sparse_iter_next(it, plan, src, start, cls);
-          ok = full_wait(2 * issued);
-          if (!ok) break;
           // the query operand of a class that reuses tile 0 is written by the
           // softmax warps before they release P(n); P.V(n) waited for that
           tc_fence_after();
