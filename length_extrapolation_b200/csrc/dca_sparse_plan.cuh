@@ -30,8 +30,6 @@ struct SparsePlan {
   int nv_eff;          // vertical keys <= the tile's last row
   int vt[3][2];        // vertical (gathered) tile range per class (indexed by CLS_*)
   int kr[3][2];        // cache key range [lo, hi) per class
-  int qbuf_of[3];      // query operand tile of each class, -1 if absent
-  int third_cls;       // class that reuses operand tile 0 (-1 if fewer than three)
   int2 iv[SPARSE_IV_MAX];  // [x, y) key ranges reached by the slashes, ascending
 };
 
@@ -99,49 +97,66 @@ DCA_HD bool sparse_iter_next(SparseIter& it, const SparsePlan& P, int& src, int&
   }
 }
 
-// Builds the plan of the query rows [i0, i_last] for a head with nvh sorted
-// vertical keys vk and nr slash runs (offset ranges [x, y), ascending, at most
-// SPARSE_IV_MAX - 1).  bn = 128.
-DCA_HD void sparse_plan_build(SparsePlan& P, const int32_t* vk, int nvh, const int2* runs, int nr,
-                              int64_t i0, int64_t i_last, int64_t s, int64_t w, int reading,
-                              int bn) {
-  int64_t klo[3], khi[3];
+// The plan is built in stages that the host and the kernel share; only the
+// lookups differ (the kernel loads the runs and searches the vertical list
+// with a whole warp).
+//
+// Stage 1: the class key ranges of the tile's rows.
+DCA_HD void sparse_plan_ranges(SparsePlan& P, int64_t i0, int64_t i_last, int64_t s, int64_t w,
+                               int reading, int64_t klo[3], int64_t khi[3]) {
   class_key_ranges(i0, i_last, s, w, reading, klo, khi);
   for (int c = 0; c < 3; ++c) {
     P.kr[c][0] = static_cast<int>(klo[c]);
     P.kr[c][1] = static_cast<int>(khi[c] > klo[c] ? khi[c] : klo[c]);
   }
-  // vertical tile ranges per class: positions of the class's key range
-  auto lower = [&](int64_t key) {
-    int lo = 0, hi = nvh;
-    while (lo < hi) {
-      const int mid = (lo + hi) >> 1;
-      if (vk[mid] < key) lo = mid + 1; else hi = mid;
-    }
-    return lo;
-  };
-  P.nv_eff = lower(i_last + 1);
+}
+
+// The keys whose position in the sorted vertical list the plan needs:
+// SPARSE_NKEYS lower bounds (i_last + 1, then lo and hi of each class).
+constexpr int SPARSE_NKEYS = 7;
+DCA_HD void sparse_plan_keys(int64_t i_last, const int64_t klo[3], const int64_t khi[3],
+                             int64_t key[SPARSE_NKEYS]) {
+  key[0] = i_last + 1;
+  for (int c = 0; c < 3; ++c) {
+    key[1 + 2 * c] = klo[c];
+    key[2 + 2 * c] = khi[c];
+  }
+}
+
+// Stage 2: vertical tile ranges per class from those lower bounds.
+DCA_HD void sparse_plan_vertical(SparsePlan& P, const int64_t klo[3], const int64_t khi[3],
+                                 const int pos[SPARSE_NKEYS], int bn) {
+  P.nv_eff = pos[0];
   for (int c = 0; c < 3; ++c) {
     int a = 0, b = 0;
     if (khi[c] > klo[c]) {
-      a = lower(klo[c]);
-      b = lower(khi[c]);
+      a = pos[1 + 2 * c];
+      b = pos[2 + 2 * c];
       if (b > P.nv_eff) b = P.nv_eff;
     }
     P.vt[c][0] = a / bn;
     P.vt[c][1] = b > a ? (b + bn - 1) / bn : a / bn;
   }
-  // slash key ranges: runs from the largest offsets down (ascending keys),
-  // the diagonal j = i always included; ranges closer than bn keys merged
+}
+
+// Stage 3: slash key ranges.  run_at(k) is the k-th run from the largest
+// offsets down (keys ascending), k < nr; the diagonal j = i comes last.
+// Ranges closer than bn keys are merged.  The output index never passes the
+// input index, so the runs may be staged in P.iv itself (run_at(k) reading
+// P.iv[k]).
+template <class RunAt>
+DCA_HD void sparse_plan_slash(SparsePlan& P, RunAt run_at, int nr, int64_t i0, int64_t i_last,
+                              int bn) {
   int n_iv = 0;
-  for (int r = nr; r >= 0; --r) {
+  for (int k = 0; k <= nr; ++k) {
     int64_t oa, ob;
-    if (r == 0) {
+    if (k == nr) {
       oa = 0;
       ob = 1;
     } else {
-      oa = runs[r - 1].x;
-      ob = runs[r - 1].y;
+      const int2 r = run_at(k);
+      oa = r.x;
+      ob = r.y;
     }
     if (oa > i_last) continue;
     int64_t ka = i0 - (ob - 1);
@@ -157,21 +172,38 @@ DCA_HD void sparse_plan_build(SparsePlan& P, const int32_t* vk, int nvh, const i
     }
   }
   P.n_iv = n_iv;
-  // item count; operand tiles alternate between the classes in order of appearance
-  for (int c = 0; c < 3; ++c) P.qbuf_of[c] = -1;
-  P.third_cls = -1;
+}
+
+// Stage 4: the item count.
+DCA_HD void sparse_plan_count(SparsePlan& P) {
   SparseIter it;
   sparse_iter_init(it);
-  int n_items = 0, src, start, cls, seen = 0;
-  while (sparse_iter_next(it, P, src, start, cls)) {
-    if (P.qbuf_of[cls] < 0) {
-      P.qbuf_of[cls] = seen & 1;
-      if (seen == 2) P.third_cls = cls;
-      ++seen;
-    }
-    ++n_items;
-  }
+  int n_items = 0, src, start, cls;
+  while (sparse_iter_next(it, P, src, start, cls)) ++n_items;
   P.n_items = n_items;
+}
+
+// Builds the plan of the query rows [i0, i_last] for a head with nvh sorted
+// vertical keys vk and nr slash runs (offset ranges [x, y), ascending, at most
+// SPARSE_IV_MAX - 1), one lookup at a time.  bn = 128.
+DCA_HD void sparse_plan_build(SparsePlan& P, const int32_t* vk, int nvh, const int2* runs, int nr,
+                              int64_t i0, int64_t i_last, int64_t s, int64_t w, int reading,
+                              int bn) {
+  int64_t klo[3], khi[3], key[SPARSE_NKEYS];
+  sparse_plan_ranges(P, i0, i_last, s, w, reading, klo, khi);
+  sparse_plan_keys(i_last, klo, khi, key);
+  int pos[SPARSE_NKEYS];
+  for (int e = 0; e < SPARSE_NKEYS; ++e) {
+    int lo = 0, hi = nvh;
+    while (lo < hi) {
+      const int mid = (lo + hi) >> 1;
+      if (vk[mid] < key[e]) lo = mid + 1; else hi = mid;
+    }
+    pos[e] = lo;
+  }
+  sparse_plan_vertical(P, klo, khi, pos, bn);
+  sparse_plan_slash(P, [&](int k) { return runs[nr - 1 - k]; }, nr, i0, i_last, bn);
+  sparse_plan_count(P);
 }
 
 }  // namespace dca

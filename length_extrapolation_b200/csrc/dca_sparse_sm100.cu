@@ -23,14 +23,18 @@
 // The slash windows come from the head's runs of consecutive offsets, merged
 // into key ranges once per CTA in shared memory (dca_sparse_plan.cuh).
 //
-// Warp roles as in the dense kernel (320 threads): warps 0-7 softmax (warp w
-// and w+4 split each row's 128 keys), warp 8 TMA producer (4-slot K/V ring,
-// no multicast), warp 9 MMA issuer.  With one head per CTA the two TMEM S
-// buffers alternate between consecutive items, so S(n+1) runs on the tensor
-// cores while the softmax warps work on S(n); P(n) overwrites the first 64
-// columns of its S buffer and feeds O += P V from TMEM.  Two query operand
-// tiles alternate between the classes in the order they appear (the third
-// class rewrites the first tile after the first class's last item).
+// Warps (320 threads): warps 0-7 softmax (warp w and w+4 split each row's 128
+// keys), warp 8 TMA producer (5-slot K/V ring, no multicast), warp 9 MMA
+// issuer.  With one head per CTA the two TMEM S buffers alternate between
+// consecutive items, so S(n+1) runs on the tensor cores while the softmax
+// warps work on S(n); P(n) overwrites the first 64 columns of its S buffer and
+// feeds O += P V from TMEM.  One query operand tile: where the class changes
+// between items n and n+1, the softmax warps rewrite it for the new class
+// after S(n) has completed and before they release P(n), and S(n+1) is issued
+// after P(n) instead of one item earlier.  Warp 0 builds the work list at the
+// start (runs staged in shared memory, the vertical-list searches done by the
+// whole warp); each softmax thread keeps its row's key range per class, so
+// an item's keep mask is a range test plus the membership bitmaps.
 // Every wait is bounded; on timeout the CTA raises its abort flag, ORs a code
 // into the device status word, drains its copies and MMAs and exits.
 #include <cuda_bf16.h>
@@ -48,7 +52,7 @@ namespace sp {
 using namespace attn;
 
 constexpr int BM = 128, BN = 128, HD = 128;
-constexpr int NSLOT = 4;
+constexpr int NSLOT = 5;
 constexpr int TILE_BYTES = 32768;
 constexpr int NUM_THREADS = 320;
 constexpr int WARP_LOAD = 8, WARP_MMA = 9;
@@ -72,7 +76,7 @@ struct SmemCtl {
   SparsePlan plan;
 };
 
-constexpr size_t SMEM_BYTES = 1024 + 2 * TILE_BYTES + NSLOT * TILE_BYTES + sizeof(SmemCtl);
+constexpr size_t SMEM_BYTES = 1024 + TILE_BYTES + NSLOT * TILE_BYTES + sizeof(SmemCtl);
 static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 
 struct Params {
@@ -98,67 +102,112 @@ struct Params {
 
 // 64 bits of a bitmap starting at bit `lo` (bits below 0 read as 0); the
 // bitmap row is padded with two zero words past its last bit.
-__device__ __forceinline__ uint64_t bits64(const uint32_t* row, int64_t lo) {
+__device__ __forceinline__ uint64_t bits64(const uint32_t* row, int lo) {
   if (lo <= -64) return 0ull;
-  const int64_t base = lo < 0 ? 0 : lo;
-  const int64_t wd = base >> 5;
-  const int sh = static_cast<int>(base & 31);
+  const int base = lo < 0 ? 0 : lo;
+  const int wd = base >> 5;
+  const int sh = base & 31;
   const uint64_t w0 = row[wd], w1 = row[wd + 1], w2 = row[wd + 2];
   uint64_t v = (w0 | (w1 << 32)) >> sh;
   if (sh) v |= w2 << (64 - sh);
-  if (lo < 0) v <<= static_cast<int>(-lo);
+  if (lo < 0) v <<= -lo;
   return v;
 }
 
 // Columns of this thread's half-row of an item (64 keys) that are attended:
-// causal and of the item's class (the row's key range for the class), and
-// members -- for a slash window the keys on a slash diagonal of the head (or
-// j = i) that are not vertical keys, for a vertical tile the gathered keys
-// inside the list.  Bit e keeps column e.  Its global loads are issued one
-// item ahead, so they overlap the softmax of the current item.
-__device__ __forceinline__ uint64_t item_keep(int src, int64_t start, int cls, int64_t i, int half,
-                                              const Params& p, int h, int nv_eff, int64_t nb,
-                                              int64_t pb) {
+// inside the row's key range [lo, hi) for the item's class (causality
+// included), and members -- for a slash window the keys on a slash diagonal
+// of the head (or j = i) that are not vertical keys, for a vertical tile the
+// gathered keys inside the range.  Bit e keeps column e.  Computed one item
+// ahead, so its loads overlap the softmax of the current item.
+__device__ __forceinline__ uint64_t item_keep(int src, int start, int i, int half, int lo, int hi,
+                                              const uint32_t* vrow, const uint32_t* srow,
+                                              const int32_t* vk, int nv_eff) {
   if (src == 1) {
-    const int64_t j0 = start + 64 * half;  // first key of the half window
-    int64_t lo, hi;
-    row_key_range<int64_t>(i, cls, p.s, p.w, p.reading, lo, hi);
-    const int64_t a = lo - j0 < 0 ? 0 : (lo - j0 > 64 ? 64 : lo - j0);
-    const int64_t b = hi - j0 < a ? a : (hi - j0 > 64 ? 64 : hi - j0);
+    const int j0 = start + 64 * half;  // first key of the half window
+    const int a = min(max(lo - j0, 0), 64);
+    const int b = min(max(hi - j0, a), 64);
     const uint64_t rng = (b >= 64 ? ~0ull : ((1ull << b) - 1)) & ~(a >= 64 ? ~0ull : ((1ull << a) - 1));
-    const uint32_t* vrow = p.vbit + static_cast<int64_t>(h) * p.wpr;
-    const uint32_t* srow = p.sbit + static_cast<int64_t>(h) * p.wpr;
     const uint64_t vm = bits64(vrow, j0);
-    const int64_t base = i - j0;  // offset of key e is base - e
+    const int base = i - j0;  // offset of key e is base - e
     uint64_t sm = __brevll(bits64(srow, base - 63));
     if (base >= 0 && base < 64) sm |= 1ull << base;
     return rng & sm & ~vm;
   }
-  const int64_t pos0 = start + 64 * half;  // first gathered position
-  const int32_t* vk = p.vidx + static_cast<int64_t>(h) * p.nv_cap + pos0;
+  const int pos0 = start + 64 * half;  // first gathered position
+  const int32_t* v = vk + pos0;
   uint64_t keep = 0;
 #pragma unroll
   for (int e4 = 0; e4 < 16; ++e4) {
     int4 jj = make_int4(0x7fffffff, 0x7fffffff, 0x7fffffff, 0x7fffffff);
     if (pos0 + 4 * e4 + 3 < nv_eff) {
-      jj = *reinterpret_cast<const int4*>(vk + 4 * e4);
+      jj = *reinterpret_cast<const int4*>(v + 4 * e4);
     } else {
-      if (pos0 + 4 * e4 + 0 < nv_eff) jj.x = vk[4 * e4 + 0];
-      if (pos0 + 4 * e4 + 1 < nv_eff) jj.y = vk[4 * e4 + 1];
-      if (pos0 + 4 * e4 + 2 < nv_eff) jj.z = vk[4 * e4 + 2];
+      if (pos0 + 4 * e4 + 0 < nv_eff) jj.x = v[4 * e4 + 0];
+      if (pos0 + 4 * e4 + 1 < nv_eff) jj.y = v[4 * e4 + 1];
+      if (pos0 + 4 * e4 + 2 < nv_eff) jj.z = v[4 * e4 + 2];
     }
     const int js[4] = {jj.x, jj.y, jj.z, jj.w};
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const int64_t j = js[u];
-      int c;
-      if (j >= nb) c = CLS_INTRA;
-      else if (j >= pb && (p.reading == READING_A || i - j < p.w)) c = CLS_SUCC;
-      else c = CLS_INTER;
-      if (j <= i && c == cls) keep |= 1ull << (4 * e4 + u);
-    }
+    for (int u = 0; u < 4; ++u)
+      if (js[u] >= lo && js[u] < hi) keep |= 1ull << (4 * e4 + u);
   }
   return keep;
+}
+
+// The work list of the CTA, built by one warp: the slash runs staged in
+// P.iv (highest offsets first) with coalesced loads, the lower bounds of
+// SPARSE_NKEYS keys in the sorted vertical list found together (each round
+// samples 32 evenly spaced positions of every key's remaining interval and
+// keeps the one sub-interval that can hold the bound; 1024 keys take two
+// rounds), then lane 0 merges the ranges and counts the items.
+__device__ void plan_build_warp(SparsePlan& P, const int32_t* vk, int nvh, const int2* runs,
+                                int nr, int64_t i0, int64_t i_last, int64_t s, int64_t w,
+                                int reading, int lane) {
+  for (int r = lane; r < nr; r += 32) P.iv[nr - 1 - r] = runs[r];
+  int64_t klo[3], khi[3], key[SPARSE_NKEYS];
+  if (lane == 0) sparse_plan_ranges(P, i0, i_last, s, w, reading, klo, khi);
+  else class_key_ranges(i0, i_last, s, w, reading, klo, khi);
+  sparse_plan_keys(i_last, klo, khi, key);
+  int lo[SPARSE_NKEYS], len[SPARSE_NKEYS];
+#pragma unroll
+  for (int e = 0; e < SPARSE_NKEYS; ++e) {
+    lo[e] = 0;
+    len[e] = nvh;
+  }
+  for (;;) {
+    bool more = false;
+#pragma unroll
+    for (int e = 0; e < SPARSE_NKEYS; ++e) more |= len[e] > 0;
+    if (!more) break;
+    int v[SPARSE_NKEYS], st[SPARSE_NKEYS];
+#pragma unroll
+    for (int e = 0; e < SPARSE_NKEYS; ++e) {
+      st[e] = (len[e] + 31) >> 5;
+      const int q = lane * st[e];
+      v[e] = (len[e] > 0 && q < len[e]) ? vk[lo[e] + q] : 0x7fffffff;
+    }
+#pragma unroll
+    for (int e = 0; e < SPARSE_NKEYS; ++e) {
+      if (len[e] == 0) continue;  // uniform across the warp
+      const int c = __popc(__ballot_sync(0xffffffffu, static_cast<int64_t>(v[e]) < key[e]));
+      if (c == 0) {
+        len[e] = 0;
+      } else {
+        const int end = lo[e] + len[e];
+        const int nlo = lo[e] + (c - 1) * st[e] + 1;
+        const int nend = min(lo[e] + c * st[e], end);
+        lo[e] = nlo;
+        len[e] = nend - nlo;
+      }
+    }
+  }
+  __syncwarp();
+  if (lane == 0) {
+    sparse_plan_vertical(P, klo, khi, lo, 128);
+    sparse_plan_slash(P, [&](int k) { return P.iv[k]; }, nr, i0, i_last, 128);
+    sparse_plan_count(P);
+  }
 }
 
 // One online-softmax step for half of a query row (see the dense kernel):
@@ -222,8 +271,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-  uint8_t* q_buf[2] = {smem, smem + TILE_BYTES};
-  uint8_t* slots = smem + 2 * TILE_BYTES;
+  uint8_t* q_buf = smem;
+  uint8_t* slots = smem + TILE_BYTES;
   SmemCtl* ctl = reinterpret_cast<SmemCtl*>(slots + NSLOT * TILE_BYTES);
 
   const int warp = threadIdx.x >> 5;
@@ -254,11 +303,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     for (int k = 0; k < 4; ++k) mbar_init(&ctl->pair_bar[k], 2);
     ctl->abort = 0;
     fence_barrier_init();
-
+  }
+  if (warp == 0) {
     // ---- the CTA's work list
-    sparse_plan_build(ctl->plan, p.vidx + static_cast<int64_t>(h) * p.nv_cap, p.nv[h],
-                      p.runs + static_cast<int64_t>(h) * SPARSE_MAX_RUNS, p.nruns[h], i0, i_last,
-                      p.s, p.w, p.reading, BN);
+    plan_build_warp(ctl->plan, p.vidx + static_cast<int64_t>(h) * p.nv_cap, p.nv[h],
+                    p.runs + static_cast<int64_t>(h) * SPARSE_MAX_RUNS, p.nruns[h], i0, i_last,
+                    p.s, p.w, p.reading, lane);
   }
   if (warp == WARP_MMA) {
     tmem_alloc(&ctl->tmem_base, 512);
@@ -297,18 +347,29 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const __nv_bfloat16* qrow =
         real ? p.q + ((i - p.q_start) * p.Hq + h) * static_cast<int64_t>(HD) : nullptr;
     const int c0 = 4 * half, c1 = 4 * half + 4;
-    const int64_t nb = (i / p.s) * p.s, pb = nb - p.s;  // chunk start of row i, and the previous
-    // query operands of the first two classes
+    // the row's key range per class (a padding row past the block keeps none)
+    int klo[3], khi[3];
 #pragma unroll
     for (int c = 0; c < 3; ++c) {
-      const int b = plan.qbuf_of[c];
-      if (b < 0 || c == plan.third_cls) continue;
-      const float2* trow = real ? p.tab + query_table_row(i, c, p.s, p.w, p.tab_c1) * 64 : nullptr;
-      write_q_row(q_buf[b], r, qrow, trow, c0, c1);
+      klo[c] = khi[c] = 0;
+      if (real)
+        row_key_range<int>(static_cast<int>(i), c, static_cast<int>(p.s), static_cast<int>(p.w),
+                           p.reading, klo[c], khi[c]);
     }
-    fence_proxy_async_smem();
-    __syncwarp();
-    if (lane == 0) mbar_arrive(&ctl->q_ready);
+    const uint32_t* vrow = p.vbit + static_cast<int64_t>(h) * p.wpr;
+    const uint32_t* srow = p.sbit + static_cast<int64_t>(h) * p.wpr;
+    const int32_t* vk = p.vidx + static_cast<int64_t>(h) * p.nv_cap;
+    const int ii = static_cast<int>(i);
+    auto keep_of = [&](int src_, int start_, int cls_) {
+      const int lo = cls_ == 0 ? klo[0] : (cls_ == 1 ? klo[1] : klo[2]);
+      const int hi = cls_ == 0 ? khi[0] : (cls_ == 1 ? khi[1] : khi[2]);
+      return item_keep(src_, start_, ii, half, lo, hi, vrow, srow, vk, plan.nv_eff);
+    };
+    auto write_q = [&](int cls_) {
+      const float2* trow = real ? p.tab + query_table_row(i, cls_, p.s, p.w, p.tab_c1) * 64 : nullptr;
+      write_q_row(q_buf, r, qrow, trow, c0, c1);
+      fence_proxy_async_smem();
+    };
 
     SparseIter it;
     sparse_iter_init(it);
@@ -318,8 +379,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     uint64_t keep = 0;
     if (N > 0) {
       sparse_iter_next(it, plan, src, start, cls);
-      keep = item_keep(src, start, cls, i, half, p, h, plan.nv_eff, nb, pb);
+      keep = keep_of(src, start, cls);
+      write_q(cls);  // the first class's query operand
     }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&ctl->q_ready);
+
     for (int n = 0; n < N && ok; ++n) {
       const int st = n & 1;
       ok = wait_poll(&ctl->s_full[st], static_cast<uint32_t>((n >> 1) & 1), abort_flag, p.status,
@@ -332,20 +397,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       uint64_t keep1 = 0;
       if (n + 1 < N) {
         sparse_iter_next(it, plan, src1, start1, cls1);
-        keep1 = item_keep(src1, start1, cls1, i, half, p, h, plan.nv_eff, nb, pb);
+        keep1 = keep_of(src1, start1, cls1);
       }
       const uint32_t tS = tbase + lane_off + static_cast<uint32_t>(st * 128);
       const uint32_t tO = tbase + lane_off + 256u;
       ok = sparse_half_step(tS, tO, n, keep, p, sc, m_ref, l_sum, pc, ctl, abort_flag, p.status);
       if (!ok) break;
-      // the first class ends: its operand tile becomes the third class's
-      if (plan.third_cls >= 0 && plan.qbuf_of[cls] == 0 && cls != plan.third_cls &&
-          n + 1 < N && cls1 != cls) {
-        const float2* trow =
-            real ? p.tab + query_table_row(i, plan.third_cls, p.s, p.w, p.tab_c1) * 64 : nullptr;
-        write_q_row(q_buf[0], r, qrow, trow, c0, c1);
-        fence_proxy_async_smem();
-      }
+      // a class change: S(n) has completed, S(n + 1) waits for P(n), so the
+      // operand tile is free for the next class's rotation
+      if (n + 1 < N && cls1 != cls) write_q(cls1);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&ctl->p_full[st]);
@@ -428,47 +488,58 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     if (lane == 0) {
       const uint32_t id_s = idesc_bf16_f32(BM, BN, false);
       const uint32_t id_o = idesc_bf16_f32(BM, HD, true);
-      const uint64_t dq[2] = {sdesc_sw128(smem_u32(q_buf[0]), 16, 1024),
-                              sdesc_sw128(smem_u32(q_buf[1]), 16, 1024)};
+      const uint64_t dq = sdesc_sw128(smem_u32(q_buf), 16, 1024);
       const uint64_t dk0 = sdesc_sw128(smem_u32(slots), 16, 1024);
       const uint64_t dv0 = sdesc_sw128(smem_u32(slots), HALF_BYTES, 1024);
       auto full_wait = [&](int li) {
         return wait_spin(&ctl->slot_full[li % NSLOT], static_cast<uint32_t>((li / NSLOT) & 1),
                          abort_flag, p.status, p.timeout_ns, ST_MMA);
       };
+      // S(k) into buffer k & 1; items come from the issue cursor
       SparseIter it;
       sparse_iter_init(it);
-      int src, start, cls;
-      // S(n) into buffer n & 1 with the class's query operand
-      auto issue_s = [&](int n) {
-        const int li = 2 * n;
+      int src, start, cls_next = -1, cls_prev = -1;
+      int issued = 0;  // S issued for items < issued
+      auto peek = [&]() {  // class of item `issued` (the cursor's next item)
+        if (issued >= N) return;
+        SparseIter t = it;
+        int s_, st_;
+        sparse_iter_next(t, plan, s_, st_, cls_next);
+      };
+      auto issue_s = [&]() {
+        sparse_iter_next(it, plan, src, start, cls_prev);
+        const int li = 2 * issued;
         const uint64_t dk = dk0 + static_cast<uint64_t>(((li % NSLOT) * TILE_BYTES) >> 4);
-        const uint64_t dqc = dq[plan.qbuf_of[cls]];
 #pragma unroll
         for (int kk = 0; kk < HD / 16; ++kk) {
           const uint64_t off = static_cast<uint64_t>(((kk >> 2) * HALF_BYTES + (kk & 3) * 32) >> 4);
-          mma_ss(tbase + static_cast<uint32_t>((n & 1) * 128), dqc + off, dk + off, id_s,
+          mma_ss(tbase + static_cast<uint32_t>((issued & 1) * 128), dq + off, dk + off, id_s,
                  kk > 0 ? 1u : 0u);
         }
-        mma_commit(&ctl->s_full[n & 1]);
+        mma_commit(&ctl->s_full[issued & 1]);
         mma_commit(&ctl->slot_empty[li % NSLOT]);
+        ++issued;
+        peek();
+      };
+      // S(k) may go once P.V(k - 2) is issued (its buffer), and, where the
+      // class changes, once P(k - 1) is released (the operand tile)
+      auto can_issue = [&](int n_done) {  // P.V issued for items < n_done
+        return issued < N && issued <= n_done + 1 && (issued <= n_done || cls_next == cls_prev);
       };
       bool ok = wait_bounded(&ctl->q_ready, 0u, abort_flag, p.status, p.timeout_ns, ST_MMA);
-      int issued = 0;  // S issued for items < issued
-      for (int k = 0; k < 2 && k < N && ok; ++k) {
-        sparse_iter_next(it, plan, src, start, cls);
-        ok = full_wait(2 * k);
+      peek();
+      while (ok && can_issue(0)) {
+        ok = full_wait(2 * issued);
         if (!ok) break;
         tc_fence_after();
-        issue_s(k);
-        ++issued;
+        issue_s();
       }
       for (int n = 0; n < N && ok; ++n) {
         const int lv = 2 * n + 1;
         ok = full_wait(lv);
         // the next S's key tile too: a wait between the P.V and the S MMAs
         // would leave the tensor pipe idle
-        if (ok && issued < N) ok = full_wait(2 * issued);
+        if (ok && can_issue(n + 1)) ok = full_wait(2 * issued);
         if (!ok) break;
         ok = wait_spin(&ctl->p_full[n & 1], static_cast<uint32_t>((n >> 1) & 1), abort_flag,
                        p.status, p.timeout_ns, ST_MMA);
@@ -482,13 +553,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
         mma_commit(&ctl->pv_done[n & 1]);
         mma_commit(&ctl->slot_empty[lv % NSLOT]);
-        if (issued < N) {  // S(n + 2) reuses buffer n & 1 after P.V(n) (in issue order)
-          sparse_iter_next(it, plan, src, start, cls);
-          // the query operand of a class that reuses tile 0 is written by the
-          // softmax warps before they release P(n); P.V(n) waited for that
+        while (ok && can_issue(n + 1)) {
+          ok = full_wait(2 * issued);
+          if (!ok) break;
           tc_fence_after();
-          issue_s(issued);
-          ++issued;
+          issue_s();
         }
       }
       if (ok && N > 0) mma_commit(&ctl->o_final);
