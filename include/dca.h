@@ -280,7 +280,9 @@ int dca_sparse_pattern_get(const dca_sparse_config* cfg, int Hq, const void* spa
  * (start a multiple of 128), src 1 = the 128 cache keys start .. start + 127,
  * a window over what the slash diagonals and the diagonal j = i reach from
  * the tile's rows; class as in dca_plan_items.  Returns the number of items
- * (which may exceed max_items) or DCA_ERR_ARG.
+ * (which may exceed max_items) or DCA_ERR_ARG; DCA_ERR_UNSUPPORTED if the
+ * plan's item count disagrees with its list (an internal consistency check:
+ * the kernels size their loops by that count).
  */
 int dca_sparse_plan_items(const int32_t* v_idx, int64_t n_v, const int32_t* s_off, int64_t n_s,
                           int64_t i0, int64_t i_last, int64_t chunk_size, int64_t local_window,

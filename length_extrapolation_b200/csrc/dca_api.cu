@@ -768,6 +768,8 @@ int dca_sparse_plan_items(const int32_t* v_idx, int64_t n_v, const int32_t* s_of
     }
     ++n;
   }
+  // the kernels size their loops by the plan's count: it must match the list
+  if (n != P[0].n_items) return DCA_ERR_UNSUPPORTED;
   return n;
 }
 

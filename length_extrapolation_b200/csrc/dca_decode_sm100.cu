@@ -198,33 +198,55 @@ __global__ void __launch_bounds__(Cfg<NR>::THREADS, 1)
     // swizzle) of the classes in the work list (the RoPE table holds the
     // positions s + r only when the cache extends past the first chunk, which
     // is when the list has successive-chunk items); task = (class, row,
-    // 8-dim chunk of each half).
-    for (int task = warp * 32 + lane; task < 3 * NR * 8; task += 32 * SW) {
+    // 8-dim chunk of each half), 3 NR 8 tasks over 32 SW = 8 NR threads:
+    // three per thread, their loads all issued before the first use.
+    constexpr int QTASKS = 3;
+    static_assert(3 * NR * 8 == QTASKS * 32 * SW, "three query tasks per softmax thread");
+    uint4 xa[QTASKS], xb[QTASKS];
+    float4 cs[QTASKS][4];
+    bool live[QTASKS];
+#pragma unroll
+    for (int u = 0; u < QTASKS; ++u) {
+      const int task = warp * 32 + lane + u * 32 * SW;
       const int cls = task / (NR * 8);
       const int rho = (task >> 3) % NR;
       const int c = task & 7;
-      uint4 oa = make_uint4(0, 0, 0, 0), ob = oa;
-      if (rho < n_rows && p.plan.hi[cls] > p.plan.lo[cls]) {
+      live[u] = rho < n_rows && p.plan.hi[cls] > p.plan.lo[cls];
+      xa[u] = xb[u] = make_uint4(0, 0, 0, 0);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) cs[u][e] = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (live[u]) {
         const int64_t rho_g = static_cast<int64_t>(rg) * NR + rho;
         const int64_t t = rho_g / p.G;
         const int h = g * p.G + static_cast<int>(rho_g % p.G);
         const __nv_bfloat16* qrow = p.q + (t * p.Hq + h) * static_cast<int64_t>(HD);
-        const float2* trow =
-            p.tab + query_table_row(p.q_start + t, cls, p.s, p.w, p.tab_c1) * (HD / 2);
-        const uint4 xa = *reinterpret_cast<const uint4*>(qrow + 8 * c);
-        const uint4 xb = *reinterpret_cast<const uint4*>(qrow + 64 + 8 * c);
-        const float4* t4 = reinterpret_cast<const float4*>(trow + 8 * c);
-        const __nv_bfloat162* a2 = reinterpret_cast<const __nv_bfloat162*>(&xa);
-        const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&xb);
+        const float4* t4 = reinterpret_cast<const float4*>(
+            p.tab + query_table_row(p.q_start + t, cls, p.s, p.w, p.tab_c1) * (HD / 2) + 8 * c);
+        xa[u] = *reinterpret_cast<const uint4*>(qrow + 8 * c);
+        xb[u] = *reinterpret_cast<const uint4*>(qrow + 64 + 8 * c);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) cs[u][e] = t4[e];
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < QTASKS; ++u) {
+      const int task = warp * 32 + lane + u * 32 * SW;
+      const int cls = task / (NR * 8);
+      const int rho = (task >> 3) % NR;
+      const int c = task & 7;
+      uint4 oa = make_uint4(0, 0, 0, 0), ob = oa;
+      if (live[u]) {
+        const __nv_bfloat162* a2 = reinterpret_cast<const __nv_bfloat162*>(&xa[u]);
+        const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&xb[u]);
         uint32_t* pa = reinterpret_cast<uint32_t*>(&oa);
         uint32_t* pb = reinterpret_cast<uint32_t*>(&ob);
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          const float4 cs = t4[e];
+          const float4 r = cs[u][e];
           const float2 x = __bfloat1622float2(a2[e]);
           const float2 y = __bfloat1622float2(b2[e]);
-          pa[e] = pack_bf16(x.x * cs.x - y.x * cs.y, x.y * cs.z - y.y * cs.w);
-          pb[e] = pack_bf16(x.x * cs.y + y.x * cs.x, x.y * cs.w + y.y * cs.z);
+          pa[e] = pack_bf16(x.x * r.x - y.x * r.y, x.y * r.z - y.y * r.w);
+          pb[e] = pack_bf16(x.x * r.y + y.x * r.x, x.y * r.w + y.y * r.z);
         }
       }
       uint8_t* dst = qv + cls * OPB + rho * 128 + ((c ^ (rho & 7)) << 4);
@@ -525,10 +547,11 @@ __global__ void __launch_bounds__(Cfg<NR>::THREADS, 1)
 // Merge the slices of each (token, head) row: with slice maxima m_k (log2
 // units), sums l_k and unnormalised outputs O_k, out = sum_k 2^(m_k - M) O_k /
 // sum_k 2^(m_k - M) l_k with M = max m_k; LSE (natural log) = (M + log2 of the
-// denominator) ln 2.  One CTA per row, one thread per dim: the slices'
-// (m, l) are fetched in parallel into shared memory, then each thread streams
-// its dim of the O_k with independent loads.
+// denominator) ln 2.  One CTA per row, one thread per dim: it loads the
+// first MERGE_BATCH slices' values of its dim, fetches the slices' (m, l)
+// into shared memory while those loads are in flight, then accumulates.
 constexpr int MERGE_MAX_SPLITS = DECODE_MAX_CTAS;
+constexpr int MERGE_BATCH = 32;
 
 __global__ void __launch_bounds__(HD)
     dca_decode_combine_kernel(const float* __restrict__ part, __nv_bfloat16* __restrict__ out,
@@ -546,12 +569,18 @@ __global__ void __launch_bounds__(HD)
   const float* pm = part + static_cast<size_t>(n_cta) * nr * HD;
   const float* pl = pm + static_cast<size_t>(n_cta) * nr;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const float* po = part + (static_cast<size_t>(c0) * nr + rho) * HD + tid;
+  const size_t stride = static_cast<size_t>(nr) * HD;
+
+  float ov[MERGE_BATCH];
+#pragma unroll
+  for (int u = 0; u < MERGE_BATCH; ++u) ov[u] = u < n_splits ? __ldcg(po + u * stride) : 0.f;
 
   float mx = -INFINITY;
   for (int k = tid; k < n_splits; k += HD) {
-    const float m = pm[(c0 + k) * nr + rho];
+    const float m = __ldcg(pm + (c0 + k) * nr + rho);
     wk[k] = m;
-    lk[k] = pl[(c0 + k) * nr + rho];
+    lk[k] = __ldcg(pl + (c0 + k) * nr + rho);
     mx = fmaxf(mx, m);
   }
 #pragma unroll
@@ -572,15 +601,17 @@ __global__ void __launch_bounds__(HD)
   __syncthreads();
   const float L = red[0] + red[1] + red[2] + red[3];
 
-  const float* po = part + (static_cast<size_t>(c0) * nr + rho) * HD + tid;
-  const size_t stride = static_cast<size_t>(nr) * HD;
   float acc[4] = {0.f, 0.f, 0.f, 0.f};
-  int k = 0;
-  for (; k + 4 <= n_splits; k += 4) {
+  for (int k0 = 0; k0 < n_splits; k0 += MERGE_BATCH) {
+    if (k0 > 0) {
 #pragma unroll
-    for (int u = 0; u < 4; ++u) acc[u] = fmaf(wk[k + u], po[(k + u) * stride], acc[u]);
+      for (int u = 0; u < MERGE_BATCH; ++u)
+        ov[u] = k0 + u < n_splits ? __ldcg(po + (k0 + u) * stride) : 0.f;
+    }
+#pragma unroll
+    for (int u = 0; u < MERGE_BATCH; ++u)
+      if (k0 + u < n_splits) acc[u & 3] = fmaf(wk[k0 + u], ov[u], acc[u & 3]);
   }
-  for (; k < n_splits; ++k) acc[0] = fmaf(wk[k], po[k * stride], acc[0]);
   const float o = (acc[0] + acc[1]) + (acc[2] + acc[3]);
   out[static_cast<size_t>(row) * HD + tid] = __float2bfloat16_rn(o / L);
   if (lse != nullptr && tid == 0) lse[row] = (M + log2f(L)) * 0.6931471805599453f;

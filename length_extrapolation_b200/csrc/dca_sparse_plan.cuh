@@ -174,13 +174,25 @@ DCA_HD void sparse_plan_slash(SparsePlan& P, RunAt run_at, int nr, int64_t i0, i
   P.n_iv = n_iv;
 }
 
-// Stage 4: the item count.
+// Stage 4: the item count, range by range (the iterator's windows: per
+// class, the vertical tiles, then each slash range clipped to the class's
+// key range, ceil(length / 128) windows).
+DCA_HD int sparse_range_items(int2 r, const int kr[3][2]) {
+  int n = 0;
+  for (int c = 0; c < 3; ++c) {
+    const int a = r.x > kr[c][0] ? r.x : kr[c][0];
+    const int b = r.y < kr[c][1] ? r.y : kr[c][1];
+    if (a < b) n += (b - a + 127) / 128;
+  }
+  return n;
+}
+DCA_HD int sparse_vertical_items(const SparsePlan& P) {
+  return (P.vt[0][1] - P.vt[0][0]) + (P.vt[1][1] - P.vt[1][0]) + (P.vt[2][1] - P.vt[2][0]);
+}
 DCA_HD void sparse_plan_count(SparsePlan& P) {
-  SparseIter it;
-  sparse_iter_init(it);
-  int n_items = 0, src, start, cls;
-  while (sparse_iter_next(it, P, src, start, cls)) ++n_items;
-  P.n_items = n_items;
+  int n = sparse_vertical_items(P);
+  for (int r = 0; r < P.n_iv; ++r) n += sparse_range_items(P.iv[r], P.kr);
+  P.n_items = n;
 }
 
 // Builds the plan of the query rows [i0, i_last] for a head with nvh sorted

@@ -25,10 +25,10 @@
 //
 // Warps (320 threads): warps 0-7 softmax (warp w and w+4 split each row's 128
 // keys), warp 8 TMA producer (5-slot K/V ring, no multicast), warp 9 MMA
-// issuer.  With one head per CTA the two TMEM S buffers alternate between
-// consecutive items, so S(n+1) runs on the tensor cores while the softmax
-// warps work on S(n); P(n) overwrites the first 64 columns of its S buffer and
-// feeds O += P V from TMEM.  One query operand tile: where the class changes
+// issuer.  With one head per CTA three TMEM S buffers rotate over
+// consecutive items, so S(n+1) and S(n+2) run on the tensor cores while the
+// softmax warps work on S(n); P(n) overwrites the first 64 columns of its S
+// buffer and feeds O += P V from TMEM.  One query operand tile: where the class changes
 // between items n and n+1, the softmax warps rewrite it for the new class
 // after S(n) has completed and before they release P(n), and S(n+1) is issued
 // after P(n) instead of one item earlier.  Warp 0 builds the work list at the
@@ -53,6 +53,8 @@ using namespace attn;
 
 constexpr int BM = 128, BN = 128, HD = 128;
 constexpr int NSLOT = 5;
+constexpr int NSBUF = 3;                 // S buffers in TMEM (P aliases their first 64 columns)
+constexpr uint32_t COL_O = NSBUF * 128;  // O after them
 constexpr int TILE_BYTES = 32768;
 constexpr int NUM_THREADS = 320;
 constexpr int WARP_LOAD = 8, WARP_MMA = 9;
@@ -63,8 +65,8 @@ constexpr unsigned ST_SOFTMAX = 0x10u, ST_LOAD = 0x100u, ST_MMA = 0x1000u, ST_DR
 struct SmemCtl {
   uint64_t slot_full[NSLOT];
   uint64_t slot_empty[NSLOT];
-  uint64_t s_full[2];
-  uint64_t p_full[2];
+  uint64_t s_full[NSBUF];
+  uint64_t p_full[NSBUF];
   uint64_t pv_done[2];
   uint64_t q_ready;
   uint64_t o_final;
@@ -100,59 +102,72 @@ struct Params {
   unsigned long long timeout_ns;
 };
 
-// 64 bits of a bitmap starting at bit `lo` (bits below 0 read as 0); the
-// bitmap row is padded with two zero words past its last bit.
-__device__ __forceinline__ uint64_t bits64(const uint32_t* row, int lo) {
-  if (lo <= -64) return 0ull;
-  const int base = lo < 0 ? 0 : lo;
-  const int wd = base >> 5;
-  const int sh = base & 31;
-  const uint64_t w0 = row[wd], w1 = row[wd + 1], w2 = row[wd + 2];
-  uint64_t v = (w0 | (w1 << 32)) >> sh;
-  if (sh) v |= w2 << (64 - sh);
-  if (lo < 0) v <<= -lo;
-  return v;
-}
-
+// Bitmap rows are padded with two zero words past their last bit; bits below
+// 0 read as 0.
 // Columns of this thread's half-row of an item (64 keys) that are attended:
 // inside the row's key range [lo, hi) for the item's class (causality
 // included), and members -- for a slash window the keys on a slash diagonal
 // of the head (or j = i) that are not vertical keys, for a vertical tile the
-// gathered keys inside the range.  Bit e keeps column e.  Computed one item
-// ahead, so its loads overlap the softmax of the current item.
-__device__ __forceinline__ uint64_t item_keep(int src, int start, int i, int half, int lo, int hi,
-                                              const uint32_t* vrow, const uint32_t* srow,
-                                              const int32_t* vk, int nv_eff) {
+// row's positions [pa, pb) of the gathered list for the class.  Bit e keeps
+// column e.  keep_fetch issues the bitmap loads of the next item before the
+// current item's softmax; keep_finish forms the mask after it.
+struct KeepFetch {
+  uint32_t v[3], s[3];  // vertical bits from key j0, slash bits from offset i - j0 - 63
+  int src, a, b;        // slash: kept columns [a, b) of the range; vertical: the same from [pa, pb)
+  int sh_v, sh_s, base;
+};
+
+__device__ __forceinline__ int clamp64(int x) { return x < 0 ? 0 : (x > 64 ? 64 : x); }
+
+__device__ __forceinline__ void bits_fetch(const uint32_t* row, int lo, uint32_t w[3], int& sh) {
+  const int base = lo < 0 ? 0 : lo;
+  const int wd = base >> 5;
+  sh = base & 31;
+  if (lo <= -64) {
+    w[0] = w[1] = w[2] = 0u;
+    return;
+  }
+  w[0] = row[wd];
+  w[1] = row[wd + 1];
+  w[2] = row[wd + 2];
+}
+
+__device__ __forceinline__ uint64_t bits_form(const uint32_t w[3], int sh, int lo) {
+  uint64_t v = (static_cast<uint64_t>(w[0]) | (static_cast<uint64_t>(w[1]) << 32)) >> sh;
+  if (sh) v |= static_cast<uint64_t>(w[2]) << (64 - sh);
+  if (lo < 0) v = lo <= -64 ? 0ull : (v << -lo);
+  return v;
+}
+
+__device__ __forceinline__ KeepFetch keep_fetch(int src, int start, int i, int half, int lo, int hi,
+                                                int pa, int pb, const uint32_t* vrow,
+                                                const uint32_t* srow) {
+  KeepFetch f;
+  f.src = src;
   if (src == 1) {
     const int j0 = start + 64 * half;  // first key of the half window
-    const int a = min(max(lo - j0, 0), 64);
-    const int b = min(max(hi - j0, a), 64);
-    const uint64_t rng = (b >= 64 ? ~0ull : ((1ull << b) - 1)) & ~(a >= 64 ? ~0ull : ((1ull << a) - 1));
-    const uint64_t vm = bits64(vrow, j0);
-    const int base = i - j0;  // offset of key e is base - e
-    uint64_t sm = __brevll(bits64(srow, base - 63));
-    if (base >= 0 && base < 64) sm |= 1ull << base;
-    return rng & sm & ~vm;
+    f.a = clamp64(lo - j0);
+    f.b = max(clamp64(hi - j0), f.a);
+    f.base = i - j0;  // offset of key e is base - e
+    bits_fetch(vrow, j0, f.v, f.sh_v);
+    bits_fetch(srow, f.base - 63, f.s, f.sh_s);
+  } else {
+    const int pos0 = start + 64 * half;  // first gathered position
+    f.a = clamp64(pa - pos0);
+    f.b = max(clamp64(pb - pos0), f.a);
   }
-  const int pos0 = start + 64 * half;  // first gathered position
-  const int32_t* v = vk + pos0;
-  uint64_t keep = 0;
-#pragma unroll
-  for (int e4 = 0; e4 < 16; ++e4) {
-    int4 jj = make_int4(0x7fffffff, 0x7fffffff, 0x7fffffff, 0x7fffffff);
-    if (pos0 + 4 * e4 + 3 < nv_eff) {
-      jj = *reinterpret_cast<const int4*>(v + 4 * e4);
-    } else {
-      if (pos0 + 4 * e4 + 0 < nv_eff) jj.x = v[4 * e4 + 0];
-      if (pos0 + 4 * e4 + 1 < nv_eff) jj.y = v[4 * e4 + 1];
-      if (pos0 + 4 * e4 + 2 < nv_eff) jj.z = v[4 * e4 + 2];
-    }
-    const int js[4] = {jj.x, jj.y, jj.z, jj.w};
-#pragma unroll
-    for (int u = 0; u < 4; ++u)
-      if (js[u] >= lo && js[u] < hi) keep |= 1ull << (4 * e4 + u);
-  }
-  return keep;
+  return f;
+}
+
+__device__ __forceinline__ uint64_t keep_finish(const KeepFetch& f, int start, int half) {
+  const uint64_t rng =
+      (f.b >= 64 ? ~0ull : ((1ull << f.b) - 1)) & ~(f.a >= 64 ? ~0ull : ((1ull << f.a) - 1));
+  if (f.src != 1) return rng;
+  const int j0 = start + 64 * half;
+  const uint64_t vm = bits_form(f.v, f.sh_v, j0);
+  uint64_t sm = __brevll(bits_form(f.s, f.sh_s, f.base - 63));
+  if (f.base >= 0 && f.base < 64) sm |= 1ull << f.base;
+  return rng & sm & ~vm;
 }
 
 // The work list of the CTA, built by one warp: the slash runs staged in
@@ -160,7 +175,7 @@ __device__ __forceinline__ uint64_t item_keep(int src, int start, int i, int hal
 // SPARSE_NKEYS keys in the sorted vertical list found together (each round
 // samples 32 evenly spaced positions of every key's remaining interval and
 // keeps the one sub-interval that can hold the bound; 1024 keys take two
-// rounds), then lane 0 merges the ranges and counts the items.
+// rounds), lane 0 merges the ranges, and the lanes count the items.
 __device__ void plan_build_warp(SparsePlan& P, const int32_t* vk, int nvh, const int2* runs,
                                 int nr, int64_t i0, int64_t i_last, int64_t s, int64_t w,
                                 int reading, int lane) {
@@ -206,8 +221,14 @@ __device__ void plan_build_warp(SparsePlan& P, const int32_t* vk, int nvh, const
   if (lane == 0) {
     sparse_plan_vertical(P, klo, khi, lo, 128);
     sparse_plan_slash(P, [&](int k) { return P.iv[k]; }, nr, i0, i_last, 128);
-    sparse_plan_count(P);
   }
+  __syncwarp();
+  // the item count (sparse_plan_count) with the ranges spread over the lanes
+  int cnt = 0;
+  for (int r = lane; r < P.n_iv; r += 32) cnt += sparse_range_items(P.iv[r], P.kr);
+#pragma unroll
+  for (int off = 16; off >= 1; off >>= 1) cnt += __shfl_xor_sync(0xffffffffu, cnt, off);
+  if (lane == 0) P.n_items = cnt + sparse_vertical_items(P);
 }
 
 // One online-softmax step for half of a query row (see the dense kernel):
@@ -226,10 +247,15 @@ __device__ __forceinline__ bool sparse_half_step(
     for (int e = 0; e < 64; ++e)
       if (!((keep >> e) & 1ull)) sv[e] = 0xff800000u;  // -inf
   }
-  float mx = max64(sv);
+  // at most one attended key in each half-row of the warp (a window that a
+  // lone diagonal crosses): its score is the half-row maximum, and one
+  // exponential per thread replaces 64
+  const bool one_key = __all_sync(0xffffffffu, __popcll(keep) <= 1);
+  const int e1 = keep ? __ffsll(static_cast<long long>(keep)) - 1 : -1;
+  const float mx_half = max64(sv);
   float mx_other = -INFINITY;
-  if (!pair_exchange(pc, mx, mx_other, abort, status, p.timeout_ns, ST_SOFTMAX)) return false;
-  mx = fmaxf(mx, mx_other);
+  if (!pair_exchange(pc, mx_half, mx_other, abort, status, p.timeout_ns, ST_SOFTMAX)) return false;
+  const float mx = fmaxf(mx_half, mx_other);
 
   const float m_new = fmaxf(m_ref, mx);
   const bool need =
@@ -241,7 +267,17 @@ __device__ __forceinline__ bool sparse_half_step(
     l_sum *= alpha;
   }
   uint32_t pk[32];
-  l_sum += exp_pack64(sv, sc, (m_ref == -INFINITY) ? 0.f : m_ref * sc, pk);
+  const float mb = (m_ref == -INFINITY) ? 0.f : m_ref * sc;
+  if (one_key) {
+    const float pv = e1 >= 0 ? ex2_approx(fmaf(mx_half, sc, -mb)) : 0.f;
+    l_sum += pv;
+    const uint32_t b = static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(pv)));
+    const uint32_t word = (e1 & 1) ? (b << 16) : b;
+#pragma unroll
+    for (int w2 = 0; w2 < 32; ++w2) pk[w2] = (w2 == (e1 >> 1)) ? word : 0u;
+  } else {
+    l_sum += exp_pack64(sv, sc, mb, pk);
+  }
   tmem_st32(tS + 32u * half, pk);
   // O holds items < n; the P.V of item n - 1 must have landed before a rescale
   if (n > 0 && __any_sync(0xffffffffu, need)) {
@@ -292,11 +328,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       mbar_init(&ctl->slot_full[k], 1);
       mbar_init(&ctl->slot_empty[k], 1);
     }
-    for (int st = 0; st < 2; ++st) {
+    for (int st = 0; st < NSBUF; ++st) {
       mbar_init(&ctl->s_full[st], 1);
       mbar_init(&ctl->p_full[st], 8);
-      mbar_init(&ctl->pv_done[st], 1);
     }
+    for (int st = 0; st < 2; ++st) mbar_init(&ctl->pv_done[st], 1);
     mbar_init(&ctl->q_ready, 8);
     mbar_init(&ctl->o_final, 1);
     mbar_init(&ctl->drain, 1);
@@ -360,10 +396,41 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const uint32_t* srow = p.sbit + static_cast<int64_t>(h) * p.wpr;
     const int32_t* vk = p.vidx + static_cast<int64_t>(h) * p.nv_cap;
     const int ii = static_cast<int>(i);
-    auto keep_of = [&](int src_, int start_, int cls_) {
+    // the row's positions [vpa, vpb) in the sorted vertical list per class:
+    // six lower bounds searched together (branch-free halving)
+    int vpa[3], vpb[3];
+    {
+      const int nvh = plan.nv_eff;
+      int pos[6];
+#pragma unroll
+      for (int e = 0; e < 6; ++e) pos[e] = 0;
+      int len = nvh;
+      while (len > 1) {
+        const int hl = len >> 1;
+#pragma unroll
+        for (int e = 0; e < 6; ++e) {
+          const int key = (e & 1) ? khi[e >> 1] : klo[e >> 1];
+          if (vk[pos[e] + hl - 1] < key) pos[e] += hl;
+        }
+        len -= hl;
+      }
+#pragma unroll
+      for (int e = 0; e < 6; ++e) {
+        const int key = (e & 1) ? khi[e >> 1] : klo[e >> 1];
+        if (len == 1 && vk[pos[e]] < key) ++pos[e];
+      }
+#pragma unroll
+      for (int c = 0; c < 3; ++c) {
+        vpa[c] = pos[2 * c];
+        vpb[c] = pos[2 * c + 1];
+      }
+    }
+    auto fetch = [&](int src_, int start_, int cls_) {
       const int lo = cls_ == 0 ? klo[0] : (cls_ == 1 ? klo[1] : klo[2]);
       const int hi = cls_ == 0 ? khi[0] : (cls_ == 1 ? khi[1] : khi[2]);
-      return item_keep(src_, start_, ii, half, lo, hi, vrow, srow, vk, plan.nv_eff);
+      const int pa = cls_ == 0 ? vpa[0] : (cls_ == 1 ? vpa[1] : vpa[2]);
+      const int pb = cls_ == 0 ? vpb[0] : (cls_ == 1 ? vpb[1] : vpb[2]);
+      return keep_fetch(src_, start_, ii, half, lo, hi, pa, pb, vrow, srow);
     };
     auto write_q = [&](int cls_) {
       const float2* trow = real ? p.tab + query_table_row(i, cls_, p.s, p.w, p.tab_c1) * 64 : nullptr;
@@ -379,36 +446,42 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     uint64_t keep = 0;
     if (N > 0) {
       sparse_iter_next(it, plan, src, start, cls);
-      keep = keep_of(src, start, cls);
+      keep = keep_finish(fetch(src, start, cls), start, half);
       write_q(cls);  // the first class's query operand
     }
     __syncwarp();
     if (lane == 0) mbar_arrive(&ctl->q_ready);
 
+    int st = 0;             // S buffer of item n (n mod 3)
+    uint32_t ph = 0u;       // its phase bits, one per buffer
     for (int n = 0; n < N && ok; ++n) {
-      const int st = n & 1;
-      ok = wait_poll(&ctl->s_full[st], static_cast<uint32_t>((n >> 1) & 1), abort_flag, p.status,
-                     p.timeout_ns, ST_SOFTMAX);
+      ok = wait_poll(&ctl->s_full[st], (ph >> st) & 1u, abort_flag, p.status, p.timeout_ns,
+                     ST_SOFTMAX);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
       tc_fence_after();
-      // the next item and its mask: their loads overlap this item's softmax
+      // the next item: its mask's loads are in flight during this item's softmax
       int src1 = src, start1 = start, cls1 = cls;
-      uint64_t keep1 = 0;
+      KeepFetch kf;
+      kf.src = 0;
+      kf.a = kf.b = 0;
       if (n + 1 < N) {
         sparse_iter_next(it, plan, src1, start1, cls1);
-        keep1 = keep_of(src1, start1, cls1);
+        kf = fetch(src1, start1, cls1);
       }
       const uint32_t tS = tbase + lane_off + static_cast<uint32_t>(st * 128);
-      const uint32_t tO = tbase + lane_off + 256u;
+      const uint32_t tO = tbase + lane_off + COL_O;
       ok = sparse_half_step(tS, tO, n, keep, p, sc, m_ref, l_sum, pc, ctl, abort_flag, p.status);
       if (!ok) break;
+      const uint64_t keep1 = keep_finish(kf, start1, half);
       // a class change: S(n) has completed, S(n + 1) waits for P(n), so the
       // operand tile is free for the next class's rotation
       if (n + 1 < N && cls1 != cls) write_q(cls1);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&ctl->p_full[st]);
+      ph ^= 1u << st;
+      st = st == 2 ? 0 : st + 1;
       src = src1;
       start = start1;
       cls = cls1;
@@ -424,7 +497,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     if (ok && N > 0) {
       const float l_tot = l_sum + l_other;
       tc_fence_after();
-      const uint32_t tO = tbase + lane_off + 256u + 64u * half;
+      const uint32_t tO = tbase + lane_off + COL_O + 64u * half;
       const float inv = 1.f / l_tot;
       __nv_bfloat16* orow =
           real ? p.out + ((i - p.q_start) * p.Hq + h) * static_cast<int64_t>(HD) + 64 * half
@@ -495,65 +568,75 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         return wait_spin(&ctl->slot_full[li % NSLOT], static_cast<uint32_t>((li / NSLOT) & 1),
                          abort_flag, p.status, p.timeout_ns, ST_MMA);
       };
-      // S(k) into buffer k & 1; items come from the issue cursor
+      // S(k) into buffer k mod 3; the cursor stands after item `issued`,
+      // cls_next its class, cls_prev the class of the last S issued
       SparseIter it;
       sparse_iter_init(it);
-      int src, start, cls_next = -1, cls_prev = -1;
-      int issued = 0;  // S issued for items < issued
-      auto peek = [&]() {  // class of item `issued` (the cursor's next item)
-        if (issued >= N) return;
-        SparseIter t = it;
-        int s_, st_;
-        sparse_iter_next(t, plan, s_, st_, cls_next);
-      };
+      int src_, start_, cls_next = -1, cls_prev = -1;
+      int issued = 0, sb = 0;
+      if (N > 0) sparse_iter_next(it, plan, src_, start_, cls_next);
       auto issue_s = [&]() {
-        sparse_iter_next(it, plan, src, start, cls_prev);
         const int li = 2 * issued;
         const uint64_t dk = dk0 + static_cast<uint64_t>(((li % NSLOT) * TILE_BYTES) >> 4);
 #pragma unroll
         for (int kk = 0; kk < HD / 16; ++kk) {
           const uint64_t off = static_cast<uint64_t>(((kk >> 2) * HALF_BYTES + (kk & 3) * 32) >> 4);
-          mma_ss(tbase + static_cast<uint32_t>((issued & 1) * 128), dq + off, dk + off, id_s,
-                 kk > 0 ? 1u : 0u);
+          mma_ss(tbase + static_cast<uint32_t>(sb * 128), dq + off, dk + off, id_s, kk > 0 ? 1u : 0u);
         }
-        mma_commit(&ctl->s_full[issued & 1]);
+        mma_commit(&ctl->s_full[sb]);
         mma_commit(&ctl->slot_empty[li % NSLOT]);
         ++issued;
-        peek();
+        sb = sb == NSBUF - 1 ? 0 : sb + 1;
+        cls_prev = cls_next;
+        if (issued < N) sparse_iter_next(it, plan, src_, start_, cls_next);
       };
-      // S(k) may go once P.V(k - 2) is issued (its buffer), and, where the
+      // S(k) may go once P.V(k - 3) is issued (its buffer), and, where the
       // class changes, once P(k - 1) is released (the operand tile)
       auto can_issue = [&](int n_done) {  // P.V issued for items < n_done
-        return issued < N && issued <= n_done + 1 && (issued <= n_done || cls_next == cls_prev);
+        return issued < N && issued <= n_done + NSBUF - 1 &&
+               (issued <= n_done || cls_next == cls_prev);
+      };
+      auto tile_landed = [&](int li) {
+        return mbar_test_wait(&ctl->slot_full[li % NSLOT], static_cast<uint32_t>((li / NSLOT) & 1));
       };
       bool ok = wait_bounded(&ctl->q_ready, 0u, abort_flag, p.status, p.timeout_ns, ST_MMA);
-      peek();
-      while (ok && can_issue(0)) {
+      while (ok && issued <= 2 && can_issue(0)) {
         ok = full_wait(2 * issued);
         if (!ok) break;
         tc_fence_after();
         issue_s();
       }
+      int pb = 0;        // buffer of P(n)
+      uint32_t pph = 0;  // p_full phase bits, one per buffer
+      // The key tile of S(k) lands in the slot that P.V(k - 3) frees, so S runs
+      // at most two items ahead of the P.V being issued: S(n + 2) needs P.V(n - 1).
       for (int n = 0; n < N && ok; ++n) {
         const int lv = 2 * n + 1;
         ok = full_wait(lv);
-        // the next S's key tile too: a wait between the P.V and the S MMAs
-        // would leave the tensor pipe idle
-        if (ok && can_issue(n + 1)) ok = full_wait(2 * issued);
+        // S ahead of P.V(n) where its key tile has already landed
+        while (ok && issued <= n + 2 && can_issue(n) && tile_landed(2 * issued)) {
+          tc_fence_after();
+          issue_s();
+        }
+        // the key tile of the S that follows P.V(n): a wait between the P.V
+        // and the S MMAs would leave the tensor pipe idle
+        if (ok && issued <= n + 2 && can_issue(n + 1)) ok = full_wait(2 * issued);
         if (!ok) break;
-        ok = wait_spin(&ctl->p_full[n & 1], static_cast<uint32_t>((n >> 1) & 1), abort_flag,
-                       p.status, p.timeout_ns, ST_MMA);
+        ok = wait_spin(&ctl->p_full[pb], (pph >> pb) & 1u, abort_flag, p.status, p.timeout_ns,
+                       ST_MMA);
         if (!ok) break;
         tc_fence_after();
         const uint64_t dv = dv0 + static_cast<uint64_t>(((lv % NSLOT) * TILE_BYTES) >> 4);
 #pragma unroll
         for (int kk = 0; kk < BN / 16; ++kk) {
-          mma_ts(tbase + 256u, tbase + static_cast<uint32_t>((n & 1) * 128 + kk * 8),
+          mma_ts(tbase + COL_O, tbase + static_cast<uint32_t>(pb * 128 + kk * 8),
                  dv + static_cast<uint64_t>((kk * 2048) >> 4), id_o, (n > 0 || kk > 0) ? 1u : 0u);
         }
         mma_commit(&ctl->pv_done[n & 1]);
         mma_commit(&ctl->slot_empty[lv % NSLOT]);
-        while (ok && can_issue(n + 1)) {
+        pph ^= 1u << pb;
+        pb = pb == NSBUF - 1 ? 0 : pb + 1;
+        while (ok && issued <= n + 2 && can_issue(n + 1)) {
           ok = full_wait(2 * issued);
           if (!ok) break;
           tc_fence_after();
