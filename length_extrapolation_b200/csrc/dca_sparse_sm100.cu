@@ -24,17 +24,18 @@
 // into key ranges once per CTA in shared memory (dca_sparse_plan.cuh).
 //
 // Warps (320 threads): warps 0-7 softmax (warp w and w+4 split each row's 128
-// keys), warp 8 TMA producer (5-slot K/V ring, no multicast), warp 9 MMA
-// issuer.  With one head per CTA three TMEM S buffers rotate over
-// consecutive items, so S(n+1) and S(n+2) run on the tensor cores while the
-// softmax warps work on S(n); P(n) overwrites the first 64 columns of its S
-// buffer and feeds O += P V from TMEM.  One query operand tile: where the class changes
-// between items n and n+1, the softmax warps rewrite it for the new class
-// after S(n) has completed and before they release P(n), and S(n+1) is issued
-// after P(n) instead of one item earlier.  Warp 0 builds the work list at the
-// start (runs staged in shared memory, the vertical-list searches done by the
-// whole warp); each softmax thread keeps its row's key range per class, so
-// an item's keep mask is a range test plus the membership bitmaps.
+// keys), warp 8 TMA producer (6-slot K/V ring, no multicast), warp 9 MMA
+// issuer.  TMEM holds two S buffers, O and the rotated query tile: S = Q K^T
+// takes Q from TMEM and the key tile from shared memory, so S(n+1) runs on
+// the tensor cores while the softmax warps work on S(n); P(n) overwrites the
+// first 64 columns of its S buffer and feeds O += P V from TMEM.  Where the
+// class changes between items n and n+1 the softmax warps rewrite the query
+// tile for the new class after S(n) has completed and before they release
+// P(n), and S(n+1) is issued after P(n) instead of one item earlier.  Warp 0
+// builds the work list at the start (runs staged in shared memory, the
+// vertical-list searches done by the whole warp); each softmax thread keeps
+// its row's key range and vertical-list positions per class, so an item's
+// keep mask is a range test plus the slash and vertical bitmaps.
 // Every wait is bounded; on timeout the CTA raises its abort flag, ORs a code
 // into the device status word, drains its copies and MMAs and exits.
 #include <cuda_bf16.h>
@@ -52,9 +53,11 @@ namespace sp {
 using namespace attn;
 
 constexpr int BM = 128, BN = 128, HD = 128;
-constexpr int NSLOT = 5;
-constexpr int NSBUF = 3;                 // S buffers in TMEM (P aliases their first 64 columns)
+constexpr int NSLOT = 6;                 // K/V ring: the key tile of S(k) reuses the slot of K(k - 3)
+static_assert(NSLOT % 2 == 0, "a key tile's slot must have held a key tile");
+constexpr int NSBUF = 2;                 // S buffers in TMEM (P aliases their first 64 columns)
 constexpr uint32_t COL_O = NSBUF * 128;  // O after them
+constexpr uint32_t COL_Q = COL_O + 128;  // the rotated query tile (MMA operand A), 64 columns
 constexpr int TILE_BYTES = 32768;
 constexpr int NUM_THREADS = 320;
 constexpr int WARP_LOAD = 8, WARP_MMA = 9;
@@ -78,7 +81,7 @@ struct SmemCtl {
   SparsePlan plan;
 };
 
-constexpr size_t SMEM_BYTES = 1024 + TILE_BYTES + NSLOT * TILE_BYTES + sizeof(SmemCtl);
+constexpr size_t SMEM_BYTES = 1024 + NSLOT * TILE_BYTES + sizeof(SmemCtl);
 static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 
 struct Params {
@@ -307,8 +310,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-  uint8_t* q_buf = smem;
-  uint8_t* slots = smem + TILE_BYTES;
+  uint8_t* slots = smem;
   SmemCtl* ctl = reinterpret_cast<SmemCtl*>(slots + NSLOT * TILE_BYTES);
 
   const int warp = threadIdx.x >> 5;
@@ -382,7 +384,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const float sc = p.scale_log2;
     const __nv_bfloat16* qrow =
         real ? p.q + ((i - p.q_start) * p.Hq + h) * static_cast<int64_t>(HD) : nullptr;
-    const int c0 = 4 * half, c1 = 4 * half + 4;
     // the row's key range per class (a padding row past the block keeps none)
     int klo[3], khi[3];
 #pragma unroll
@@ -432,10 +433,36 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const int pb = cls_ == 0 ? vpb[0] : (cls_ == 1 ? vpb[1] : vpb[2]);
       return keep_fetch(src_, start_, ii, half, lo, hi, pa, pb, vrow, srow);
     };
+    // the row rotated for a class, into the query operand in TMEM (column c
+    // holds dims 2c, 2c + 1; this thread: dims 32 half .. +31 and 64 + the same)
     auto write_q = [&](int cls_) {
-      const float2* trow = real ? p.tab + query_table_row(i, cls_, p.s, p.w, p.tab_c1) * 64 : nullptr;
-      write_q_row(q_buf, r, qrow, trow, c0, c1);
-      fence_proxy_async_smem();
+      uint32_t wa[16], wb[16];
+#pragma unroll
+      for (int e = 0; e < 16; ++e) wa[e] = wb[e] = 0u;
+      if (real) {
+        const float2* trow = p.tab + query_table_row(i, cls_, p.s, p.w, p.tab_c1) * 64;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          const int d0 = 32 * half + 8 * c;
+          const uint4 xa = *reinterpret_cast<const uint4*>(qrow + d0);
+          const uint4 xb = *reinterpret_cast<const uint4*>(qrow + 64 + d0);
+          const float4* t4 = reinterpret_cast<const float4*>(trow + d0);
+          const __nv_bfloat162* a2 = reinterpret_cast<const __nv_bfloat162*>(&xa);
+          const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&xb);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float4 t = t4[e];
+            const float2 x = __bfloat1622float2(a2[e]);
+            const float2 y = __bfloat1622float2(b2[e]);
+            wa[4 * c + e] = pack_bf16(x.x * t.x - y.x * t.y, x.y * t.z - y.y * t.w);
+            wb[4 * c + e] = pack_bf16(x.x * t.y + y.x * t.x, x.y * t.w + y.y * t.z);
+          }
+        }
+      }
+      const uint32_t tq = tbase + lane_off + COL_Q + 16u * half;
+      tmem_st16(tq, wa);
+      tmem_st16(tq + 32u, wb);
+      tmem_st_wait();
     };
 
     SparseIter it;
@@ -449,10 +476,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       keep = keep_finish(fetch(src, start, cls), start, half);
       write_q(cls);  // the first class's query operand
     }
+    tc_fence_before();
     __syncwarp();
     if (lane == 0) mbar_arrive(&ctl->q_ready);
 
-    int st = 0;             // S buffer of item n (n mod 3)
+    int st = 0;             // S buffer of item n (n mod NSBUF)
     uint32_t ph = 0u;       // its phase bits, one per buffer
     for (int n = 0; n < N && ok; ++n) {
       ok = wait_poll(&ctl->s_full[st], (ph >> st) & 1u, abort_flag, p.status, p.timeout_ns,
@@ -481,7 +509,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&ctl->p_full[st]);
       ph ^= 1u << st;
-      st = st == 2 ? 0 : st + 1;
+      st = st == NSBUF - 1 ? 0 : st + 1;
       src = src1;
       start = start1;
       cls = cls1;
@@ -561,14 +589,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     if (lane == 0) {
       const uint32_t id_s = idesc_bf16_f32(BM, BN, false);
       const uint32_t id_o = idesc_bf16_f32(BM, HD, true);
-      const uint64_t dq = sdesc_sw128(smem_u32(q_buf), 16, 1024);
       const uint64_t dk0 = sdesc_sw128(smem_u32(slots), 16, 1024);
       const uint64_t dv0 = sdesc_sw128(smem_u32(slots), HALF_BYTES, 1024);
       auto full_wait = [&](int li) {
         return wait_spin(&ctl->slot_full[li % NSLOT], static_cast<uint32_t>((li / NSLOT) & 1),
                          abort_flag, p.status, p.timeout_ns, ST_MMA);
       };
-      // S(k) into buffer k mod 3; the cursor stands after item `issued`,
+      // S(k) = Q K^T into buffer k mod NSBUF (Q from TMEM, the key tile from
+      // shared memory); the cursor stands after item `issued`,
       // cls_next its class, cls_prev the class of the last S issued
       SparseIter it;
       sparse_iter_init(it);
@@ -581,7 +609,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 #pragma unroll
         for (int kk = 0; kk < HD / 16; ++kk) {
           const uint64_t off = static_cast<uint64_t>(((kk >> 2) * HALF_BYTES + (kk & 3) * 32) >> 4);
-          mma_ss(tbase + static_cast<uint32_t>(sb * 128), dq + off, dk + off, id_s, kk > 0 ? 1u : 0u);
+          mma_ts(tbase + static_cast<uint32_t>(sb * 128), tbase + COL_Q + static_cast<uint32_t>(kk * 8),
+                 dk + off, id_s, kk > 0 ? 1u : 0u);
         }
         mma_commit(&ctl->s_full[sb]);
         mma_commit(&ctl->slot_empty[li % NSLOT]);
@@ -590,8 +619,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         cls_prev = cls_next;
         if (issued < N) sparse_iter_next(it, plan, src_, start_, cls_next);
       };
-      // S(k) may go once P.V(k - 3) is issued (its buffer), and, where the
-      // class changes, once P(k - 1) is released (the operand tile)
+      // S(k) may go once P.V(k - NSBUF) is issued (its buffer), and, where
+      // the class changes, once P(k - 1) is released (the query operand)
       auto can_issue = [&](int n_done) {  // P.V issued for items < n_done
         return issued < N && issued <= n_done + NSBUF - 1 &&
                (issued <= n_done || cls_next == cls_prev);
@@ -600,7 +629,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         return mbar_test_wait(&ctl->slot_full[li % NSLOT], static_cast<uint32_t>((li / NSLOT) & 1));
       };
       bool ok = wait_bounded(&ctl->q_ready, 0u, abort_flag, p.status, p.timeout_ns, ST_MMA);
-      while (ok && issued <= 2 && can_issue(0)) {
+      while (ok && can_issue(0)) {
         ok = full_wait(2 * issued);
         if (!ok) break;
         tc_fence_after();
@@ -608,19 +637,19 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       }
       int pb = 0;        // buffer of P(n)
       uint32_t pph = 0;  // p_full phase bits, one per buffer
-      // The key tile of S(k) lands in the slot that P.V(k - 3) frees, so S runs
-      // at most two items ahead of the P.V being issued: S(n + 2) needs P.V(n - 1).
+      // The key tile of S(k) lands in the slot that S(k - 3) frees, so no key
+      // tile waits for a P.V.
       for (int n = 0; n < N && ok; ++n) {
         const int lv = 2 * n + 1;
         ok = full_wait(lv);
         // S ahead of P.V(n) where its key tile has already landed
-        while (ok && issued <= n + 2 && can_issue(n) && tile_landed(2 * issued)) {
+        while (ok && can_issue(n) && tile_landed(2 * issued)) {
           tc_fence_after();
           issue_s();
         }
         // the key tile of the S that follows P.V(n): a wait between the P.V
         // and the S MMAs would leave the tensor pipe idle
-        if (ok && issued <= n + 2 && can_issue(n + 1)) ok = full_wait(2 * issued);
+        if (ok && can_issue(n + 1)) ok = full_wait(2 * issued);
         if (!ok) break;
         ok = wait_spin(&ctl->p_full[pb], (pph >> pb) & 1u, abort_flag, p.status, p.timeout_ns,
                        ST_MMA);
@@ -636,7 +665,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         mma_commit(&ctl->slot_empty[lv % NSLOT]);
         pph ^= 1u << pb;
         pb = pb == NSBUF - 1 ? 0 : pb + 1;
-        while (ok && issued <= n + 2 && can_issue(n + 1)) {
+        while (ok && can_issue(n + 1)) {
           ok = full_wait(2 * issued);
           if (!ok) break;
           tc_fence_after();
