@@ -145,31 +145,39 @@ DCA_HD void sparse_plan_vertical(SparsePlan& P, const int64_t klo[3], const int6
 // input index, so the runs may be staged in P.iv itself (run_at(k) reading
 // P.iv[k]).
 template <class RunAt>
-DCA_HD void sparse_plan_slash(SparsePlan& P, RunAt run_at, int nr, int64_t i0, int64_t i_last,
+DCA_HD void sparse_plan_slash(SparsePlan& P, RunAt run_at, int nr, int64_t i0_, int64_t i_last_,
                               int bn) {
-  int n_iv = 0;
+  const int i0 = static_cast<int>(i0_), i_last = static_cast<int>(i_last_);
+  int n_iv = 0, cx = 0, cy = 0;
+  bool open = false;  // a range [cx, cy) is being merged
   for (int k = 0; k <= nr; ++k) {
-    int64_t oa, ob;
-    if (k == nr) {
-      oa = 0;
-      ob = 1;
-    } else {
+    int oa = 0, ob = 1;
+    if (k < nr) {
       const int2 r = run_at(k);
       oa = r.x;
       ob = r.y;
     }
     if (oa > i_last) continue;
-    int64_t ka = i0 - (ob - 1);
-    if (ka < 0) ka = 0;
-    const int ta = static_cast<int>(ka), tb = static_cast<int>(i_last - oa + 1);
-    if (n_iv > 0 && ta < P.iv[n_iv - 1].y + bn) {
-      if (tb > P.iv[n_iv - 1].y) P.iv[n_iv - 1].y = tb;
-      if (ta < P.iv[n_iv - 1].x) P.iv[n_iv - 1].x = ta;
+    const int ta = i0 - (ob - 1) > 0 ? i0 - (ob - 1) : 0;
+    const int tb = i_last - oa + 1;
+    if (open && ta < cy + bn) {
+      if (tb > cy) cy = tb;
+      if (ta < cx) cx = ta;
     } else {
-      P.iv[n_iv].x = ta;
-      P.iv[n_iv].y = tb;
-      ++n_iv;
+      if (open) {  // index <= k: run k is already read
+        P.iv[n_iv].x = cx;
+        P.iv[n_iv].y = cy;
+        ++n_iv;
+      }
+      cx = ta;
+      cy = tb;
+      open = true;
     }
+  }
+  if (open) {
+    P.iv[n_iv].x = cx;
+    P.iv[n_iv].y = cy;
+    ++n_iv;
   }
   P.n_iv = n_iv;
 }
