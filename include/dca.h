@@ -420,8 +420,8 @@ int dca_noalloc_device_status(void* cuda_stream);
  * wait (default 10 s).  dca_set_debug_flags(1) makes the next attention launch
  * withhold its first key-tile load, so that its waits run out and the kernel
  * returns through the timeout path (status word set, DCA_ERR_TIMEOUT from
- * dca_device_status); flags reset to 0 after that launch.  The decode kernel
- * honours the same flag.
+ * dca_device_status); flags reset to 0 after that launch.  The decode and
+ * sparse kernels honour the same flag.
  */
 void dca_set_wait_timeout_ns(int64_t ns);
 void dca_set_debug_flags(int flags);

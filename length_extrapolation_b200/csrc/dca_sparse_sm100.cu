@@ -103,6 +103,7 @@ struct Params {
   float scale_log2;
   unsigned int* status;
   unsigned long long timeout_ns;
+  int debug;
 };
 
 // Bitmap rows are padded with two zero words past their last bit; bits below
@@ -568,6 +569,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                               abort_flag, p.status, p.timeout_ns, ST_LOAD);
             if (!ok) break;
           }
+          if ((p.debug & 1) && li == 0) continue;  // test hook: withhold the first key tile
           uint8_t* dst = slots + slot * TILE_BYTES;
           const CUtensorMap* tm = src == 1 ? (which ? &tm_v : &tm_k) : (which ? &tm_gv : &tm_gk);
           const int head_coord = src == 1 ? g : h;
@@ -723,6 +725,7 @@ cudaError_t launch_sparse_sm100(const AttnArgs& a, const SparseArgs& sa, cudaStr
   p.scale_log2 = a.scale_log2;
   p.status = a.status;
   p.timeout_ns = a.timeout_ns;
+  p.debug = a.debug;
   const int64_t blocks = static_cast<int64_t>(p.n_qtiles) * p.Hq;
   if (blocks > 0x7fffffffLL) return cudaErrorInvalidValue;
   cudaError_t e = cudaFuncSetAttribute(dca_sparse_kernel,

@@ -208,6 +208,48 @@ def test_sparse_parity(w, sizes, reading):
     assert_close(out.double().cpu().numpy(), want, torch.bfloat16, w.name)
 
 
+def _sparse_staged(w, pat, q, k, v):
+    kw = dict(chunk_size=w.chunk_size, local_window=w.local_window,
+              pretrain_window=w.pretrain_window)
+    ws = dca.Workspace(w.L, w.Hq, w.Hkv, 128, w.chunk_size, w.local_window, w.pretrain_window,
+                       q.dtype, DEV)
+    sp = dca.SparseWorkspace(w.L, w.Hq, pat.max_vertical(), pat.max_slash(), DEV)
+    dca.prepare(k, kv_len=w.L, k_rows_valid=0, rope_base=w.rope_base, workspace=ws, **kw)
+    dca.sparse_prepare(pat, v, kv_len=w.L, workspace=ws, sparse=sp, **kw)
+
+    def attend(out):
+        dca.sparse_attend(q, v, out, q_start=0, kv_len=w.L, yarn_scale=w.yarn_scale,
+                          workspace=ws, sparse=sp, **kw)
+        return ws.status()
+    return attend
+
+
+@pytest.mark.gpu
+def test_sparse_bounded_wait_timeout_reports_and_recovers():
+    """Withhold the first key tile (flag 1): the waits of every role of that
+    CTA run out after the short limit, the CTA drains its copies and MMAs
+    and exits, the status word reports the timeout, and the next launch on
+    the same workspace is correct."""
+    from tests.gpu_helpers import assert_close
+    w = wl("sp_timeout", 1100, 4, 2, 256, 64, 512)
+    V, S = sparse_pattern(w.L, w.Hq, 60, 32, 12, seed=5)
+    pat = dca.SparsePattern(V, S)
+    q, k, v = generate(w, device=DEV, seed=2)
+    attend = _sparse_staged(w, pat, q, k, v)
+    out = torch.zeros_like(q)
+    dca.set_wait_timeout_ns(20_000_000)
+    try:
+        dca.set_debug_flags(1)
+        assert attend(out) == N.DCA_ERR_TIMEOUT
+    finally:
+        dca.set_debug_flags(0)
+        dca.set_wait_timeout_ns(0)
+    out2 = torch.empty_like(q)
+    assert attend(out2) == N.DCA_OK
+    want = oracle.sparse_attention(q.cpu(), k.cpu(), v.cpu(), vertical=V, slash=S, **w.params())
+    assert_close(out2.double().cpu().numpy(), want, torch.bfloat16, "after timeout")
+
+
 @pytest.mark.gpu
 def test_sparse_all_offsets_equals_dense():
     """Every offset selected: the sparse path computes dense DCA attention."""
