@@ -91,6 +91,14 @@ size_t select_scratch_bytes(int64_t Lk, int Hq, int64_t n_chunks);
 // statistics `part` [Hq][select_slices(Lk)][64]; pass 2 reads the merged
 // `stats` [Hq][64] and writes vert (stored) and slash (accumulated).
 int select_slices(int64_t Lk);
+// Pass 1 alone (the row statistics), with the estimate rows of two heads as
+// the MMA M: `part` [Hq][select_stat_slices(Lk)][64].
+cudaError_t launch_select_row_stats(const void* kr, const float* qv, const float2* crot,
+                                    float2* part, int64_t i_first, int64_t Lk, int64_t s, int64_t w,
+                                    int n_last, int Hq, int Hkv, int reading, int continuous,
+                                    unsigned int* status, unsigned long long timeout_ns,
+                                    cudaStream_t st);
+int select_stat_slices(int64_t Lk);
 cudaError_t launch_select_scores(const void* kr, const float* qv, const float2* crot, float2* part,
                                  const float2* stats, float* vert, float* slash, int64_t i_first,
                                  int64_t Lk, int64_t s, int64_t w, int n_last, int Hq, int Hkv,

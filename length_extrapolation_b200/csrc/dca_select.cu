@@ -432,10 +432,9 @@ cudaError_t launch_select(const SelectArgs& sa, cudaStream_t st) {
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
   const int64_t i_first = sa.q_start + sa.Lq - sa.n_last;
-  const int n_slices = select_slices(sa.Lk);
-  e = launch_select_scores(sa.kr, qv, crot, part, stats, vert, slash, i_first, sa.Lk, sa.s, sa.w,
-                           sa.n_last, sa.Hq, sa.Hkv, sa.reading, sa.continuous, 1, sa.status,
-                           sa.timeout_ns, st);
+  const int n_slices = select_stat_slices(sa.Lk);
+  e = launch_select_row_stats(sa.kr, qv, crot, part, i_first, sa.Lk, sa.s, sa.w, sa.n_last, sa.Hq,
+                              sa.Hkv, sa.reading, sa.continuous, sa.status, sa.timeout_ns, st);
   if (e != cudaSuccess) return e;
   sel_stats_kernel<<<static_cast<unsigned>((sa.Hq * ROWS * 32 + 255) / 256), 256, 0, st>>>(
       part, stats, n_slices, sa.Hq);

@@ -43,6 +43,7 @@
 #include "dca_internal.h"
 #include "dca_plan.cuh"
 #include "dca_select_rows.cuh"
+#include "dca_softmax.cuh"
 #include "sm100_ptx.cuh"
 
 namespace dca {
@@ -125,12 +126,14 @@ struct Cursor {
 // they do not all ask L2 for the same key tile at once.  Continuous
 // positions rotate only a single-chunk slice (the operand buffers need the
 // chunks in order).
-__device__ __forceinline__ int phys_item(const SmemCtl* ctl, int n) {
+template <class Ctl>
+__device__ __forceinline__ int phys_item(const Ctl* ctl, int n) {
   const int q = n + ctl->rot;
   return q >= ctl->n_items ? q - ctl->n_items : q;
 }
 
-__device__ __forceinline__ void dca_item(const SmemCtl* ctl, Cursor& it) {
+template <class Ctl>
+__device__ __forceinline__ void dca_item(const Ctl* ctl, Cursor& it) {
   const int c2 = ctl->hi[CLS_INTER] - ctl->lo[CLS_INTER];
   const int c1 = ctl->hi[CLS_SUCC] - ctl->lo[CLS_SUCC];
   const int q = phys_item(ctl, it.n);
@@ -146,7 +149,8 @@ __device__ __forceinline__ void dca_item(const SmemCtl* ctl, Cursor& it) {
   }
 }
 
-__device__ __forceinline__ Cursor first_item(const SmemCtl* ctl, const Params& p) {
+template <class Ctl, class Prm>
+__device__ __forceinline__ Cursor first_item(const Ctl* ctl, const Prm& p) {
   Cursor it;
   it.n = 0;
   if (p.continuous) {
@@ -160,7 +164,8 @@ __device__ __forceinline__ Cursor first_item(const SmemCtl* ctl, const Params& p
   return it;
 }
 
-__device__ __forceinline__ void next_item(const SmemCtl* ctl, const Params& p, Cursor& it) {
+template <class Ctl, class Prm>
+__device__ __forceinline__ void next_item(const Ctl* ctl, const Prm& p, Cursor& it) {
   ++it.n;
   if (p.continuous && ctl->c_first == ctl->c_last) {
     it.kt = ctl->kt0 + phys_item(ctl, it.n);  // one item per k-tile
@@ -582,9 +587,357 @@ __global__ void __launch_bounds__(THREADS, 1)
   }
 }
 
+
+// ---------------------------------------------------------------------------
+// Pass 1 with the estimate rows as the MMA M.  The row statistics need, per
+// row, only a running (max, sum) over the keys, which is one register pair
+// when the thread owns the row: S = Q K'^T with M = 128 rows -- the 64
+// estimate rows of two heads of a KV group -- and N = 128 keys, so each key
+// tile serves two heads and each softmax thread keeps its row's statistics
+// the way the attention kernels do.  The query operand (bf16 hi + lo of the
+// fp32 rows, in log2 units) sits in TMEM as the MMA A operand; shared memory
+// holds a 6-slot key-tile ring; three S buffers let the MMA run two items
+// ahead.  The operand is rewritten where the item's variant (DCA: the pair
+// class; continuous: the key chunk) changes, after the last S that read it
+// has completed.  Warps: 0-3 softmax (thread = row = TMEM lane), 4 TMA
+// producer (no multicast), 5 MMA issuer.  One CTA = (KV group, pair of its
+// heads, slice of 16384 keys); its (max, sum) per row goes to the slice's
+// entry of `part`, which sel_stats_kernel merges.
+constexpr int R_ROWS = 128;               // two heads x 64 estimate rows
+constexpr int R_SLICE = 16384;            // keys per CTA
+constexpr int R_NSLOT = 6;                // key-tile ring
+constexpr int R_NSB = 3;                  // S buffers in TMEM
+constexpr uint32_t R_COL_QHI = R_NSB * 128, R_COL_QLO = R_COL_QHI + 64;
+constexpr int R_THREADS = 192;
+constexpr int R_WARP_LOAD = 4, R_WARP_MMA = 5;
+constexpr float R_RESCALE_LOG2 = 8.0f;    // the running max moves only when it grows by more
+
+struct RowCtl {
+  uint64_t slot_full[R_NSLOT];
+  uint64_t slot_empty[R_NSLOT];
+  uint64_t s_full[R_NSB];
+  uint64_t s_free[R_NSB];
+  uint64_t q_ready;         // the operand of the next variant is written (one arrival per warp)
+  uint64_t drain;
+  uint32_t tmem_base;
+  int abort;
+  int n_items;
+  int rot;                  // 0: items in list order
+  int lo[3], hi[3];         // DCA: k-tile range per class, clipped to the slice
+  int kt0;                  // continuous: first k-tile of the slice
+  int64_t kend;             // continuous: end of the slice's causal keys
+  int64_t c_first, c_last;  // continuous: key chunks met
+};
+
+constexpr size_t R_SMEM_BYTES = 1024 + R_NSLOT * TILE_BYTES + sizeof(RowCtl);
+static_assert(R_SMEM_BYTES <= 232448, "shared memory budget");
+
+struct RowParams {
+  const float* qv;          // [Hq][nvar][ROWS][HD] rotated query rows, log2 units
+  const float2* crot;       // continuous: (cos, sin) of s*n*theta_k [n_chunks][64]
+  float2* part;             // out: [Hq][n_slices][ROWS] (max, sum)
+  int64_t i_first, Lk, s, w;
+  int n_last, Hq, Hkv, G, n_pairs, n_slices, reading, continuous;
+  unsigned int* status;
+  unsigned long long timeout_ns;
+};
+
+__device__ __forceinline__ int64_t item_variant(const RowParams& p, const Cursor& it) {
+  return p.continuous ? it.c : static_cast<int64_t>(it.v);
+}
+
+__global__ void __launch_bounds__(R_THREADS, 1)
+    sel_rows_kernel(const __grid_constant__ CUtensorMap tm_k, const RowParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint8_t* slots = smem;
+  RowCtl* ctl = reinterpret_cast<RowCtl*>(slots + R_NSLOT * TILE_BYTES);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // the head pairs of one KV group and slice are adjacent: they read the same keys
+  const int hp = static_cast<int>(blockIdx.x) % p.n_pairs;
+  const int rest = static_cast<int>(blockIdx.x) / p.n_pairs;
+  const int sl = rest % p.n_slices;
+  const int g = rest / p.n_slices;
+  const int64_t ka = static_cast<int64_t>(sl) * R_SLICE;
+  const int64_t i_last = p.i_first + p.n_last - 1;
+
+  if (warp == 0) {
+    // work list of the slice; continuous: per k-tile the chunks its causal
+    // keys meet, counted by the lanes and summed over the warp
+    int n = 0;
+    if (p.continuous) {
+      int64_t kend = ka + R_SLICE;
+      if (kend > i_last + 1) kend = i_last + 1;
+      if (kend > p.Lk) kend = p.Lk;
+      const uint32_t s32 = static_cast<uint32_t>(p.s);
+      for (int t = lane; t < R_SLICE / BN; t += 32) {
+        const int64_t t0 = ka + static_cast<int64_t>(t) * BN;
+        if (t0 < kend) {
+          const int64_t t1 = (t0 + BN < kend ? t0 + BN : kend) - 1;
+          n += static_cast<int>(static_cast<uint32_t>(t1) / s32 - static_cast<uint32_t>(t0) / s32 + 1);
+        }
+      }
+      n = __reduce_add_sync(0xffffffffu, n);
+      if (lane == 0) {
+        ctl->kend = kend;
+        ctl->kt0 = static_cast<int>(ka / BN);
+        ctl->c_first = kend > ka ? ka / p.s : 0;
+        ctl->c_last = kend > ka ? (kend - 1) / p.s : 0;
+      }
+    } else if (lane == 0) {
+      const TilePlan P = make_plan(p.i_first, i_last, p.s, p.w, BN, p.reading);
+      const int t0 = static_cast<int>(ka / BN), t1 = static_cast<int>((ka + R_SLICE) / BN);
+      for (int c = 0; c < 3; ++c) {
+        const int a = P.lo[c] > t0 ? P.lo[c] : t0;
+        int b = P.hi[c] < t1 ? P.hi[c] : t1;
+        if (b < a) b = a;
+        ctl->lo[c] = a;
+        ctl->hi[c] = b;
+        n += b - a;
+      }
+    }
+    if (lane == 0) {
+      for (int k = 0; k < R_NSLOT; ++k) {
+        mbar_init(&ctl->slot_full[k], 1);
+        mbar_init(&ctl->slot_empty[k], 1);
+      }
+      for (int k = 0; k < R_NSB; ++k) {
+        mbar_init(&ctl->s_full[k], 1);
+        mbar_init(&ctl->s_free[k], 4);
+      }
+      mbar_init(&ctl->q_ready, 4);
+      mbar_init(&ctl->drain, 1);
+      ctl->abort = 0;
+      ctl->n_items = n;
+      ctl->rot = 0;
+      fence_barrier_init();
+    }
+  }
+  if (warp == R_WARP_MMA) {
+    tmem_alloc(&ctl->tmem_base, 512);
+    tmem_relinquish();
+  }
+  if (warp == R_WARP_LOAD && lane == 0) tma_prefetch_desc(&tm_k);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tbase = ctl->tmem_base;
+  volatile int* abort_flag = &ctl->abort;
+  const int N = ctl->n_items;
+
+  if (warp < 4) {
+    // =========================================================== softmax warps
+    const int r = warp * 32 + lane;  // TMEM lane = row of the MMA
+    const int hh = r >> 6, rr = r & 63;
+    const bool head_ok = 2 * hp + hh < p.G;
+    const int h = g * p.G + (head_ok ? 2 * hp + hh : 0);
+    const bool row_ok = head_ok && rr < p.n_last;
+    const int64_t i = p.i_first + rr;
+    const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+    const int nvar = p.continuous ? 1 : 3;
+    // the row's operand for the item's variant: hi and lo bf16 parts, column
+    // c holding dims 2c, 2c + 1; continuous: rotated back by the chunk angle
+    auto write_q = [&](const Cursor& c) {
+      uint32_t qh[64], ql[64];
+#pragma unroll
+      for (int e = 0; e < 64; ++e) qh[e] = ql[e] = 0u;
+      if (row_ok) {
+        const int v = p.continuous ? 0 : c.v;
+        const float* src = p.qv + ((static_cast<int64_t>(h) * nvar + v) * ROWS + rr) * HD;
+        const float2* cs = p.continuous ? p.crot + c.c * (HD / 2) : nullptr;
+#pragma unroll
+        for (int k = 0; k < HD / 2; k += 2) {
+          float a0 = src[k], a1 = src[k + 1], b0 = src[HD / 2 + k], b1 = src[HD / 2 + k + 1];
+          if (cs != nullptr) {  // R(-phi): (a cos + b sin, b cos - a sin)
+            const float2 t0 = cs[k], t1 = cs[k + 1];
+            const float ra0 = a0 * t0.x + b0 * t0.y, rb0 = b0 * t0.x - a0 * t0.y;
+            const float ra1 = a1 * t1.x + b1 * t1.y, rb1 = b1 * t1.x - a1 * t1.y;
+            a0 = ra0; b0 = rb0; a1 = ra1; b1 = rb1;
+          }
+          split_pack(a0, a1, qh[k / 2], ql[k / 2]);
+          split_pack(b0, b1, qh[32 + k / 2], ql[32 + k / 2]);
+        }
+      }
+      tmem_st64(tbase + lane_off + R_COL_QHI, qh);
+      tmem_st64(tbase + lane_off + R_COL_QLO, ql);
+      tmem_st_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&ctl->q_ready);
+    };
+
+    float m_ref = NEG_BIG, l_sum = 0.f;
+    Cursor it = first_item(ctl, p);
+    if (N > 0) write_q(it);
+    for (int n = 0; n < N; ++n) {
+      const int buf = n % R_NSB;
+      if (!wait_warp(&ctl->s_full[buf], static_cast<uint32_t>((n / R_NSB) & 1), abort_flag,
+                     p.status, p.timeout_ns, ST_SOFTMAX, lane))
+        break;
+      tc_fence_after();
+      // S(n) has completed, and with it every S that read this operand: where
+      // the next item has another variant, rewrite the operand now
+      Cursor nx = it;
+      if (n + 1 < N) {
+        next_item(ctl, p, nx);
+        if (item_variant(p, nx) != item_variant(p, it)) write_q(nx);
+      }
+      uint32_t sv[128];
+      tmem_ld128(tbase + lane_off + static_cast<uint32_t>(buf * 128), sv);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&ctl->s_free[buf]);
+      // the row's keys of this item: its class (or chunk), causal, j < Lk
+      int64_t lo = 0, hi = 0;
+      if (row_ok) {
+        if (p.continuous) {
+          lo = it.c * p.s;
+          hi = lo + p.s < i + 1 ? lo + p.s : i + 1;
+        } else {
+          row_key_range<int64_t>(i, it.v, p.s, p.w, p.reading, lo, hi);
+        }
+        if (hi > p.Lk) hi = p.Lk;
+      }
+      const int64_t j0 = static_cast<int64_t>(it.kt) * BN;
+      const int ea = lo - j0 < 0 ? 0 : (lo - j0 > BN ? BN : static_cast<int>(lo - j0));
+      const int eb = hi - j0 < ea ? ea : (hi - j0 > BN ? BN : static_cast<int>(hi - j0));
+      if (ea > 0 || eb < BN) {
+#pragma unroll
+        for (int e = 0; e < BN; ++e)
+          if (e < ea || e >= eb) sv[e] = 0xff800000u;  // -inf
+      }
+      float m8[8];
+#pragma unroll
+      for (int c = 0; c < 8; ++c) m8[c] = __uint_as_float(sv[c]);
+#pragma unroll
+      for (int e = 8; e < BN; e += 8)
+#pragma unroll
+        for (int c = 0; c < 8; ++c) m8[c] = fmaxf(m8[c], __uint_as_float(sv[e + c]));
+      const float mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
+                             fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
+      if (mx > m_ref + R_RESCALE_LOG2) {  // m_ref = NEG_BIG: l_sum is 0 and stays 0
+        l_sum *= ex2_approx(m_ref - mx);
+        m_ref = mx;
+      }
+      it = nx;
+      if (mx == -INFINITY) continue;  // no key of the row in this item
+      // 2^(x - m_ref) <= 2^8; one pair in eight on the FMA pipe
+      const float2 nm = make_float2(-m_ref, -m_ref);
+      float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                       make_float2(0.f, 0.f)};
+#pragma unroll
+      for (int e = 0; e < BN / 2; ++e) {
+        float2 x = add2(make_float2(__uint_as_float(sv[2 * e]), __uint_as_float(sv[2 * e + 1])), nm);
+        if ((e & 7) == 0) {
+          x.x = attn::exp2_poly1(x.x);
+          x.y = attn::exp2_poly1(x.y);
+        } else {
+          x.x = ex2_approx(x.x);
+          x.y = ex2_approx(x.y);
+        }
+        acc[e & 3] = add2(acc[e & 3], x);
+      }
+      const float2 a = add2(add2(acc[0], acc[1]), add2(acc[2], acc[3]));
+      l_sum += a.x + a.y;
+    }
+    if (head_ok)
+      p.part[(static_cast<int64_t>(h) * p.n_slices + sl) * ROWS + rr] = make_float2(m_ref, l_sum);
+  } else if (warp == R_WARP_LOAD) {
+    // =========================================================== TMA producer
+    if (lane == 0) {
+      int last[R_NSLOT];
+#pragma unroll
+      for (int k = 0; k < R_NSLOT; ++k) last[k] = -1;
+      Cursor it = first_item(ctl, p);
+      for (int n = 0; n < N; ++n) {
+        const int slot = n % R_NSLOT, use = n / R_NSLOT;
+        if (use > 0 &&
+            !wait_bounded(&ctl->slot_empty[slot], static_cast<uint32_t>((use - 1) & 1),
+                          abort_flag, p.status, p.timeout_ns, ST_LOAD))
+          break;
+        uint8_t* dst = slots + slot * TILE_BYTES;
+        mbar_arrive_expect_tx(&ctl->slot_full[slot], TILE_BYTES);
+        tma_load_3d(dst, &tm_k, &ctl->slot_full[slot], 0, g, it.kt * BN);
+        tma_load_3d(dst + HALF_BYTES, &tm_k, &ctl->slot_full[slot], 64, g, it.kt * BN);
+        last[slot] = n;
+        next_item(ctl, p, it);
+      }
+      for (int k = 0; k < R_NSLOT; ++k)
+        if (last[k] >= 0)
+          wait_drain(&ctl->slot_full[k], static_cast<uint32_t>((last[k] / R_NSLOT) & 1), p.status,
+                     p.timeout_ns, ST_DRAIN);
+    }
+    __syncwarp();
+  } else if (warp == R_WARP_MMA) {
+    // =========================================================== MMA issuer
+    if (lane == 0) {
+      const uint32_t id = idesc_bf16_f32(R_ROWS, BN, false);
+      const uint64_t dk0 = sdesc_sw128(smem_u32(slots), 16, 1024);
+      bool ok = true;
+      Cursor it = first_item(ctl, p);
+      int64_t have = -1;  // the variant whose operand is known to be written
+      uint32_t qph = 0;   // operand writes waited for
+      for (int n = 0; n < N && ok; ++n) {
+        const int64_t var = item_variant(p, it);
+        if (n == 0 || var != have) {
+          ok = wait_spin(&ctl->q_ready, qph & 1u, abort_flag, p.status, p.timeout_ns, ST_MMA);
+          if (!ok) break;
+          ++qph;
+          have = var;
+        }
+        if (n >= R_NSB) {
+          ok = wait_spin(&ctl->s_free[n % R_NSB], static_cast<uint32_t>(((n - R_NSB) / R_NSB) & 1),
+                         abort_flag, p.status, p.timeout_ns, ST_MMA);
+          if (!ok) break;
+        }
+        const int slot = n % R_NSLOT;
+        ok = wait_spin(&ctl->slot_full[slot], static_cast<uint32_t>((n / R_NSLOT) & 1), abort_flag,
+                       p.status, p.timeout_ns, ST_MMA);
+        if (!ok) break;
+        tc_fence_after();
+        const uint64_t dk = dk0 + static_cast<uint64_t>((slot * TILE_BYTES) >> 4);
+        const uint32_t d_tmem = tbase + static_cast<uint32_t>((n % R_NSB) * 128);
+#pragma unroll
+        for (int part = 0; part < 2; ++part) {  // hi, then lo
+          const uint32_t tq = tbase + (part ? R_COL_QLO : R_COL_QHI);
+#pragma unroll
+          for (int kk = 0; kk < HD / 16; ++kk) {
+            const uint64_t off = static_cast<uint64_t>(((kk >> 2) * HALF_BYTES + (kk & 3) * 32) >> 4);
+            mma_ts(d_tmem, tq + static_cast<uint32_t>(kk * 8), dk + off, id,
+                   (part > 0 || kk > 0) ? 1u : 0u);
+          }
+        }
+        mma_commit(&ctl->s_full[n % R_NSB]);
+        mma_commit(&ctl->slot_empty[slot]);
+        next_item(ctl, p, it);
+      }
+      mma_commit(&ctl->drain);
+      wait_drain(&ctl->drain, 0u, p.status, p.timeout_ns, ST_DRAIN);
+    }
+    __syncwarp();
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == R_WARP_MMA) {
+    tc_fence_after();
+    tmem_dealloc(tbase, 512);
+  }
+}
+
 }  // namespace selm
 
 int select_slices(int64_t Lk) { return static_cast<int>((Lk + selm::SLICE - 1) / selm::SLICE); }
+
+#ifndef DCA_SEL_ROWS
+#define DCA_SEL_ROWS 1
+#endif
+int select_stat_slices(int64_t Lk) {
+  return DCA_SEL_ROWS ? static_cast<int>((Lk + selm::R_SLICE - 1) / selm::R_SLICE)
+                      : select_slices(Lk);
+}
 
 cudaError_t launch_select_scores(const void* kr, const float* qv, const float2* crot, float2* part,
                                  const float2* stats, float* vert, float* slash, int64_t i_first,
@@ -621,6 +974,44 @@ cudaError_t launch_select_scores(const void* kr, const float* qv, const float2* 
                                        static_cast<int>(SMEM_BYTES));
   if (e != cudaSuccess) return e;
   kern<<<static_cast<unsigned>(blocks), THREADS, SMEM_BYTES, st>>>(tm_k, p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_select_row_stats(const void* kr, const float* qv, const float2* crot,
+                                    float2* part, int64_t i_first, int64_t Lk, int64_t s, int64_t w,
+                                    int n_last, int Hq, int Hkv, int reading, int continuous,
+                                    unsigned int* status, unsigned long long timeout_ns,
+                                    cudaStream_t st) {
+  if (!DCA_SEL_ROWS)
+    return launch_select_scores(kr, qv, crot, part, nullptr, nullptr, nullptr, i_first, Lk, s, w,
+                                n_last, Hq, Hkv, reading, continuous, 1, status, timeout_ns, st);
+  using namespace selm;
+  CUtensorMap tm_k;
+  if (!encode_kv_map(&tm_k, kr, Lk, Hkv)) return cudaErrorInvalidValue;
+  RowParams p;
+  p.qv = qv;
+  p.crot = crot;
+  p.part = part;
+  p.i_first = i_first;
+  p.Lk = Lk;
+  p.s = s;
+  p.w = w;
+  p.n_last = n_last;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.G = Hq / Hkv;
+  p.n_pairs = (p.G + 1) / 2;
+  p.n_slices = select_stat_slices(Lk);
+  p.reading = reading;
+  p.continuous = continuous;
+  p.status = status;
+  p.timeout_ns = timeout_ns;
+  const int64_t blocks = static_cast<int64_t>(Hkv) * p.n_slices * p.n_pairs;
+  if (blocks > 0x7fffffffLL) return cudaErrorInvalidValue;
+  cudaError_t e = cudaFuncSetAttribute(sel_rows_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(R_SMEM_BYTES));
+  if (e != cudaSuccess) return e;
+  sel_rows_kernel<<<static_cast<unsigned>(blocks), R_THREADS, R_SMEM_BYTES, st>>>(tm_k, p);
   return cudaGetLastError();
 }
 
