@@ -87,23 +87,22 @@ struct SelectArgs {
   unsigned long long timeout_ns;
 };
 size_t select_scratch_bytes(int64_t Lk, int Hq, int64_t n_chunks);
-// Score passes of the selection (tcgen05): pass 1 writes per-slice row
-// statistics `part` [Hq][select_slices(Lk)][64]; pass 2 reads the merged
-// `stats` [Hq][64] and writes vert (stored) and slash (accumulated).
-int select_slices(int64_t Lk);
-// Pass 1 alone (the row statistics), with the estimate rows of two heads as
-// the MMA M: `part` [Hq][select_stat_slices(Lk)][64].
+// Score passes of the selection (tcgen05).  Pass 1 writes per-slice row
+// statistics `part` [Hq][select_stat_slices(Lk)][64] (max, sum); pass 2 reads
+// the merged `stats` [Hq][64] and writes vert (stored, [Hq][Lk]) and slash
+// (accumulated, [Hq][Lk]), in slices of select_slices(Lk).
 cudaError_t launch_select_row_stats(const void* kr, const float* qv, const float2* crot,
                                     float2* part, int64_t i_first, int64_t Lk, int64_t s, int64_t w,
                                     int n_last, int Hq, int Hkv, int reading, int continuous,
                                     unsigned int* status, unsigned long long timeout_ns,
                                     cudaStream_t st);
 int select_stat_slices(int64_t Lk);
-cudaError_t launch_select_scores(const void* kr, const float* qv, const float2* crot, float2* part,
-                                 const float2* stats, float* vert, float* slash, int64_t i_first,
-                                 int64_t Lk, int64_t s, int64_t w, int n_last, int Hq, int Hkv,
-                                 int reading, int continuous, int pass, unsigned int* status,
-                                 unsigned long long timeout_ns, cudaStream_t st);
+cudaError_t launch_select_sums(const void* kr, const float* qv, const float2* crot,
+                               const float2* stats, float* vert, float* slash, int64_t i_first,
+                               int64_t Lk, int64_t s, int64_t w, int n_last, int Hq, int Hkv,
+                               int reading, int continuous, unsigned int* status,
+                               unsigned long long timeout_ns, cudaStream_t st);
+int select_slices(int64_t Lk);
 cudaError_t launch_select(const SelectArgs& sa, cudaStream_t st);
 
 // Host-side argument checks of dca_prefill (no device work): the dca_status

@@ -439,9 +439,9 @@ cudaError_t launch_select(const SelectArgs& sa, cudaStream_t st) {
   sel_stats_kernel<<<static_cast<unsigned>((sa.Hq * ROWS * 32 + 255) / 256), 256, 0, st>>>(
       part, stats, n_slices, sa.Hq);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  e = launch_select_scores(sa.kr, qv, crot, part, stats, vert, slash, i_first, sa.Lk, sa.s, sa.w,
-                           sa.n_last, sa.Hq, sa.Hkv, sa.reading, sa.continuous, 2, sa.status,
-                           sa.timeout_ns, st);
+  e = launch_select_sums(sa.kr, qv, crot, stats, vert, slash, i_first, sa.Lk, sa.s, sa.w,
+                         sa.n_last, sa.Hq, sa.Hkv, sa.reading, sa.continuous, sa.status,
+                         sa.timeout_ns, st);
   if (e != cudaSuccess) return e;
   SelectOut o;
   o.nv = sa.nv;

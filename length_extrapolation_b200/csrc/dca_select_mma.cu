@@ -2,39 +2,34 @@
 // cores (dca_select.cu holds the rest of the selection and states what it
 // computes: vertical and slash sums of the last rows' softmax).
 //
-// One CTA = one query head x one slice of 4096 keys.  The 64 estimate rows
-// are the MMA N: S^T = K' Q_v^T (M = 128 keys, N = 64 rows, K = 128 dims,
-// tcgen05.mma kind::f16, fp32 accumulators in TMEM), so TMEM lane t holds
-// key t's logits for all rows and each softmax thread owns one key.
-//
 // The query operand is the fp32 rotated query row (log2 units) split into
-// bf16 hi + lo parts, two MMAs accumulating into one S^T, so the logits keep
+// bf16 hi + lo parts, two MMAs accumulating into one S, so the logits keep
 // the precision of an fp32 dot product with the bf16 cached keys.  DCA: one
 // operand per pair class (INTER, SUCC, INTRA ranges, as in dca_plan.cuh).
 // Continuous positions: <R(i) q, R(j) k> = <R(-s n_j) R(i) q, R(j mod s) k>,
 // so the cached keys are used as they are and the operand is the query
-// rotated back by its key chunk's angle; a work item is (key tile, chunk)
-// and two operand buffers alternate as the chunk advances.
+// rotated back by its key chunk's angle; a work item is (key tile, chunk).
 //
-// Two passes over the same items:
-//   1  per thread and row an online (max, sum of 2^(x - max)) over its keys,
-//      merged over the row's 128 key threads and written per (head, slice,
-//      row);
-//      sel_stats_kernel merges the slices;
-//   2  p = 2^(x - M) / L: the per-key sum over the rows (vertical) into a
-//      shared-memory bin per key of the slice; the sums along the diagonals
-//      i - j (slash) in registers, one lane per diagonal class mod 32 fed by a
-//      rotating shuffle, then once per item into a bin per offset; the bins
-//      are stored / added to the score arrays once per CTA.
-// The rows of an item's class (and of causality) are one contiguous range
-// per key (class_row_range), so masking is a range test.
-// Warps: 0-7 softmax (two per SMSP: warp w reads the TMEM lane quarter
-// w % 4, i.e. 32 keys, and rows 32 (w / 4) .. + 31), 8 TMA producer (ring of
-// 3 -- continuous positions: 4 -- 32 KiB key tiles, no multicast), 9 MMA
-// issuer.  Every mbarrier wait is bounded; on timeout the CTA raises its abort
-// flag, ORs a code into the status word, drains its copies and MMAs, frees
-// TMEM and exits.  The softmax warps' own barriers (bar.sync 1, 256) are
-// reached by all eight warps on every path.
+// Pass 1 (sel_rows_kernel, the row statistics) is described at its kernel.
+// Pass 2 (sel_sums_kernel): one CTA = one query head x one slice of 4096
+// keys.  The 64 estimate rows are the MMA N: S^T = K' Q_v^T (M = 128 keys,
+// N = 64 rows, K = 128 dims, fp32 accumulators in TMEM), so TMEM lane t holds
+// key t's logits for all rows and each softmax thread owns one key.
+// p = 2^(x - M) / L: the per-key sum over the rows (vertical) goes into a
+// shared-memory bin per key of the slice; the sums along the diagonals i - j
+// (slash) into registers, one lane per diagonal class mod 32 fed by a
+// rotating shuffle, then once per item into a bin per offset; the bins are
+// stored / added to the score arrays once per CTA.  The rows of an item's
+// class (and of causality) are one contiguous range per key
+// (class_row_range), so masking is a range test.  Warps: 0-7 softmax (two per
+// SMSP: warp w reads the TMEM lane quarter w % 4, i.e. 32 keys, and rows
+// 32 (w / 4) .. + 31), 8 TMA producer (ring of 3 -- continuous positions: 4
+// -- 32 KiB key tiles, no multicast), 9 MMA issuer; DCA keeps the three
+// class operands, continuous positions two chunk operands that alternate as
+// the chunk advances.  Every mbarrier wait is bounded; on timeout the CTA
+// raises its abort flag, ORs a code into the status word, drains its copies
+// and MMAs, frees TMEM and exits.  The softmax warps' own barriers
+// (bar.sync 1, 256) are reached by all eight warps on every path.
 #include <cuda_bf16.h>
 #include <math.h>
 
@@ -64,13 +59,10 @@ constexpr int WARP_LOAD = SM_WARPS, WARP_MMA = SM_WARPS + 1;
 constexpr int NSBUF = 4;                  // S^T buffers in TMEM (the MMA runs up to 3 items ahead)
 constexpr uint32_t TMEM_COLS = NSBUF * ROWS;
 constexpr int SBINS = SLICE + ROWS;       // offsets i - j met by a slice
-constexpr int MSTRIDE = 144;              // row stride of the merge buffers (conflict-free)
-constexpr int MROWS = 16;                 // rows per merge round
-// pass 2: vertical bins [SLICE] (key j: one atomic add per row half) and the
-// slash bins [SBINS] (each lane adds its two diagonal sums once per item,
-// atomically: the warps' diagonal ranges overlap)
-constexpr int BIN_FLOATS =
-    (SLICE + SBINS) > 2 * MROWS * MSTRIDE ? (SLICE + SBINS) : 2 * MROWS * MSTRIDE;
+// vertical bins [SLICE] (key j: one atomic add per row half) and slash bins
+// [SBINS] (each lane adds its two diagonal sums once per item, atomically:
+// the warps' diagonal ranges overlap)
+constexpr int BIN_FLOATS = SLICE + SBINS;
 constexpr float NEG_BIG = -1e30f;         // finite "no value yet" maximum
 
 constexpr unsigned ST_SOFTMAX = 0x10u, ST_LOAD = 0x100u, ST_MMA = 0x1000u, ST_DRAIN = 0x10000u;
@@ -100,10 +92,9 @@ static_assert(SLICE % BN == 0 && SLICE / BN <= 32, "one counting lane per k-tile
 struct Params {
   const float* qv;          // [Hq][nvar][ROWS][HD] rotated query rows, log2 units
   const float2* crot;       // continuous: (cos, sin) of s*n*theta_k [n_chunks][64]
-  float2* part;             // pass 1 out: [Hq][n_slices][ROWS] (max, sum)
-  const float2* stats;      // pass 2 in: [Hq][ROWS] (max, sum)
-  float* vert;              // pass 2 out: [Hq][Lk]
-  float* slash;             // pass 2 out: [Hq][Lk] (accumulated)
+  const float2* stats;      // [Hq][ROWS] (max, sum) over all keys
+  float* vert;              // out: [Hq][Lk]
+  float* slash;             // out: [Hq][Lk] (accumulated)
   int64_t i_first, Lk, s, w;
   int n_last, Hq, Hkv, G, n_slices, reading, continuous;
   unsigned int* status;
@@ -267,23 +258,16 @@ __device__ __forceinline__ void build_operand(uint8_t* op_hi, const float* __res
   }
 }
 
-// (max, sum) merge of two partial row statistics (maxima finite).
-__device__ __forceinline__ float2 merge_stat(float2 a, float2 b) {
-  const float m = fmaxf(a.x, b.x);
-  return make_float2(m, a.y * exp2f(a.x - m) + b.y * exp2f(b.x - m));
-}
-
-template <int PASS>
 __global__ void __launch_bounds__(THREADS, 1)
-    sel_mma_kernel(const __grid_constant__ CUtensorMap tm_k, const Params p) {
+    sel_sums_kernel(const __grid_constant__ CUtensorMap tm_k, const Params p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   uint8_t* slots = smem;
   uint8_t* opnd = slots + NSLOT * TILE_BYTES;
   float* bins = reinterpret_cast<float*>(opnd + NOPND * QOP);
-  float* vbin = bins;            // [SLICE]     pass 2
-  float* sbin = bins + SLICE;    // [SBINS]     pass 2
+  float* vbin = bins;            // [SLICE]
+  float* sbin = bins + SLICE;    // [SBINS]
   SmemCtl* ctl = reinterpret_cast<SmemCtl*>(bins + BIN_FLOATS);
 
   // key-tile ring: 3 slots, and in continuous mode (4 operands, not 6) a
@@ -351,8 +335,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       fence_barrier_init();
     }
   }
-  if (PASS == 2)
-    for (int e = threadIdx.x; e < SLICE + SBINS; e += THREADS) bins[e] = 0.f;
+  for (int e = threadIdx.x; e < SLICE + SBINS; e += THREADS) bins[e] = 0.f;
   if (warp == WARP_MMA) {
     tmem_alloc(&ctl->tmem_base, TMEM_COLS);
     tmem_relinquish();
@@ -391,21 +374,12 @@ __global__ void __launch_bounds__(THREADS, 1)
       }
     }
 
-    // pass 1: running (max, sum) per row; pass 2: C_r = M_r + log2 L_r, so
-    // p = 2^(x - C_r)
-    constexpr int NR1 = PASS == 1 ? 32 : 1, NR2 = PASS == 2 ? 32 : 1;
-    float m[NR1], l[NR1], C[NR2];
+    // C_r = M_r + log2 L_r, so p = 2^(x - C_r)
+    float C[32];
 #pragma unroll
-    for (int e = 0; e < NR1; ++e) {
-      m[e] = NEG_BIG;
-      l[e] = 0.f;
-    }
-    if (PASS == 2) {
-#pragma unroll
-      for (int e = 0; e < NR2; ++e) {
-        const float2 st = p.stats[h * ROWS + r0 + e];
-        C[e] = st.y > 0.f ? st.x + __log2f(st.y) : 0.f;
-      }
+    for (int e = 0; e < 32; ++e) {
+      const float2 st = p.stats[h * ROWS + r0 + e];
+      C[e] = st.y > 0.f ? st.x + __log2f(st.y) : 0.f;
     }
     Cursor it = first_item(ctl, p);
     for (int n = 0; n < N; ++n) {
@@ -437,22 +411,12 @@ __global__ void __launch_bounds__(THREADS, 1)
 #pragma unroll
         for (int e = 0; e < 32; ++e) {
           const int r = r0 + e;
-          if (PASS == 1) {
-            float x = __uint_as_float(sv[e]);
-            if (MASKED) x = (r >= ra && r < rb) ? x : -INFINITY;
-            const float d = x - m[e];  // m is finite: a masked x gives -inf, t = 0
-            const float t = ex2_approx(-fabsf(d));
-            const bool up = d > 0.f;
-            l[e] = up ? fmaf(l[e], t, 1.f) : l[e] + t;
-            m[e] = up ? x : m[e];
-          } else {
-            float pr = ex2_approx(__uint_as_float(sv[e]) - C[e]);
-            if (MASKED) pr = (r >= ra && r < rb) ? pr : 0.f;
-            vsum += pr;
-            // source lane (e - L) mod 32: the shuffle takes the index mod 32
-            const float v = __shfl_sync(0xffffffffu, pr, e - lane);
-            if (lane <= e) a1 += v; else a0 += v;
-          }
+          float pr = ex2_approx(__uint_as_float(sv[e]) - C[e]);
+          if (MASKED) pr = (r >= ra && r < rb) ? pr : 0.f;
+          vsum += pr;
+          // source lane (e - L) mod 32: the shuffle takes the index mod 32
+          const float v = __shfl_sync(0xffffffffu, pr, e - lane);
+          if (lane <= e) a1 += v; else a0 += v;
         }
       };
       // one version per case, so no branch sits between the rows
@@ -460,14 +424,12 @@ __global__ void __launch_bounds__(THREADS, 1)
         rows(std::false_type{});
       else
         rows(std::true_type{});
-      if (PASS == 2) {
-        atomicAdd(&vbin[j - ka], vsum);  // the two row halves of key j
-        // bin of diagonal d: offset i - j minus the slice's smallest offset,
-        // (ka + SLICE - 1 - j_t) + r = (ka + SLICE - 1 - j_0) + d
-        float* bw = sbin + (ka + SLICE - 1 - (static_cast<int64_t>(it.kt) * BN + kq * 32)) + r0;
-        if (lane > 0) atomicAdd(&bw[lane - 32], a0);
-        atomicAdd(&bw[lane], a1);
-      }
+      atomicAdd(&vbin[j - ka], vsum);  // the two row halves of key j
+      // bin of diagonal d: offset i - j minus the slice's smallest offset,
+      // (ka + SLICE - 1 - j_t) + r = (ka + SLICE - 1 - j_0) + d
+      float* bw = sbin + (ka + SLICE - 1 - (static_cast<int64_t>(it.kt) * BN + kq * 32)) + r0;
+      if (lane > 0) atomicAdd(&bw[lane - 32], a0);
+      atomicAdd(&bw[lane], a1);
 
       // continuous: the last item of chunk c frees its operand buffer for c + 2
       if (p.continuous) {
@@ -486,35 +448,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
 
     // ---- per-CTA results (every softmax warp runs this, whatever happened)
-    if (PASS == 1) {
-      // per row over the 128 keys: 4 rounds of 8 rows of each half; 16
-      // threads per row each merge 8 entries, then a 16-lane shuffle merge
-      float* mb = bins;
-      float* lb = bins + MROWS * MSTRIDE;
-      const int rr = stid >> 4, q = stid & 15;
-#pragma unroll
-      for (int round = 0; round < 4; ++round) {
-        if (round > 0) softmax_bar();  // the previous round's reads are done
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          mb[((r0 >> 2) + e) * MSTRIDE + tau] = m[round * 8 + e];
-          lb[((r0 >> 2) + e) * MSTRIDE + tau] = l[round * 8 + e];
-        }
-        softmax_bar();
-        float2 acc = make_float2(NEG_BIG, 0.f);
-#pragma unroll
-        for (int e = 0; e < 8; ++e)
-          acc = merge_stat(acc, make_float2(mb[rr * MSTRIDE + q + 16 * e], lb[rr * MSTRIDE + q + 16 * e]));
-#pragma unroll
-        for (int off = 1; off < 16; off <<= 1)
-          acc = merge_stat(acc, make_float2(__shfl_xor_sync(0xffffffffu, acc.x, off),
-                                            __shfl_xor_sync(0xffffffffu, acc.y, off)));
-        if (q == 0) {
-          const int row = (rr >> 3) * 32 + round * 8 + (rr & 7);
-          p.part[(static_cast<int64_t>(h) * p.n_slices + sl) * ROWS + row] = acc;
-        }
-      }
-    } else {
+    {
       softmax_bar();  // every bin update is done
       float* vrow = p.vert + static_cast<int64_t>(h) * p.Lk;
       float* srow = p.slash + static_cast<int64_t>(h) * p.Lk;
@@ -959,26 +893,21 @@ __global__ void __launch_bounds__(R_THREADS, 1)
 
 int select_slices(int64_t Lk) { return static_cast<int>((Lk + selm::SLICE - 1) / selm::SLICE); }
 
-#ifndef DCA_SEL_ROWS
-#define DCA_SEL_ROWS 1
-#endif
 int select_stat_slices(int64_t Lk) {
-  return DCA_SEL_ROWS ? static_cast<int>((Lk + selm::R_SLICE - 1) / selm::R_SLICE)
-                      : select_slices(Lk);
+  return static_cast<int>((Lk + selm::R_SLICE - 1) / selm::R_SLICE);
 }
 
-cudaError_t launch_select_scores(const void* kr, const float* qv, const float2* crot, float2* part,
-                                 const float2* stats, float* vert, float* slash, int64_t i_first,
-                                 int64_t Lk, int64_t s, int64_t w, int n_last, int Hq, int Hkv,
-                                 int reading, int continuous, int pass, unsigned int* status,
-                                 unsigned long long timeout_ns, cudaStream_t st) {
+cudaError_t launch_select_sums(const void* kr, const float* qv, const float2* crot,
+                               const float2* stats, float* vert, float* slash, int64_t i_first,
+                               int64_t Lk, int64_t s, int64_t w, int n_last, int Hq, int Hkv,
+                               int reading, int continuous, unsigned int* status,
+                               unsigned long long timeout_ns, cudaStream_t st) {
   using namespace selm;
   CUtensorMap tm_k;
   if (!encode_kv_map(&tm_k, kr, Lk, Hkv)) return cudaErrorInvalidValue;
   Params p;
   p.qv = qv;
   p.crot = crot;
-  p.part = part;
   p.stats = stats;
   p.vert = vert;
   p.slash = slash;
@@ -997,11 +926,10 @@ cudaError_t launch_select_scores(const void* kr, const float* qv, const float2* 
   p.timeout_ns = timeout_ns;
   const int64_t blocks = static_cast<int64_t>(p.n_slices) * Hq;
   if (blocks > 0x7fffffffLL) return cudaErrorInvalidValue;
-  auto kern = pass == 1 ? sel_mma_kernel<1> : sel_mma_kernel<2>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  cudaError_t e = cudaFuncSetAttribute(sel_sums_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(SMEM_BYTES));
   if (e != cudaSuccess) return e;
-  kern<<<static_cast<unsigned>(blocks), THREADS, SMEM_BYTES, st>>>(tm_k, p);
+  sel_sums_kernel<<<static_cast<unsigned>(blocks), THREADS, SMEM_BYTES, st>>>(tm_k, p);
   return cudaGetLastError();
 }
 
@@ -1010,9 +938,6 @@ cudaError_t launch_select_row_stats(const void* kr, const float* qv, const float
                                     int n_last, int Hq, int Hkv, int reading, int continuous,
                                     unsigned int* status, unsigned long long timeout_ns,
                                     cudaStream_t st) {
-  if (!DCA_SEL_ROWS)
-    return launch_select_scores(kr, qv, crot, part, nullptr, nullptr, nullptr, i_first, Lk, s, w,
-                                n_last, Hq, Hkv, reading, continuous, 1, status, timeout_ns, st);
   using namespace selm;
   CUtensorMap tm_k;
   if (!encode_kv_map(&tm_k, kr, Lk, Hkv)) return cudaErrorInvalidValue;
